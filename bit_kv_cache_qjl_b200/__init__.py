@@ -1,0 +1,178 @@
+"""B200 (sm_100a) QJL / FQJL 1-bit key sketches for the KV cache.
+
+A thin Python binding over the C ABI in include/qjl.h. It marshals torch
+tensors into device pointers and the current CUDA stream and raises on error
+statuses. Every step of the hot path runs in the library's CUDA kernels, and
+nothing here computes. PyTorch provides device memory and streams only.
+
+Methods (web pages, cited by title and section):
+  * QJL abstract (Zandieh, Daliri, Han) on the "Majid Daliri" author page:
+    the sign-bit key sketch plus ||k||, and the asymmetric estimator with an
+    unquantised JL-projected query.
+  * "Fast Quantized Johnson - Lindenstrauss Transforms": D-FQJL and P-FQJL,
+    two randomized Hadamard transforms with a Gaussian second diagonal.
+  * KIVI abstract on the "Vladimir Braverman" author page: 2-bit per-token
+    values, and the decode step that reads the whole cache per token.
+"""
+
+import ctypes
+
+import torch
+
+from ._lib import Options, lib
+
+__all__ = ["Projection", "QJLError", "quantize_keys", "project_queries", "scores",
+           "quantize_values_2bit", "decode_attention", "decode_workspace_bytes", "lib", "KINDS"]
+
+KINDS = {"dense": 0, "dfqjl": 1, "pfqjl": 2}
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+_EXPORT = {"S": 0, "D_r": 1, "perm": 2, "D_g": 3}
+
+
+class QJLError(RuntimeError):
+    def __init__(self, status, where):
+        L = lib()
+        self.status = status
+        msg = L.qjl_last_error_message().decode()
+        super().__init__("%s: %s (%s)" % (where, L.qjl_status_string(status).decode(), msg))
+
+
+def _check(status, where):
+    if status != 0:
+        raise QJLError(status, where)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cuda(t, name):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda):
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+class Projection:
+    """A drawn random map (dense S, D-FQJL or P-FQJL) resident on the current device."""
+
+    def __init__(self, seed, d, m, kind="dense", dither_sigma_rel=0.5, dg_outer=False, s_bf16=True):
+        L = lib()
+        opt = Options(float(dither_sigma_rel), int(bool(dg_outer)), int(bool(s_bf16)))
+        h = ctypes.c_void_p()
+        _check(L.qjl_make_projection(int(seed), int(d), int(m), KINDS[kind], ctypes.byref(opt), ctypes.byref(h)),
+               "qjl_make_projection")
+        self._h = h
+        self.seed, self.d, self.m, self.kind = int(seed), int(d), int(m), kind
+        self.dither_sigma_rel, self.dg_outer, self.s_bf16 = float(dither_sigma_rel), bool(dg_outer), bool(s_bf16)
+        es = ctypes.c_float()
+        _check(L.qjl_projection_info(h, None, None, None, ctypes.byref(es)), "qjl_projection_info")
+        self.est_scale = es.value
+
+    @property
+    def handle(self):
+        return self._h
+
+    def export(self, what):
+        """Copy a parameter array to a host torch tensor ('S', 'D_r', 'perm', 'D_g')."""
+        nb = self.m // self.d
+        shape = (self.m, self.d) if what == "S" else (nb, self.d)
+        out = torch.empty(shape, dtype=torch.int32 if what == "perm" else torch.float32)
+        _check(lib().qjl_projection_export(self._h, _EXPORT[what], _ptr(out), out.numel() * 4),
+               "qjl_projection_export")
+        return out
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib().qjl_destroy_projection(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def quantize_keys(proj, keys, first_token=0, bits=None, norms=None, stream=None):
+    """keys [n, d] (fp32 or bf16, CUDA) -> (bits [n, m/32] int32 words, norms [n] fp32)."""
+    _cuda(keys, "keys")
+    n, d = keys.shape
+    if d != proj.d:
+        raise ValueError("keys have d=%d, projection has d=%d" % (d, proj.d))
+    if bits is None:
+        bits = torch.empty((n, proj.m // 32), dtype=torch.int32, device=keys.device)
+    if norms is None:
+        norms = torch.empty((n,), dtype=torch.float32, device=keys.device)
+    _check(lib().qjl_quantize_keys(proj.handle, _ptr(keys), _DTYPES[keys.dtype], n, keys.stride(0),
+                                   int(first_token), _ptr(bits), _ptr(norms), _stream(stream)), "qjl_quantize_keys")
+    return bits, norms
+
+
+def project_queries(proj, q, out=None, stream=None):
+    """q [nq, d] fp32 -> S_eff q [nq, m] fp32 (no quantisation)."""
+    _cuda(q, "q")
+    nq = q.shape[0]
+    if out is None:
+        out = torch.empty((nq, proj.m), dtype=torch.float32, device=q.device)
+    _check(lib().qjl_project_queries(proj.handle, _ptr(q), nq, q.stride(0), _ptr(out), _stream(stream)),
+           "qjl_project_queries")
+    return out
+
+
+def scores(proj, bits, norms, sq, out=None, stream=None):
+    """bits [G, N, m/32], norms [G, N], sq [G, J, m] -> estimates [G, J, N] fp32."""
+    for t, nm in ((bits, "bits"), (norms, "norms"), (sq, "sq")):
+        _cuda(t, nm)
+    G, N = norms.shape
+    J = sq.shape[1]
+    if out is None:
+        out = torch.empty((G, J, N), dtype=torch.float32, device=norms.device)
+    _check(lib().qjl_scores(proj.handle, _ptr(bits), _ptr(norms), G, N, _ptr(sq), J, _ptr(out), _stream(stream)),
+           "qjl_scores")
+    return out
+
+
+def quantize_values_2bit(v, codes=None, scale=None, zero=None, stream=None):
+    """v [n, d] (fp32 or bf16) -> (codes [n, d/16] int32, scale [n, d/32] fp16, zero [n, d/32] fp16)."""
+    _cuda(v, "v")
+    n, d = v.shape
+    if codes is None:
+        codes = torch.empty((n, d // 16), dtype=torch.int32, device=v.device)
+    if scale is None:
+        scale = torch.empty((n, d // 32), dtype=torch.float16, device=v.device)
+    if zero is None:
+        zero = torch.empty((n, d // 32), dtype=torch.float16, device=v.device)
+    _check(lib().qjl_quantize_values_2bit(_ptr(v), _DTYPES[v.dtype], n, d, _ptr(codes), _ptr(scale), _ptr(zero),
+                                          _stream(stream)), "qjl_quantize_values_2bit")
+    return codes, scale, zero
+
+
+def decode_workspace_bytes(groups, q_per_group, N, d):
+    return int(lib().qjl_decode_workspace_bytes(groups, q_per_group, N, d))
+
+
+def decode_attention(proj, bits, norms, codes, scale, zero, sq, softmax_scale, out=None, workspace=None,
+                     stream=None):
+    """Fused softmax(est * softmax_scale) . V_hat -> out [G, J, d] fp32."""
+    for t, nm in ((bits, "bits"), (norms, "norms"), (codes, "codes"), (scale, "scale"), (zero, "zero"),
+                  (sq, "sq")):
+        _cuda(t, nm)
+    G, N = norms.shape
+    J = sq.shape[1]
+    d = proj.d
+    if out is None:
+        out = torch.empty((G, J, d), dtype=torch.float32, device=norms.device)
+    need = decode_workspace_bytes(G, J, N, d)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=norms.device)
+    _check(lib().qjl_decode_attention(proj.handle, _ptr(bits), _ptr(norms), _ptr(codes), _ptr(scale), _ptr(zero),
+                                      G, N, _ptr(sq), J, float(softmax_scale), _ptr(out), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)),
+           "qjl_decode_attention")
+    return out

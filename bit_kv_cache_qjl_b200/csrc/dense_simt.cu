@@ -1,0 +1,93 @@
+// Dense JL projection on the fp32 SIMT pipe (QJL abstract: "a JL transform
+// followed by sign-bit quantization"; the query side is the same transform
+// without quantisation).
+//
+// One warp per row (key or query). Lane l owns output coordinates
+// c0 + 32 r + l, so __ballot_sync over the lanes yields packed sign word
+// (c0/32 + r) directly (bit = 1 iff y >= 0). S_eff^T is read from global
+// memory in coalesced 128-byte rows; every warp reads the same matrix, so it
+// stays in L1/L2. This path serves fp32 keys, fp32 S_eff and every query
+// projection. bf16 keys with bf16 S_eff go to the tcgen05 kernel.
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qjl_internal.h"
+
+namespace {
+
+constexpr int kRowsPerPass = 8;  // 8 x 32 = 256 output coordinates per pass
+
+template <int DTYPE>
+__device__ __forceinline__ float load_elem(const void* base, int64_t idx) {
+  if (DTYPE == QJL_F32) return __ldg(reinterpret_cast<const float*>(base) + idx);
+  const unsigned short b = __ldg(reinterpret_cast<const unsigned short*>(base) + idx);
+  return __uint_as_float((uint32_t)b << 16);
+}
+
+template <int DTYPE>
+__global__ void __launch_bounds__(256) dense_simt_kernel(const void* __restrict__ x, int64_t rows,
+                                                         int64_t ld, int d, int m,
+                                                         const float* __restrict__ St,
+                                                         uint32_t* __restrict__ bits,
+                                                         float* __restrict__ norms,
+                                                         float* __restrict__ proj_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int W = m >> 5;
+  for (int64_t row = warp; row < rows; row += nwarps) {
+    const int64_t xoff = row * ld;
+    float sumsq = 0.f;
+    for (int c0 = 0; c0 < m; c0 += 32 * kRowsPerPass) {
+      float acc[kRowsPerPass];
+#pragma unroll
+      for (int r = 0; r < kRowsPerPass; ++r) acc[r] = 0.f;
+      for (int j0 = 0; j0 < d; j0 += 32) {
+        const int j = j0 + lane;
+        const float xv = (j < d) ? load_elem<DTYPE>(x, xoff + j) : 0.f;
+        if (c0 == 0) sumsq = fmaf(xv, xv, sumsq);
+        const int jn = min(32, d - j0);
+        for (int jj = 0; jj < jn; ++jj) {
+          const float xj = __shfl_sync(0xffffffffu, xv, jj);
+          const float* srow = St + (int64_t)(j0 + jj) * m + c0 + lane;
+#pragma unroll
+          for (int r = 0; r < kRowsPerPass; ++r)
+            if (c0 + 32 * r < m) acc[r] = fmaf(__ldg(srow + 32 * r), xj, acc[r]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kRowsPerPass; ++r) {
+        const int c = c0 + 32 * r;
+        if (c >= m) break;
+        if (bits) {
+          const uint32_t word = __ballot_sync(0xffffffffu, acc[r] >= 0.f);
+          if (lane == 0) bits[row * W + (c >> 5)] = word;
+        }
+        if (proj_out) proj_out[row * (int64_t)m + c + lane] = acc[r];
+      }
+    }
+    if (norms) {
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
+      if (lane == 0) norms[row] = sqrtf(sumsq);
+    }
+  }
+}
+
+}  // namespace
+
+qjl_status launch_dense_simt(const qjl_projection* P, const void* x, int dtype, int64_t n, int64_t ld,
+                             uint32_t* bits, float* norms, float* proj_out, cudaStream_t st) {
+  const int threads = 256;
+  const int64_t want = (n + 7) / 8;
+  const int blocks = (int)std::min<int64_t>(want, (int64_t)qjl_num_sms(P->device) * 16);
+  if (dtype == QJL_F32)
+    dense_simt_kernel<QJL_F32><<<blocks, threads, 0, st>>>(x, n, ld, P->d, P->m, P->St_f32, bits,
+                                                           norms, proj_out);
+  else
+    dense_simt_kernel<QJL_BF16><<<blocks, threads, 0, st>>>(x, n, ld, P->d, P->m, P->St_f32, bits,
+                                                            norms, proj_out);
+  return qjl_check_launch("dense_simt_kernel");
+}

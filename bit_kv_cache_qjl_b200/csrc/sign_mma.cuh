@@ -1,0 +1,141 @@
+// Sign-bit dot products on the s8 tensor-core path (mma.sync m16n8k32).
+//
+// Shared by the score kernel and the fused decode kernel. The scheme is
+// described at the top of scores.cu: 16-bit fixed-point Sq split into int8
+// hi/lo columns, and sign bits fed as u8 A fragments of value 2^J, one AND
+// per 4 bits. A 16-key tile needs W MMAs per column tile of 4 queries.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qjl_sign {
+
+constexpr int kQmax = 32639;  // 127 * 256 + 127: both int8 halves stay in range
+
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ int quant16(float v, float inv) {
+  const float q = rintf(v * inv);
+  return (int)fminf(fmaxf(q, (float)-kQmax), (float)kQmax);
+}
+
+// Fills per-query scale data and the B fragments for group `gi`.
+// Btab[(pt * W + mu) * 32 + lane] = (b0, b1) for column tile pt and MMA index
+// mu = 8 p + j. The entries need W % 8 == 0.
+template <int W>
+__device__ void build_tables(const float* __restrict__ sqg, int J, int NT, float est_scale,
+                             float* s_inv, float* s_mul, int* s_qsum, uint2* Btab, int nwarps) {
+  constexpr int m = 32 * W;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int j = warp; j < J; j += nwarps) {
+    const float* row = sqg + (int64_t)j * m;
+    float mx = 0.f;
+    for (int i = lane; i < m; i += 32) mx = fmaxf(mx, fabsf(row[i]));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float inv = mx > 0.f ? (float)kQmax / mx : 0.f;
+    int qs = 0;
+    for (int i = lane; i < m; i += 32) qs += quant16(row[i], inv);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+    if (lane == 0) {
+      s_inv[j] = inv;
+      s_mul[j] = est_scale * (mx > 0.f ? mx / (float)kQmax : 0.f);
+      s_qsum[j] = qs;
+    }
+  }
+  __syncthreads();
+  const int entries = NT * W * 32;
+  for (int idx = threadIdx.x; idx < entries; idx += blockDim.x) {
+    const int ln = idx & 31;
+    const int mu = (idx >> 5) % W;
+    const int pt = (idx >> 5) / W;
+    const int n = ln >> 2, qq = ln & 3;
+    const int jq = pt * 4 + (n >> 1);
+    const int half = n & 1;  // 0: hi byte, 1: lo byte
+    const int p = mu >> 3, jb = mu & 7;
+    uint32_t b[2] = {0u, 0u};
+    if (jq < J) {
+      const float* row = sqg + (int64_t)jq * m;
+      const float inv = s_inv[jq];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int word = qq * (W / 4) + 2 * p + r;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int Q = quant16(row[32 * word + 8 * e + jb], inv);
+          const int lo = (int)(int8_t)(Q & 0xFF);
+          const int hi = (Q - lo) >> 8;
+          b[r] |= ((uint32_t)(half ? lo : hi) & 0xFFu) << (8 * e);
+        }
+      }
+    }
+    Btab[idx] = make_uint2(b[0], b[1]);
+  }
+  __syncthreads();
+}
+
+template <int W>
+__device__ __forceinline__ void load_words(const uint32_t* __restrict__ base, int64_t row, int64_t N,
+                                           int q, uint32_t (&w)[W / 4]) {
+  if (row < N) {
+    const uint32_t* p = base + row * W + q * (W / 4);
+    if constexpr (W == 8) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+      w[0] = v.x; w[1] = v.y;
+    } else {
+#pragma unroll
+      for (int k = 0; k < W / 16; ++k) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p) + k);
+        w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < W / 4; ++k) w[k] = 0u;
+  }
+}
+
+
+// One column tile (4 queries) over a 16-key tile. Thread (g = lane/4,
+// q = lane%4) receives 64 * sum_i b_i hi_i (hi) and 64 * sum_i b_i lo_i (lo)
+// for query q of the column tile and key rows g (r = 0) and g + 8 (r = 1).
+template <int W>
+__device__ __forceinline__ void tile_sums(const uint32_t (&w0)[W / 4], const uint32_t (&w1)[W / 4],
+                                          const uint2* __restrict__ Btab_pt, int lane, int (&hi)[2],
+                                          int (&lo)[2]) {
+  int acc[4][4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[b][c] = 0;
+#pragma unroll
+  for (int p = 0; p < W / 8; ++p) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const uint32_t x0 = w0[2 * p] >> s, x1 = w1[2 * p] >> s;
+      const uint32_t x2 = w0[2 * p + 1] >> s, x3 = w1[2 * p + 1] >> s;
+#pragma unroll
+      for (int Ji = 0; Ji < 4; ++Ji) {
+        const uint32_t M = 0x01010101u << (2 * Ji);
+        const uint2 bb = Btab_pt[(8 * p + 2 * Ji + s) * 32 + lane];
+        mma_u8s8(acc[Ji], x0 & M, x1 & M, x2 & M, x3 & M, bb.x, bb.y);
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    hi[r] = ((acc[0][2 * r] * 4 + acc[1][2 * r]) * 4 + acc[2][2 * r]) * 4 + acc[3][2 * r];
+    lo[r] = ((acc[0][2 * r + 1] * 4 + acc[1][2 * r + 1]) * 4 + acc[2][2 * r + 1]) * 4 + acc[3][2 * r + 1];
+  }
+}
+
+}  // namespace qjl_sign

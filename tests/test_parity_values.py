@@ -1,0 +1,38 @@
+"""2-bit per-token value quantisation on the GPU vs the oracle: bit-exact.
+
+Both sides take the code decision in fp32 with the same IEEE operations, so
+codes, scales and zeros must match exactly.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_kv_cache_qjl_b200 import quantize_values_2bit
+from bit_kv_cache_qjl_b200 import workloads as wl
+from helpers import host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("n,d,dtype", [(1000, 128, torch.bfloat16), (33, 32, torch.bfloat16),
+                                       (17, 256, torch.float32), (5, 96, torch.bfloat16), (1, 224, torch.float32)])
+def test_values_bit_exact(cuda_ok, n, d, dtype):
+    v = wl.normal((n, d), 600 + n, "cuda", dtype)
+    codes, scale, zero = quantize_values_2bit(v)
+    torch.cuda.synchronize()
+    oc, os_, oz = oracle.kivi.quantize_values_2bit(host(v).astype(np.float32))
+    assert np.array_equal(host(codes), oc)
+    assert np.array_equal(scale.cpu().numpy().view(np.uint16), os_.view(np.uint16))
+    assert np.array_equal(zero.cpu().numpy().view(np.uint16), oz.view(np.uint16))
+
+
+def test_values_constant_groups(cuda_ok):
+    v = torch.zeros((3, 64), dtype=torch.bfloat16, device="cuda")
+    v[1] = 2.5
+    v[2, :32] = -1.0
+    codes, scale, zero = quantize_values_2bit(v)
+    torch.cuda.synchronize()
+    assert torch.all(codes == 0) and torch.all(scale == 0)
+    assert torch.equal(zero.float().cpu(), torch.tensor([[0, 0], [2.5, 2.5], [-1.0, 0.0]]))
