@@ -1,0 +1,399 @@
+"""Throughput of the QJL key-quantize + decode-score hot path on B200.
+
+One step is a whole pass of the path over one batch of the Llama-2-7B-shaped
+decode workload: B=8, 32 heads, N=32768 cached keys per head, d=128,
+m=256, dense bf16 S. The step:
+  (1) sketches every key (tcgen05 kernel): bits + ||k||;
+  (2) projects one query per head (unquantised JL map);
+  (3) scores every cached key against its head's query (estimator).
+`value` is cached keys processed per second over whole steps, with inputs
+already resident in HBM. The 2.1 GB keys exceed the 126 MB L2, so no flush
+is needed. `e2e` is the same metric through the same C-ABI calls with host
+buffers: each step copies the keys and queries in from pinned host memory and
+copies the scores back.
+
+Multi-GPU (torchrun): the (batch, head) groups are independent, so every
+rank processes its own copy of the workload (weak scaling). No collective
+touches the data path. Ranks meet at a barrier around the timed region, and
+the time is the max over ranks.
+
+--impl reference times the CPU oracle on a bounded sample of the same
+workload (the reference arm). It runs on rank 0 only.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QJL decode scores keys/s (HBM GB/s vs ~8 TB/s); key-quantize vectors/s"
+WORKLOAD = "decode_llama7b"
+B, H, N, D, M = 8, 32, 32768, 128, 256
+KEYS = B * H * N
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# algorithmic bytes per key for each kernel of the step
+BYTES_QUANT = D * 2 + M // 8 + 4          # bf16 key in, bits + norm out = 292
+BYTES_SCORE = M // 8 + 4 + 4              # bits + norm in, score out = 40
+FLOP_QUANT = 2 * D * M                    # bf16 contraction per key
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload, src):
+    """Per-launch DRAM bytes from profiles/traffic.txt, valid only for the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    h = source_hash(os.path.join(ROOT, "bit_kv_cache_qjl_b200", "csrc", src))
+    for line in open(p):
+        f = line.split()
+        if len(f) >= 4 and not line.startswith("#") and f[0] == kernel and f[1] == workload and f[3] == h:
+            return float(f[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_oracle_rate(sample_keys, seconds_hint=None):
+    """Time the oracle (as it stands) on `sample_keys` keys of the workload: keys/s, threads."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    import oracle
+    from bit_kv_cache_qjl_b200 import workloads as wl
+    O = oracle.params.make_projection(2, D, M, oracle.params.KIND_DENSE, s_bf16=True)
+    heads = max(1, sample_keys // N)
+    per = min(N, sample_keys)
+    keys = wl.llama_keys("cpu", B=1, H=heads, N=per).reshape(heads, per, D).to("cpu").float().numpy()
+    q = wl.llama_queries("cpu", B=1, H=heads).reshape(heads, D).numpy()
+    t0 = time.perf_counter()
+    for h in range(heads):
+        words, norms, _ = oracle.qjl.quantize_keys(O, keys[h].astype(np.float64))
+        sq = oracle.qjl.project_queries(O, q[h:h + 1].astype(np.float64))
+        oracle.qjl.scores(O, words[None], norms[None], sq[None])
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return heads * per / dt, dt, threads, heads * per
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    sample = args.ref_sample
+    for _ in range(args.warmup):
+        cpu_oracle_rate(sample)
+    total_keys, total_t = 0, 0.0
+    threads = 1
+    for _ in range(args.steps):
+        rate, dt, threads, k = cpu_oracle_rate(sample)
+        total_keys += k
+        total_t += dt
+    value = total_keys / total_t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD + " (CPU oracle sample)", "sample_keys": sample,
+                                            "B": B, "H": H, "N": N, "d": D, "m": M},
+            "cpu_baseline": {"value": value, "unit": "keys/s", "cores": threads, "kind": "oracle",
+                             "sample": "%d keys (one head slice) per step: oracle quantize + project + score" % sample},
+            "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def profile_case(case, n):
+    """A small case of one kernel for ncu: inputs > L2 (126 MB) but a few GB at most; 2 + 3 launches."""
+    import torch
+    import bit_kv_cache_qjl_b200 as qjl
+    from bit_kv_cache_qjl_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    if case == "quantize":
+        P = qjl.Projection(2, D, M, "dense")
+        keys = wl.llama_keys(dev, B=1, H=max(1, n // N), N=min(N, n), d=D).reshape(-1, D)
+        run = lambda: qjl.quantize_keys(P, keys)
+    elif case in ("fqjl", "fqjl1024"):
+        m = 256 if case == "fqjl" else 1024
+        P = qjl.Projection(4, 256, m, "pfqjl")
+        keys = wl.bulk_keys(dev, n=n, d=256)
+        run = lambda: qjl.quantize_keys(P, keys)
+    elif case == "scores":
+        P = qjl.Projection(2, D, M, "dense")
+        G = max(1, n // N)
+        keys = wl.llama_keys(dev, B=1, H=G, N=N, d=D).reshape(-1, D)
+        bits, norms = qjl.quantize_keys(P, keys)
+        sq = qjl.project_queries(P, wl.llama_queries(dev, B=1, H=G, d=D).reshape(-1, D))
+        run = lambda: qjl.scores(P, bits.view(G, N, M // 32), norms.view(G, N), sq.view(G, 1, M))
+    elif case == "values":
+        v = wl.normal((n, D), 506, dev, torch.bfloat16)
+        run = lambda: qjl.quantize_values_2bit(v)
+    else:
+        P = qjl.Projection(5, D, M, "dfqjl")
+        G = max(1, n // 16384)
+        keys, vals = wl.decode_kv(dev, B=1, H=G, N=16384, d=D)
+        bits, norms = qjl.quantize_keys(P, keys.reshape(-1, D))
+        codes, sc, zr = qjl.quantize_values_2bit(vals.reshape(-1, D))
+        sq = qjl.project_queries(P, wl.decode_queries(dev, B=1, H=G, d=D).reshape(-1, D))
+        run = lambda: qjl.decode_attention(P, bits.view(G, 16384, M // 32), norms.view(G, 16384),
+                                           codes.view(G, 16384, D // 16), sc.view(G, 16384, D // 32),
+                                           zr.view(G, 16384, D // 32), sq.view(G, 1, M), 1 / math.sqrt(D))
+    torch.cuda.synchronize()
+    for _ in range(5):
+        run()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": case, "n": n, "status": "ok"}))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-sample", type=int, default=4096)
+    ap.add_argument("--cpu-sample", type=int, default=1 << 18)
+    ap.add_argument("--profile-case", default=None,
+                    choices=["quantize", "scores", "fqjl", "fqjl1024", "values", "decode"],
+                    help="run one small case of a single kernel (3 launches after 2 warm-ups) for ncu")
+    ap.add_argument("--profile-keys", type=int, default=1 << 20)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.profile_case:
+        return profile_case(args.profile_case, args.profile_keys)
+
+    import torch
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import bit_kv_cache_qjl_b200 as qjl
+    from bit_kv_cache_qjl_b200 import workloads as wl
+
+    P = qjl.Projection(2, D, M, "dense", s_bf16=True)
+    keys = wl.llama_keys(dev, B=B, H=H, N=N, d=D).reshape(-1, D)
+    queries = wl.llama_queries(dev, B=B, H=H, d=D).reshape(-1, D)
+    bits = torch.empty((KEYS, M // 32), dtype=torch.int32, device=dev)
+    norms = torch.empty((KEYS,), dtype=torch.float32, device=dev)
+    sq = torch.empty((B * H, M), dtype=torch.float32, device=dev)
+    out = torch.empty((B * H, 1, N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        qjl.quantize_keys(P, keys, bits=bits, norms=norms)
+        if ev is not None:
+            ev[1].record(stream)
+        qjl.project_queries(P, queries, out=sq)
+        if ev is not None:
+            ev[2].record(stream)
+        qjl.scores(P, bits.view(B * H, N, M // 32), norms.view(B * H, N), sq.view(B * H, 1, M), out=out)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), world)
+    ms_step = ms_total / args.steps
+    k_quant = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    k_proj = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    k_score = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    value = world * KEYS / (ms_step * 1e-3)
+
+    # end to end through the same calls with host buffers (pinned), copies inside the timed region
+    h_keys = torch.empty((KEYS, D), dtype=torch.bfloat16, pin_memory=True)
+    h_keys.copy_(keys)
+    h_q = torch.empty((B * H, D), dtype=torch.float32, pin_memory=True)
+    h_q.copy_(queries)
+    h_out = torch.empty((B * H, 1, N), dtype=torch.float32, pin_memory=True)
+    torch.cuda.synchronize()
+
+    def e2e_step():
+        keys.copy_(h_keys, non_blocking=True)
+        queries.copy_(h_q, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
+    h2d = h_keys.numel() * 2 + h_q.numel() * 4
+    d2h = h_out.numel() * 4
+
+    pk, pk_kind = peaks()
+    hbm = pk["hbm_gbs"]
+    tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    q_gbs = KEYS * BYTES_QUANT / (k_quant * 1e-3) / 1e9
+    s_gbs = KEYS * BYTES_SCORE / (k_score * 1e-3) / 1e9
+    q_tflops = KEYS * FLOP_QUANT / (k_quant * 1e-3) / 1e12
+    traffic = ncu_traffic("dense_tc_kernel", WORKLOAD, "dense_tc.cu")
+    clocks = clk.summary()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rate, dt, threads, k = cpu_oracle_rate(args.cpu_sample)
+        cpu = {"value": rate, "unit": "keys/s", "cores": threads, "kind": "oracle",
+               "sample": "%d keys of the workload (%d head slices of %d keys): oracle quantize + project + "
+                         "score, %.1f s" % (k, max(1, k // N), min(N, k), dt)}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "%s: B=%d, heads=%d, N=%d, d=%d, m=%d dense bf16 S; quantize all keys, project "
+                               "1 query/head, score all keys" % (WORKLOAD, B, H, N, D, M),
+                   "keys_per_step": KEYS * world, "l2": "inputs larger than L2 (2.15 GB keys/step), no flush",
+                   "parallelism": "replicas (weak)" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "kernel": "dense_tc_kernel (key quantize)", "achieved": q_gbs,
+                     "peak": hbm, "unit": "GB/s", "frac": q_gbs / hbm, "peak_kind": pk_kind,
+                     "traffic": traffic,
+                     "bytes_per_launch": KEYS * BYTES_QUANT, "tensor_tflops": q_tflops,
+                     "tensor_frac_of_sustained": q_tflops / tf},
+        "kernels": {
+            "quantize_keys": {"ms": k_quant, "vectors_per_s": KEYS / (k_quant * 1e-3), "gbs": q_gbs,
+                              "frac_hbm_measured": q_gbs / hbm, "frac_8tbs": q_gbs / 8000.0},
+            "project_queries": {"ms": k_proj},
+            "scores": {"ms": k_score, "keys_per_s": KEYS / (k_score * 1e-3), "gbs": s_gbs,
+                       "frac_hbm_measured": s_gbs / hbm, "frac_8tbs": s_gbs / 8000.0},
+        },
+        "e2e": {"value": world * KEYS / (e2e_ms * 1e-3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

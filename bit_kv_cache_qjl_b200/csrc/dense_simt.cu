@@ -76,7 +76,44 @@ __global__ void __launch_bounds__(256) dense_simt_kernel(const void* __restrict_
   }
 }
 
+// Query projection Sq = S_eff q: one CTA per query, q staged in shared memory.
+// Thread i owns coordinates i, i + 256, ... Its column of S_eff^T is read with
+// consecutive threads on consecutive addresses, using four partial sums for ILP.
+__global__ void __launch_bounds__(256) project_dense_kernel(const float* __restrict__ q, int64_t ld, int d, int m,
+                                                           const float* __restrict__ St,
+                                                           float* __restrict__ out) {
+  extern __shared__ float qs[];
+  const int64_t row = blockIdx.x;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) qs[j] = __ldg(q + row * ld + j);
+  __syncthreads();
+  for (int i = threadIdx.x; i < m; i += blockDim.x) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int j = 0;
+    for (; j + 4 <= d; j += 4) {
+      a0 = fmaf(__ldg(St + (int64_t)(j + 0) * m + i), qs[j + 0], a0);
+      a1 = fmaf(__ldg(St + (int64_t)(j + 1) * m + i), qs[j + 1], a1);
+      a2 = fmaf(__ldg(St + (int64_t)(j + 2) * m + i), qs[j + 2], a2);
+      a3 = fmaf(__ldg(St + (int64_t)(j + 3) * m + i), qs[j + 3], a3);
+    }
+    for (; j < d; ++j) a0 = fmaf(__ldg(St + (int64_t)j * m + i), qs[j], a0);
+    out[row * (int64_t)m + i] = (a0 + a1) + (a2 + a3);
+  }
+}
+
 }  // namespace
+
+qjl_status launch_project_dense(const qjl_projection* P, const float* q, int64_t nq, int64_t ld, float* out,
+                                cudaStream_t st) {
+  const size_t smem = (size_t)P->d * sizeof(float);
+  for (int64_t r0 = 0; r0 < nq; r0 += 65535) {
+    const int64_t cnt = std::min<int64_t>(65535, nq - r0);
+    project_dense_kernel<<<(unsigned)cnt, 256, smem, st>>>(q + r0 * ld, ld, P->d, P->m, P->St_f32,
+                                                           out + r0 * (int64_t)P->m);
+    qjl_status s = qjl_check_launch("project_dense_kernel");
+    if (s != QJL_OK) return s;
+  }
+  return QJL_OK;
+}
 
 qjl_status launch_dense_simt(const qjl_projection* P, const void* x, int dtype, int64_t n, int64_t ld,
                              uint32_t* bits, float* norms, float* proj_out, cudaStream_t st) {

@@ -149,12 +149,41 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// 32 fp32 accumulators -> sign word (bit i = 1 iff value i >= 0 as a sign bit).
-__device__ __forceinline__ uint32_t sign_word(const uint32_t (&r)[32]) {
-  uint32_t w = 0;
+// Two back-to-back 32-column TMEM loads (64 columns of this thread's row), one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr + 32u));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 64 fp32 accumulators -> 2 sign words (bit i of word k = 1 iff value 32k+i >= 0
+// as a sign bit). Eight independent 8-step funnel-shift chains keep the
+// dependency depth at 8 instead of 32.
+__device__ __forceinline__ void sign_words2(const uint32_t (&r)[64], uint32_t& w0, uint32_t& w1) {
+  uint32_t c[8];
 #pragma unroll
-  for (int i = 31; i >= 0; --i) w = __funnelshift_l(r[i], w, 1);
-  return ~w;
+  for (int k = 0; k < 8; ++k) c[k] = 0u;
+#pragma unroll
+  for (int i = 7; i >= 0; --i) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) c[k] = __funnelshift_l(r[8 * k + i], c[k], 1);
+  }
+  w0 = ~(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24));
+  w1 = ~(c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
 }
 
 __device__ __forceinline__ void flag_error(int* err, int code) { atomicOr(err, code); }
@@ -218,34 +247,39 @@ __global__ void __launch_bounds__(kThreads, 1) dense_tc_kernel(const __grid_cons
         for (int rb = 0; rb < sblocks; ++rb)
           tma_load_2d(sS + ((size_t)a * m + rb * 256) * 128, &tmS, sbar, a * 64, rb * 256);
       int64_t issued = 0;
-      bool ok = true;
-      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++issued) {
-        const int s = (int)(issued % NS);
-        const uint32_t ph = (uint32_t)((issued / NS) & 1);
-        if (!mbar_wait(&empty[s], ph ^ 1u)) { flag_error(prm.err, 1); ok = false; break; }
+      int s = 0;
+      uint32_t ph = 0;
+      for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++issued) {
+        if (!mbar_wait(&empty[s], ph ^ 1u)) { flag_error(prm.err, 1); break; }
         mbar_expect_tx(&full[s], kStageBytes);
         unsigned char* dst = sK + (size_t)s * kStageBytes;
         for (int a = 0; a < KA; ++a) tma_load_2d(dst + a * BM * 128, &tmK, &full[s], a * 64, (int)(t * BM));
+        if (++s == NS) { s = 0; ph ^= 1u; }
       }
-      // drain: the most recent phase of every stage must have landed before exit
-      const int64_t last = issued < NS ? issued : NS;
-      for (int64_t k = issued - last; k < issued; ++k)
-        if (!mbar_wait(&full[k % NS], (uint32_t)((k / NS) & 1))) flag_error(prm.err, 2);
+      // drain: the most recent phase of every used stage must have landed before exit
+      const int used = issued < NS ? (int)issued : NS;
+      for (int j = 0; j < used; ++j) {
+        int st = s - 1 - j;
+        uint32_t p = ph;
+        if (st < 0) { st += NS; p ^= 1u; }
+        if (!mbar_wait(&full[st], p)) flag_error(prm.err, 2);
+      }
       if (!mbar_wait(sbar, 0)) flag_error(prm.err, 2);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       bool ok = mbar_wait(sbar, 0);
       if (!ok) flag_error(prm.err, 4);
-      int64_t i = 0, u = 0;
-      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++i) {
-        const int s = (int)(i % NS);
-        if (!mbar_wait(&full[s], (uint32_t)((i / NS) & 1))) { flag_error(prm.err, 4); ok = false; break; }
+      uint32_t u = 0;
+      int s = 0;
+      uint32_t ph = 0;
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&full[s], ph)) { flag_error(prm.err, 4); ok = false; break; }
         tc_fence_after();
         const uint32_t a_base = smem_u32(sK + (size_t)s * kStageBytes);
         for (int c = 0; c < nchunk && ok; ++c, ++u) {
-          const int buf = (int)(u & 1);
-          if (!mbar_wait(&tempty[buf], (uint32_t)(((u >> 1) & 1) ^ 1))) { flag_error(prm.err, 4); ok = false; break; }
+          const int buf = (int)(u & 1u);
+          if (!mbar_wait(&tempty[buf], ((u >> 1) & 1u) ^ 1u)) { flag_error(prm.err, 4); ok = false; break; }
           tc_fence_after();
           const int N = min(256, m - 256 * c);
           const uint32_t idesc = idesc_bf16(N);
@@ -261,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_tc_kernel(const __grid_cons
           mma_commit(&tfull[buf]);
         }
         mma_commit(&empty[s]);
+        if (++s == NS) { s = 0; ph ^= 1u; }
       }
       // every MMA this thread issued has completed before TMEM is released
       mma_commit(dbar);
@@ -271,11 +306,12 @@ __global__ void __launch_bounds__(kThreads, 1) dense_tc_kernel(const __grid_cons
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int W = m >> 5;
-    int64_t i = 0, u = 0;
+    uint32_t u = 0;
+    int s = 0;
+    uint32_t ph = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++i) {
-      const int s = (int)(i % NS);
-      if (!mbar_wait(&full[s], (uint32_t)((i / NS) & 1))) { flag_error(prm.err, 16); ok = false; break; }
+    for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      if (!mbar_wait(&full[s], ph)) { flag_error(prm.err, 16); ok = false; break; }
       // ||k|| from the swizzled tile: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
       const unsigned char* tile = sK + (size_t)s * kStageBytes;
       float ss = 0.f;
@@ -298,18 +334,18 @@ __global__ void __launch_bounds__(kThreads, 1) dense_tc_kernel(const __grid_cons
       const int64_t row = t * BM + r;
       if (row < prm.n) prm.norms[row] = sqrtf(ss);
       for (int c = 0; c < nchunk; ++c, ++u) {
-        const int buf = (int)(u & 1);
-        if (!mbar_wait(&tfull[buf], (uint32_t)((u >> 1) & 1))) { flag_error(prm.err, 16); ok = false; break; }
+        const int buf = (int)(u & 1u);
+        if (!mbar_wait(&tfull[buf], (u >> 1) & 1u)) { flag_error(prm.err, 16); ok = false; break; }
         tc_fence_after();
         const int N = min(256, m - 256 * c);
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * 256);
         for (int cb = 0; cb < N / 32; cb += 4) {
           uint32_t wq[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            uint32_t v[32];
-            tmem_ld32(taddr + (uint32_t)((cb + k) * 32), v);
-            wq[k] = sign_word(v);
+          for (int k = 0; k < 4; k += 2) {
+            uint32_t v[64];
+            tmem_ld64(taddr + (uint32_t)((cb + k) * 32), v);
+            sign_words2(v, wq[k], wq[k + 1]);
           }
           if (row < prm.n)
             *reinterpret_cast<uint4*>(prm.bits + row * W + c * 8 + cb) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
@@ -318,6 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_tc_kernel(const __grid_cons
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);
       }
+      if (++s == NS) { s = 0; ph ^= 1u; }
     }
   }
   tc_fence_before();
@@ -371,21 +408,6 @@ int pick_stages(int d, int m) {
   return 0;
 }
 
-// Per-device error flag the kernel may set (bounded wait expired).
-int* error_flag(int dev) {
-  static std::mutex mu;
-  static int* flags[64] = {};
-  std::lock_guard<std::mutex> lock(mu);
-  if (dev < 0 || dev >= 64) return nullptr;
-  if (!flags[dev]) {
-    void* p = nullptr;
-    if (cudaMalloc(&p, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return nullptr; }
-    cudaMemset(p, 0, sizeof(int));
-    flags[dev] = (int*)p;
-  }
-  return flags[dev];
-}
-
 }  // namespace
 
 bool dense_tc_supported(const qjl_projection* P, int dtype, const void* keys, int64_t ld) {
@@ -402,7 +424,7 @@ qjl_status launch_dense_tc(const qjl_projection* P, const void* keys, int64_t n,
   if (!make_map(&tmK, keys, (uint64_t)n, (uint64_t)P->d, (uint64_t)ld, BM) ||
       !make_map(&tmS, P->S_bf16, (uint64_t)P->m, (uint64_t)P->d, (uint64_t)P->d, (uint32_t)std::min(P->m, 256)))
     return qjl_set_error(QJL_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-  int* err = error_flag(P->device);
+  int* err = qjl_error_flag(P->device);
   if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
   const int ns = pick_stages(P->d, P->m);
   const size_t smem = smem_bytes(P->d, P->m, ns);
@@ -419,6 +441,7 @@ qjl_status launch_dense_tc(const qjl_projection* P, const void* keys, int64_t n,
   }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return qjl_check_launch("dense_tc_kernel smem attribute");
+  qjl_log_launch("dense_tc_kernel", grid, kThreads, smem, 1);
   kern<<<grid, kThreads, smem, st>>>(tmK, tmS, prm);
   return qjl_check_launch("dense_tc_kernel");
 }

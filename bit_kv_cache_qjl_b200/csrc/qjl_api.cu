@@ -46,6 +46,34 @@ int qjl_num_sms(int device) {
   return cache[device];
 }
 
+void qjl_log_launch(const char* kernel, int64_t grid, int block, size_t smem, int per_sm) {
+  static const bool on = getenv("QJL_LOG_LAUNCH") != nullptr;
+  if (on)
+    fprintf(stderr, "[qjl] %s grid=%lld block=%d smem=%zu ctas_per_sm=%d\n", kernel, (long long)grid, block, smem,
+            per_sm);
+}
+
+int* qjl_error_flag(int device) {
+  static std::mutex mu;
+  static int* flags[64] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (device < 0 || device >= 64) return nullptr;
+  if (!flags[device]) {
+    void* p = nullptr;
+    if (cudaMalloc(&p, sizeof(int)) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    if (cudaMemset(p, 0, sizeof(int)) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(p);
+      return nullptr;
+    }
+    flags[device] = (int*)p;
+  }
+  return flags[device];
+}
+
 namespace {
 
 // Switch to the projection's device for the duration of a call.
@@ -314,7 +342,7 @@ qjl_status qjl_project_queries(const qjl_projection* P, const float* q, int64_t 
   DeviceGuard g(P->device);
   if (!g.ok) return qjl_set_error(QJL_ERR_CUDA, "cannot select the projection's device");
   cudaStream_t st = (cudaStream_t)stream;
-  if (P->kind == QJL_DENSE) return launch_dense_simt(P, q, QJL_F32, nq, ld, nullptr, nullptr, sq, st);
+  if (P->kind == QJL_DENSE) return launch_project_dense(P, q, nq, ld, sq, st);
   return launch_fqjl(P, q, QJL_F32, nq, ld, 0, nullptr, nullptr, sq, st);
 }
 

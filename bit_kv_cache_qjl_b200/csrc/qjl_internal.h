@@ -36,6 +36,8 @@ qjl_status qjl_check_launch(const char* what);
 qjl_status launch_dense_simt(const qjl_projection* P, const void* keys, int dtype, int64_t n,
                              int64_t ld, uint32_t* bits, float* norms, float* proj_out,
                              cudaStream_t st);
+qjl_status launch_project_dense(const qjl_projection* P, const float* q, int64_t nq, int64_t ld,
+                                float* out, cudaStream_t st);
 bool dense_tc_supported(const qjl_projection* P, int dtype, const void* keys, int64_t ld);
 qjl_status launch_dense_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld,
                            uint32_t* bits, float* norms, cudaStream_t st);
@@ -43,6 +45,9 @@ qjl_status launch_fqjl(const qjl_projection* P, const void* keys, int dtype, int
                        int64_t ld, uint64_t first_token, uint32_t* bits, float* norms,
                        float* proj_out, cudaStream_t st);
 bool scores_mma_supported(int m);
+bool scores_tc_supported(int m, int J);
+qjl_status launch_scores_tc(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t groups,
+                            int64_t N, const float* sq, int J, float* scores, cudaStream_t st);
 qjl_status launch_scores(const qjl_projection* P, const uint32_t* bits, const float* norms,
                          int64_t groups, int64_t N, const float* sq, int J, float* scores,
                          cudaStream_t st);
@@ -53,6 +58,14 @@ qjl_status launch_decode(const qjl_projection* P, const uint32_t* bits, const fl
                          const uint32_t* codes, const uint16_t* scale, const uint16_t* zero,
                          int64_t groups, int64_t N, const float* sq, int J, float softmax_scale,
                          float* out, void* ws, size_t ws_bytes, cudaStream_t st);
+
+// Per-device int the kernels set when a bounded wait expires (qjl_api.cu).
+// It is allocated on first use and never freed.
+int* qjl_error_flag(int device);
+
+// When the environment variable QJL_LOG_LAUNCH is set, print a launch's
+// grid and occupancy to stderr (qjl_api.cu).
+void qjl_log_launch(const char* kernel, int64_t grid, int block, size_t smem, int per_sm);
 
 // Device properties cached per device (qjl_api.cu).
 int qjl_num_sms(int device);

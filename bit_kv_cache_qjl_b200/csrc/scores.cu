@@ -30,20 +30,136 @@
 
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
+
+#include <algorithm>
+#include <string.h>
 
 #include "qjl_internal.h"
+#include "mbarrier.cuh"
 #include "sign_mma.cuh"
 
 namespace {
 
 using namespace qjl_sign;
-constexpr int kWarps = 8;
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kStageKeys = 256;
+constexpr int kTilesPerWarp = kStageKeys / 16 / kConsumerWarps;  // 4
+static_assert(kTilesPerWarp % 2 == 0, "tiles are consumed in pairs");
 
-// NTR column tiles (4 queries each) per pass over the keys' bits.
-template <int W, int NTR>
-__global__ void __launch_bounds__(kWarps * 32) scores_mma_kernel(
+// KT 16-key tiles of one stage (tiles tile0, tile0 + 8, ...), their MMAs
+// interleaved, written straight to `scores` from registers.
+template <int W, int NTR, int KT>
+__device__ __forceinline__ void consume_tiles(int tile0, const uint32_t* __restrict__ sb,
+                                              const float* __restrict__ sn, const float* __restrict__ nsrc,
+                                              bool nbulk, int cnt, const uint2* __restrict__ Btab,
+                                              const float* __restrict__ s_mul, const int* __restrict__ s_qsum,
+                                              int npass, int J, int64_t N, int64_t g, int64_t n0,
+                                              float* __restrict__ scores) {
+  const int lane = threadIdx.x & 31;
+  const int gq = lane >> 2, q = lane & 3;
+    int rr[KT][2];
+    uint32_t w0[KT][W / 4], w1[KT][W / 4];
+    float nrm[KT][2];
+#pragma unroll
+    for (int t2 = 0; t2 < KT; ++t2) {
+      const int tl = tile0 + t2 * kConsumerWarps;
+      rr[t2][0] = tl * 16 + gq;
+      rr[t2][1] = rr[t2][0] + 8;
+#pragma unroll
+      for (int kk = 0; kk < W / 8; ++kk) {
+        const uint2 a = (rr[t2][0] < cnt) ? *reinterpret_cast<const uint2*>(sb + rr[t2][0] * W + q * (W / 4) + 2 * kk)
+                                          : make_uint2(0, 0);
+        const uint2 b = (rr[t2][1] < cnt) ? *reinterpret_cast<const uint2*>(sb + rr[t2][1] * W + q * (W / 4) + 2 * kk)
+                                          : make_uint2(0, 0);
+        w0[t2][2 * kk] = a.x; w0[t2][2 * kk + 1] = a.y;
+        w1[t2][2 * kk] = b.x; w1[t2][2 * kk + 1] = b.y;
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        nrm[t2][r] = rr[t2][r] < cnt ? (nbulk ? sn[rr[t2][r]] : __ldg(nsrc + rr[t2][r])) : 0.f;
+    }
+    if (tile0 * 16 < cnt) {
+      for (int pass = 0; pass < npass; ++pass) {
+        int acc[KT][NTR][4][4];
+#pragma unroll
+        for (int t2 = 0; t2 < KT; ++t2)
+#pragma unroll
+          for (int a = 0; a < NTR; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+#pragma unroll
+              for (int c = 0; c < 4; ++c) acc[t2][a][b][c] = 0;
+#pragma unroll
+        for (int p = 0; p < W / 8; ++p) {
+#pragma unroll
+          for (int sh = 0; sh < 2; ++sh) {
+            uint32_t x[KT][4];
+#pragma unroll
+            for (int t2 = 0; t2 < KT; ++t2) {
+              x[t2][0] = w0[t2][2 * p] >> sh;
+              x[t2][1] = w1[t2][2 * p] >> sh;
+              x[t2][2] = w0[t2][2 * p + 1] >> sh;
+              x[t2][3] = w1[t2][2 * p + 1] >> sh;
+            }
+#pragma unroll
+            for (int Ji = 0; Ji < 4; ++Ji) {
+              const uint32_t M = 0x01010101u << (2 * Ji);
+              const int mu = 8 * p + 2 * Ji + sh;
+#pragma unroll
+              for (int nt = 0; nt < NTR; ++nt) {
+                const uint2 bb = Btab[((pass * NTR + nt) * W + mu) * 32 + lane];
+#pragma unroll
+                for (int t2 = 0; t2 < KT; ++t2)
+                  mma_u8s8(acc[t2][nt][Ji], x[t2][0] & M, x[t2][1] & M, x[t2][2] & M, x[t2][3] & M, bb.x, bb.y);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NTR; ++nt) {
+          const int jq = (pass * NTR + nt) * 4 + q;
+          if (jq >= J) continue;
+          const float mul = s_mul[jq] * 0.03125f;
+          const float qs32 = 32.f * (float)s_qsum[jq];
+          float* orow = scores + (g * J + jq) * N + n0;
+#pragma unroll
+          for (int t2 = 0; t2 < KT; ++t2) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const int row = rr[t2][r];
+              if (row >= cnt) continue;
+              const int hi = ((acc[t2][nt][0][2 * r] * 4 + acc[t2][nt][1][2 * r]) * 4 + acc[t2][nt][2][2 * r]) * 4 +
+                             acc[t2][nt][3][2 * r];
+              const int lo = ((acc[t2][nt][0][2 * r + 1] * 4 + acc[t2][nt][1][2 * r + 1]) * 4 +
+                              acc[t2][nt][2][2 * r + 1]) * 4 + acc[t2][nt][3][2 * r + 1];
+              // 32 * sum (2b - 1) Q in fp32: |hi| < 2^24 is exact, and the
+              // rounding of the sum is far below the 16-bit rounding of Sq
+              const float D = fmaf((float)hi, 256.f, (float)lo) - qs32;
+              orow[row] = mul * nrm[t2][r] * D;
+            }
+          }
+        }
+      }
+    }
+}
+
+// Streaming kernel. Persistent CTAs each take a contiguous range of work
+// items (group g, chunk of kStageKeys keys), g-major, so a CTA crosses at most
+// a few group boundaries. Warp 4 (one lane) is the producer. It moves each
+// chunk's packed bits, and its norms when they are 16-byte aligned, into an
+// NS-stage shared-memory ring with cp.async.bulk, completing on the stage's
+// mbarrier. Warps 0-3 consume: each takes four 16-key tiles of the stage,
+// runs the sign-sum MMAs against the group's B tables, and writes scores
+// straight from registers. At a group boundary the consumer warps rebuild
+// the tables behind a named barrier.
+template <int W, int NTR, int KT>
+__global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 1) scores_stream_kernel(
     const uint32_t* __restrict__ bits, const float* __restrict__ norms, const float* __restrict__ sq,
-    int64_t N, int J, float est_scale, int64_t tiles_per_cta, float* __restrict__ scores) {
+    int64_t G, int64_t N, int J, int NS, float est_scale, int64_t items_per_cta, float* __restrict__ scores,
+    int* __restrict__ err) {
+  using namespace qjl_sync;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int NT = (J + 3) / 4;
   const int npass = (NT + NTR - 1) / NTR;
@@ -52,85 +168,259 @@ __global__ void __launch_bounds__(kWarps * 32) scores_mma_kernel(
   float* s_mul = s_inv + 64;
   int* s_qsum = reinterpret_cast<int*>(s_mul + 64);
   uint2* Btab = reinterpret_cast<uint2*>(smem_raw + 3 * 64 * 4);
-
-  const int64_t gi = blockIdx.y;
-  build_tables<W>(sq + gi * (int64_t)J * (32 * W), J, NTP, est_scale, s_inv, s_mul, s_qsum, Btab,
-                  kWarps);
+  uint32_t* sbits = reinterpret_cast<uint32_t*>(Btab + (size_t)NTP * W * 32);   // [NS][kStageKeys * W]
+  float* snorm = reinterpret_cast<float*>(sbits + (size_t)NS * kStageKeys * W); // [NS][kStageKeys]
+  uint64_t* full = reinterpret_cast<uint64_t*>(snorm + (size_t)NS * kStageKeys);
+  uint64_t* empty = full + NS;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, q = lane & 3;
-  const int64_t ntiles = (N + 15) >> 4;
-  const int64_t t_begin = (int64_t)blockIdx.x * tiles_per_cta;
-  const int64_t t_end = min(ntiles, t_begin + tiles_per_cta);
-  const uint32_t* gbits = bits + gi * N * W;
-  const float* gnorm = norms + gi * N;
+  const int64_t cpg = (N + kStageKeys - 1) / kStageKeys;
+  const int64_t total = G * cpg;
+  const int64_t i0 = (int64_t)blockIdx.x * items_per_cta;
+  const int64_t i1 = min(total, i0 + items_per_cta);
 
-  int64_t t = t_begin + warp;
-  uint32_t cur[2][W / 4], nxt[2][W / 4];
-  if (t < t_end) {
-    load_words<W>(gbits, t * 16 + g, N, q, cur[0]);
-    load_words<W>(gbits, t * 16 + g + 8, N, q, cur[1]);
-  }
-  for (; t < t_end; t += kWarps) {
-    const int64_t tn = t + kWarps;
-    if (tn < t_end) {
-      load_words<W>(gbits, tn * 16 + g, N, q, nxt[0]);
-      load_words<W>(gbits, tn * 16 + g + 8, N, q, nxt[1]);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
     }
-    const int64_t row0 = t * 16 + g, row1 = row0 + 8;
-    float nrm[2] = {0.f, 0.f};
-    if (row0 < N) nrm[0] = __ldg(gnorm + row0);
-    if (row1 < N) nrm[1] = __ldg(gnorm + row1);
-    for (int pass = 0; pass < npass; ++pass) {
-      int acc[NTR][4][4];
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      // incremental (group, chunk) and (stage, phase): no 64-bit division in the loop
+      int64_t g = i0 / cpg, c = i0 - (i0 / cpg) * cpg;
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      for (int64_t it = i0; it < i1; ++it, ++issued) {
+        if (!mbar_wait(&empty[s], ph ^ 1u)) { atomicOr(err, 1); break; }
+        const int64_t n0 = c * kStageKeys;
+        const int cnt = (int)(N - n0 < kStageKeys ? N - n0 : kStageKeys);
+        const float* nsrc = norms + g * N + n0;
+        const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
+        const uint32_t bbytes = (uint32_t)cnt * W * 4;
+        mbar_expect_tx(&full[s], bbytes + (nbulk ? (uint32_t)cnt * 4 : 0u));
+        bulk_g2s(sbits + (size_t)s * kStageKeys * W, bits + (g * N + n0) * W, bbytes, &full[s]);
+        if (nbulk) bulk_g2s(snorm + (size_t)s * kStageKeys, nsrc, (uint32_t)cnt * 4, &full[s]);
+        if (++c == cpg) { c = 0; ++g; }
+        if (++s == NS) { s = 0; ph ^= 1u; }
+      }
+      // every copy issued into a stage has landed before the CTA exits: the
+      // most recent phase of each used stage is waited on again
+      const int used = issued < NS ? (int)issued : NS;
+      for (int j = 0; j < used; ++j) {
+        // stage (s - 1 - j) mod NS; its last phase parity flips when we wrap back past 0
+        int st = s - 1 - j;
+        uint32_t p = ph;
+        if (st < 0) { st += NS; p ^= 1u; }
+        if (!mbar_wait(&full[st], p)) atomicOr(err, 2);
+      }
+    }
+    return;
+  }
+
+  // consumers
+  int64_t cur_g = -1;
+  int64_t g = i0 / cpg, c = i0 - (i0 / cpg) * cpg;
+  int s = 0;
+  uint32_t ph = 0;
+  for (int64_t it = i0; it < i1; ++it) {
+    const int64_t n0 = c * kStageKeys;
+    const int cnt = (int)(N - n0 < kStageKeys ? N - n0 : kStageKeys);
+    if (g != cur_g) {
+      named_sync(1, kConsumerWarps * 32);
+      build_tables<W>(sq + g * (int64_t)J * (32 * W), J, NTP, est_scale, s_inv, s_mul, s_qsum, Btab,
+                      kConsumerWarps, 1);
+      cur_g = g;
+    }
+    if (!mbar_wait(&full[s], ph)) { atomicOr(err, 4); break; }
+    const float* nsrc = norms + g * N + n0;
+    const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
+    const uint32_t* sb = sbits + (size_t)s * kStageKeys * W;
+    const float* sn = snorm + (size_t)s * kStageKeys;
+    // this warp's tiles of the stage, KT at a time (KT = 2 interleaves two
+    // tiles' MMAs for ILP where registers allow)
+#pragma unroll 1
+    for (int i = 0; i < kTilesPerWarp; i += KT)
+      consume_tiles<W, NTR, KT>(warp + i * kConsumerWarps, sb, sn, nsrc, nbulk, cnt, Btab, s_mul, s_qsum, npass, J,
+                                N, g, n0, scores);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (++c == cpg) { c = 0; ++g; }
+    if (++s == NS) { s = 0; ph ^= 1u; }
+  }
+}
+
+// Decode fast path: at most 4 queries per group (one n8 column tile), so each
+// consumer thread keeps its B fragments in registers (2 W of them), loaded
+// from the shared table once per group. The first MMA of each accumulator
+// takes a zero C operand. Stages are 512 keys (16 KB of bits at m = 256) and
+// two tiles' MMAs are interleaved per consumer warp.
+constexpr int kDecStageKeys = 512;
+constexpr int kDecTilesPerWarp = kDecStageKeys / 16 / kConsumerWarps;  // 8
+
+__device__ __forceinline__ void mma_u8s8_zc(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};\n"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
+
+template <int W>
+__global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 2) scores_decode_kernel(
+    const uint32_t* __restrict__ bits, const float* __restrict__ norms, const float* __restrict__ sq,
+    int64_t G, int64_t N, int J, int NS, float est_scale, int64_t items_per_cta, float* __restrict__ scores,
+    int* __restrict__ err) {
+  using namespace qjl_sync;
+  constexpr int SK = kDecStageKeys;
+  constexpr int KT = 2;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* s_inv = reinterpret_cast<float*>(smem_raw);
+  float* s_mul = s_inv + 64;
+  int* s_qsum = reinterpret_cast<int*>(s_mul + 64);
+  uint2* Btab = reinterpret_cast<uint2*>(smem_raw + 3 * 64 * 4);
+  uint32_t* sbits = reinterpret_cast<uint32_t*>(Btab + (size_t)W * 32);     // [NS][SK * W]
+  float* snorm = reinterpret_cast<float*>(sbits + (size_t)NS * SK * W);    // [NS][SK]
+  uint64_t* full = reinterpret_cast<uint64_t*>(snorm + (size_t)NS * SK);
+  uint64_t* empty = full + NS;
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t cpg = (N + SK - 1) / SK;
+  const int64_t total = G * cpg;
+  const int64_t i0 = (int64_t)blockIdx.x * items_per_cta;
+  const int64_t i1 = min(total, i0 + items_per_cta);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      int64_t g = i0 / cpg, c = i0 - (i0 / cpg) * cpg;
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      for (int64_t it = i0; it < i1; ++it, ++issued) {
+        if (!mbar_wait(&empty[s], ph ^ 1u)) { atomicOr(err, 1); break; }
+        const int64_t n0 = c * SK;
+        const int cnt = (int)(N - n0 < SK ? N - n0 : SK);
+        const float* nsrc = norms + g * N + n0;
+        const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
+        const uint32_t bbytes = (uint32_t)cnt * W * 4;
+        mbar_expect_tx(&full[s], bbytes + (nbulk ? (uint32_t)cnt * 4 : 0u));
+        bulk_g2s(sbits + (size_t)s * SK * W, bits + (g * N + n0) * W, bbytes, &full[s]);
+        if (nbulk) bulk_g2s(snorm + (size_t)s * SK, nsrc, (uint32_t)cnt * 4, &full[s]);
+        if (++c == cpg) { c = 0; ++g; }
+        if (++s == NS) { s = 0; ph ^= 1u; }
+      }
+      const int used = issued < NS ? (int)issued : NS;
+      for (int j = 0; j < used; ++j) {
+        int st = s - 1 - j;
+        uint32_t p = ph;
+        if (st < 0) { st += NS; p ^= 1u; }
+        if (!mbar_wait(&full[st], p)) atomicOr(err, 2);
+      }
+    }
+    return;
+  }
+
+  const int gq = lane >> 2, q = lane & 3;
+  int64_t g = i0 / cpg, c = i0 - (i0 / cpg) * cpg;
+  int64_t cur_g = -1;
+  int s = 0;
+  uint32_t ph = 0;
+  uint2 breg[W];
+  float mul = 0.f, qs32 = 0.f;
+  for (int64_t it = i0; it < i1; ++it) {
+    const int64_t n0 = c * SK;
+    const int cnt = (int)(N - n0 < SK ? N - n0 : SK);
+    if (g != cur_g) {
+      named_sync(1, kConsumerWarps * 32);
+      build_tables<W>(sq + g * (int64_t)J * (32 * W), J, 1, est_scale, s_inv, s_mul, s_qsum, Btab, kConsumerWarps,
+                      1);
 #pragma unroll
-      for (int a = 0; a < NTR; ++a)
+      for (int mu = 0; mu < W; ++mu) breg[mu] = Btab[mu * 32 + lane];
+      mul = q < J ? s_mul[q] * 0.03125f : 0.f;
+      qs32 = q < J ? 32.f * (float)s_qsum[q] : 0.f;
+      cur_g = g;
+    }
+    if (!mbar_wait(&full[s], ph)) { atomicOr(err, 4); break; }
+    const float* nsrc = norms + g * N + n0;
+    const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
+    const uint32_t* sb = sbits + (size_t)s * SK * W;
+    const float* sn = snorm + (size_t)s * SK;
+    float* gout = scores + (g * J + q) * N + n0;
+#pragma unroll 1
+    for (int i = 0; i < kDecTilesPerWarp; i += KT) {
+      const int tile0 = warp + i * kConsumerWarps;
+      if (tile0 * 16 >= cnt) break;
+      int rr[KT][2];
+      uint32_t w0[KT][W / 4], w1[KT][W / 4];
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
+      for (int t2 = 0; t2 < KT; ++t2) {
+        rr[t2][0] = (tile0 + t2 * kConsumerWarps) * 16 + gq;
+        rr[t2][1] = rr[t2][0] + 8;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) acc[a][b][c] = 0;
+        for (int r = 0; r < 2; ++r) {
+          // rows past cnt read stale stage data; their results are never stored
+          const uint32_t* src = sb + min(rr[t2][r], SK - 1) * W + q * (W / 4);
+#pragma unroll
+          for (int kk = 0; kk < W / 8; ++kk) {
+            const uint2 v = *reinterpret_cast<const uint2*>(src + 2 * kk);
+            (r ? w1 : w0)[t2][2 * kk] = v.x;
+            (r ? w1 : w0)[t2][2 * kk + 1] = v.y;
+          }
+        }
+      }
+      int acc[KT][4][4];
 #pragma unroll
       for (int p = 0; p < W / 8; ++p) {
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          const uint32_t x0 = cur[0][2 * p] >> s, x1 = cur[1][2 * p] >> s;
-          const uint32_t x2 = cur[0][2 * p + 1] >> s, x3 = cur[1][2 * p + 1] >> s;
+        for (int sh = 0; sh < 2; ++sh) {
 #pragma unroll
           for (int Ji = 0; Ji < 4; ++Ji) {
             const uint32_t M = 0x01010101u << (2 * Ji);
-            const int mu = 8 * p + 2 * Ji + s;
+            const uint2 bb = breg[8 * p + 2 * Ji + sh];
 #pragma unroll
-            for (int nt = 0; nt < NTR; ++nt) {
-              const uint2 bb = Btab[((pass * NTR + nt) * W + mu) * 32 + lane];
-              mma_u8s8(acc[nt][Ji], x0 & M, x1 & M, x2 & M, x3 & M, bb.x, bb.y);
+            for (int t2 = 0; t2 < KT; ++t2) {
+              const uint32_t a0 = (w0[t2][2 * p] >> sh) & M, a1 = (w1[t2][2 * p] >> sh) & M;
+              const uint32_t a2 = (w0[t2][2 * p + 1] >> sh) & M, a3 = (w1[t2][2 * p + 1] >> sh) & M;
+              if (p == 0 && sh == 0) mma_u8s8_zc(acc[t2][Ji], a0, a1, a2, a3, bb.x, bb.y);
+              else mma_u8s8(acc[t2][Ji], a0, a1, a2, a3, bb.x, bb.y);
             }
           }
         }
       }
+      if (q < J) {
 #pragma unroll
-      for (int nt = 0; nt < NTR; ++nt) {
-        const int jq = (pass * NTR + nt) * 4 + q;
-        if (jq >= J) continue;
-        const float mul = s_mul[jq];
-        const long long qs32 = 32LL * s_qsum[jq];
+        for (int t2 = 0; t2 < KT; ++t2) {
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int64_t row = row0 + 8 * r;
-          if (row >= N) continue;
-          const int hi = ((acc[nt][0][2 * r] * 4 + acc[nt][1][2 * r]) * 4 + acc[nt][2][2 * r]) * 4 +
-                         acc[nt][3][2 * r];
-          const int lo = ((acc[nt][0][2 * r + 1] * 4 + acc[nt][1][2 * r + 1]) * 4 +
-                          acc[nt][2][2 * r + 1]) * 4 + acc[nt][3][2 * r + 1];
-          const long long D = 256LL * hi + lo - qs32;  // 32 * sum (2b - 1) Q
-          scores[(gi * J + jq) * N + row] = mul * nrm[r] * ((float)D * 0.03125f);
+          for (int r = 0; r < 2; ++r) {
+            const int row = rr[t2][r];
+            if (row >= cnt) continue;
+            const int hi = ((acc[t2][0][2 * r] * 4 + acc[t2][1][2 * r]) * 4 + acc[t2][2][2 * r]) * 4 + acc[t2][3][2 * r];
+            const int lo = ((acc[t2][0][2 * r + 1] * 4 + acc[t2][1][2 * r + 1]) * 4 + acc[t2][2][2 * r + 1]) * 4 +
+                           acc[t2][3][2 * r + 1];
+            const float nrm = nbulk ? sn[row] : __ldg(nsrc + row);
+            gout[row] = mul * nrm * (fmaf((float)hi, 256.f, (float)lo) - qs32);
+          }
         }
       }
     }
-#pragma unroll
-    for (int k = 0; k < W / 4; ++k) {
-      cur[0][k] = nxt[0][k];
-      cur[1][k] = nxt[1][k];
-    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (++c == cpg) { c = 0; ++g; }
+    if (++s == NS) { s = 0; ph ^= 1u; }
   }
 }
 
@@ -160,25 +450,62 @@ __global__ void __launch_bounds__(256) scores_simt_kernel(
   }
 }
 
+size_t stream_smem(int W, int NTP, int NS) {
+  return 3 * 64 * 4 + (size_t)NTP * W * 32 * sizeof(uint2) + (size_t)NS * kStageKeys * (W + 1) * 4 +
+         (size_t)2 * NS * 8;
+}
+
 template <int W, int NTR>
 qjl_status launch_mma(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t G,
                       int64_t N, const float* sq, int J, float* scores, cudaStream_t st) {
   const int NT = (J + 3) / 4;
   const int NTP = ((NT + NTR - 1) / NTR) * NTR;
-  const size_t smem = 3 * 64 * 4 + (size_t)NTP * W * 32 * sizeof(uint2);
-  auto kern = scores_mma_kernel<W, NTR>;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return qjl_check_launch("scores_mma_kernel smem attribute");
-  const int64_t ntiles = (N + 15) / 16;
-  const int64_t target = (int64_t)qjl_num_sms(P->device) * 4;
-  int64_t splits = (target + G - 1) / G;
-  splits = std::max<int64_t>(1, std::min<int64_t>(splits, (ntiles + kWarps - 1) / kWarps));
-  const int64_t tpc = (ntiles + splits - 1) / splits;
-  splits = (ntiles + tpc - 1) / tpc;
-  dim3 grid((unsigned)splits, (unsigned)G);
-  kern<<<grid, kWarps * 32, smem, st>>>(bits, norms, sq, N, J, P->est_scale, tpc, scores);
-  return qjl_check_launch("scores_mma_kernel");
+  int NS = W <= 8 ? 4 : (W <= 16 ? 3 : 2);
+  while (NS > 2 && stream_smem(W, NTP, NS) > 200 * 1024) --NS;
+  const size_t smem = stream_smem(W, NTP, NS);
+  auto kern = scores_stream_kernel<W, NTR, (W <= 16 && NTR == 1) ? 2 : 1>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+    return qjl_check_launch("scores_stream_kernel smem attribute");
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess || per_sm < 1)
+    return qjl_check_launch("scores_stream_kernel occupancy");
+  int* err = qjl_error_flag(P->device);
+  if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  const int64_t total = G * ((N + kStageKeys - 1) / kStageKeys);
+  const int64_t slots = (int64_t)qjl_num_sms(P->device) * per_sm;
+  const int64_t grid = std::min<int64_t>(total, slots);
+  const int64_t ipc = (total + grid - 1) / grid;
+  const int64_t nblk = (total + ipc - 1) / ipc;
+  qjl_log_launch("scores_stream_kernel", nblk, kThreads, smem, per_sm);
+  kern<<<(unsigned)nblk, kThreads, smem, st>>>(bits, norms, sq, G, N, J, NS, P->est_scale, ipc, scores, err);
+  return qjl_check_launch("scores_stream_kernel");
+}
+
+template <int W>
+qjl_status launch_decode_fast(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t G,
+                              int64_t N, const float* sq, int J, float* scores, cudaStream_t st) {
+  const int NS = W == 8 ? 4 : 3;
+  const size_t smem = 3 * 64 * 4 + (size_t)W * 32 * sizeof(uint2) + (size_t)NS * kDecStageKeys * (W + 1) * 4 +
+                      (size_t)2 * NS * 8;
+  auto kern = scores_decode_kernel<W>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+    return qjl_check_launch("scores_decode_kernel smem attribute");
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return qjl_check_launch("scores_decode_kernel attributes");
+  const int regs_per_cta = ((fa.numRegs * 32 + 255) / 256) * 256 * (kThreads / 32);
+  const int per_sm = std::max(1, std::min(65536 / std::max(regs_per_cta, 1), (int)((228u * 1024u) / (smem + 1024))));
+  int* err = qjl_error_flag(P->device);
+  if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  const int64_t total = G * ((N + kDecStageKeys - 1) / kDecStageKeys);
+  const int64_t slots = (int64_t)qjl_num_sms(P->device) * per_sm;
+  const int64_t grid = std::min<int64_t>(total, slots);
+  const int64_t ipc = (total + grid - 1) / grid;
+  const int64_t nblk = (total + ipc - 1) / ipc;
+  qjl_log_launch("scores_decode_kernel", nblk, kThreads, smem, per_sm);
+  kern<<<(unsigned)nblk, kThreads, smem, st>>>(bits, norms, sq, G, N, J, NS, P->est_scale, ipc, scores, err);
+  return qjl_check_launch("scores_decode_kernel");
 }
 
 }  // namespace
@@ -187,7 +514,21 @@ bool scores_mma_supported(int m) { return m == 256 || m == 512 || m == 1024; }
 
 qjl_status launch_scores(const qjl_projection* P, const uint32_t* bits, const float* norms,
                          int64_t G, int64_t N, const float* sq, int J, float* scores, cudaStream_t st) {
-  if (G > 65535) return qjl_set_error(QJL_ERR_UNSUPPORTED, "groups > 65535");
+  // J <= 4 at m = 256 or 512 takes the register-resident decode kernel. The
+  // tcgen05 variant (QJL_SCORES_KERNEL=tc) computes the same sums on the 5th-gen
+  // tensor cores, but at about 48 cycles per 128x8x32 MMA its A-operand reads
+  // (one byte per sign bit) cap it below the mma.sync path; it is kept for
+  // comparison. QJL_SCORES_KERNEL=stream selects the generic streaming kernel.
+  static const int choice = [] {
+    const char* v = getenv("QJL_SCORES_KERNEL");
+    if (v && strcmp(v, "tc") == 0) return 1;
+    if (v && strcmp(v, "stream") == 0) return 2;
+    return 0;
+  }();
+  if (choice == 1 && scores_tc_supported(P->m, J)) return launch_scores_tc(P, bits, norms, G, N, sq, J, scores, st);
+  if (choice == 0 && J <= 4 && (P->m == 256 || P->m == 512))
+    return P->m == 256 ? launch_decode_fast<8>(P, bits, norms, G, N, sq, J, scores, st)
+                       : launch_decode_fast<16>(P, bits, norms, G, N, sq, J, scores, st);
   const int NTR = J > 4 ? 2 : 1;
   switch (scores_mma_supported(P->m) ? P->m : 0) {
     case 256: return NTR == 1 ? launch_mma<8, 1>(P, bits, norms, G, N, sq, J, scores, st)

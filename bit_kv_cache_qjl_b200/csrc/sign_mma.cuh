@@ -32,9 +32,13 @@ __device__ __forceinline__ int quant16(float v, float inv) {
 // mu = 8 p + j. The entries need W % 8 == 0.
 template <int W>
 __device__ void build_tables(const float* __restrict__ sqg, int J, int NT, float est_scale,
-                             float* s_inv, float* s_mul, int* s_qsum, uint2* Btab, int nwarps) {
+                             float* s_inv, float* s_mul, int* s_qsum, uint2* Btab, int nwarps,
+                             int bar_id = 0) {
+  // bar_id 0: all threads of the block take part; otherwise the first
+  // 32 * nwarps threads synchronise on named barrier bar_id.
   constexpr int m = 32 * W;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nthreads = 32 * nwarps;
   for (int j = warp; j < J; j += nwarps) {
     const float* row = sqg + (int64_t)j * m;
     float mx = 0.f;
@@ -52,9 +56,10 @@ __device__ void build_tables(const float* __restrict__ sqg, int J, int NT, float
       s_qsum[j] = qs;
     }
   }
-  __syncthreads();
+  if (bar_id) asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthreads) : "memory");
+  else __syncthreads();
   const int entries = NT * W * 32;
-  for (int idx = threadIdx.x; idx < entries; idx += blockDim.x) {
+  for (int idx = threadIdx.x; idx < entries; idx += nthreads) {
     const int ln = idx & 31;
     const int mu = (idx >> 5) % W;
     const int pt = (idx >> 5) / W;
@@ -80,7 +85,8 @@ __device__ void build_tables(const float* __restrict__ sqg, int J, int NT, float
     }
     Btab[idx] = make_uint2(b[0], b[1]);
   }
-  __syncthreads();
+  if (bar_id) asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthreads) : "memory");
+  else __syncthreads();
 }
 
 template <int W>

@@ -1,0 +1,74 @@
+"""The hot path runs the intended kernels of libqjl_b200.so.
+
+The CUDA profiler (CUPTI, through torch.profiler) lists every kernel launched
+in the process. Each call must launch its own library kernel, with no torch
+kernels and no CPU work standing in.
+"""
+
+import pytest
+import torch
+
+import bit_kv_cache_qjl_b200 as qjl
+from bit_kv_cache_qjl_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def _kernels(fn):
+    torch.cuda.synchronize()
+    with torch.profiler.profile(activities=[torch.profiler.ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    return names
+
+
+def _has(names, frag):
+    return any(frag in n for n in names)
+
+
+def test_dense_bf16_uses_tcgen05_kernel(cuda_ok):
+    P = qjl.Projection(2, 128, 256, "dense")
+    keys = wl.normal((4096, 128), 1, "cuda", torch.bfloat16)
+    names = _kernels(lambda: qjl.quantize_keys(P, keys))
+    assert _has(names, "dense_tc_kernel"), names
+    assert not _has(names, "dense_simt_kernel")
+
+
+def test_fp32_keys_use_simt_kernel(cuda_ok):
+    P = qjl.Projection(2, 128, 256, "dense", s_bf16=False)
+    keys = wl.normal((512, 128), 1, "cuda")
+    assert _has(_kernels(lambda: qjl.quantize_keys(P, keys)), "dense_simt_kernel")
+
+
+def test_fqjl_kernel(cuda_ok):
+    P = qjl.Projection(4, 256, 1024, "pfqjl")
+    keys = wl.normal((512, 256), 1, "cuda", torch.bfloat16)
+    assert _has(_kernels(lambda: qjl.quantize_keys(P, keys)), "fqjl_kernel")
+
+
+def test_scores_and_projection_kernels(cuda_ok):
+    P = qjl.Projection(2, 128, 256, "dense")
+    bits = torch.zeros((4, 1000, 8), dtype=torch.int32, device="cuda")
+    norms = torch.ones((4, 1000), device="cuda")
+    q = wl.normal((4, 128), 3, "cuda")
+    names = _kernels(lambda: qjl.scores(P, bits, norms, qjl.project_queries(P, q).view(4, 1, 256)))
+    assert _has(names, "scores_decode_kernel") and _has(names, "project_dense_kernel"), names
+    # more than 4 queries per group take the streaming mma.sync kernel
+    sq8 = torch.ones((4, 8, 256), device="cuda")
+    assert _has(_kernels(lambda: qjl.scores(P, bits, norms, sq8)), "scores_stream_kernel")
+
+
+def test_values_and_decode_kernels(cuda_ok):
+    P = qjl.Projection(5, 128, 256, "dfqjl")
+    v = wl.normal((2 * 300, 128), 4, "cuda", torch.bfloat16)
+    bits = torch.zeros((2, 300, 8), dtype=torch.int32, device="cuda")
+    norms = torch.ones((2, 300), device="cuda")
+    sq = torch.ones((2, 1, 256), device="cuda")
+
+    def run():
+        c, s, z = qjl.quantize_values_2bit(v)
+        qjl.decode_attention(P, bits, norms, c.view(2, 300, 8), s.view(2, 300, 4), z.view(2, 300, 4), sq, 0.1)
+    names = _kernels(run)
+    for k in ("values_2bit_kernel", "decode_partial_kernel", "decode_combine_kernel"):
+        assert _has(names, k), (k, names)

@@ -39,7 +39,8 @@ def _case(kind, d, m, G, J, N, seed=0):
 
 @pytest.mark.parametrize("m,G,J,N", [(256, 3, 1, 1000), (256, 1, 4, 4096), (256, 2, 16, 333), (512, 2, 4, 2049),
                                      (512, 1, 5, 100), (1024, 1, 64, 300), (1024, 2, 1, 1), (256, 4, 3, 17),
-                                     (256, 1, 64, 200)])
+                                     (256, 1, 64, 200), (256, 50, 1, 100), (256, 37, 2, 300), (512, 20, 4, 129),
+                                     (512, 9, 3, 1000), (256, 300, 1, 7)])
 def test_scores_tensor_core(cuda_ok, m, G, J, N):
     _case("dense", 128, m, G, J, N)
 
