@@ -7,7 +7,7 @@
 // is the slow one to apply, so it runs on the tensor cores: bf16 operands
 // with fp32 accumulators in TMEM.
 //
-// Persistent kernel, one CTA per SM, 6 warps:
+// Persistent kernel, one CTA per SM, 12 warps:
 //   warp 0     TMA producer. S_eff [m][d] is loaded once into shared memory.
 //              Then 128-key tiles stream through an NS-stage ring, each
 //              stage 128 rows x d bf16 in 128-byte swizzled atoms of 64
@@ -16,11 +16,16 @@
 //              One elected lane issues tcgen05.mma M=128, N<=256, K=16 over
 //              d/16 steps per work unit. A work unit is (tile, 256-column
 //              chunk of m). Completion goes to mbarriers via tcgen05.commit.
-//   warps 2-5  epilogue. Warp w reads TMEM lanes 32*(w%4)..+31, so each
-//              thread owns one key row. tcgen05.ld moves 32 columns, and 32
-//              funnel shifts gather the sign bits into one word (bit = 1 iff
-//              y >= 0). Words leave as 16-byte stores. ||k|| comes from the
-//              swizzled key tile already in shared memory.
+//   warps 2-9  epilogue. Warp w reads TMEM lanes 32*(w%4)..+31, so each
+//              thread owns one key row. The two warps on a lane quarter take
+//              half of the accumulator columns each: four tcgen05.ld of 32
+//              columns with one wait, and eight independent funnel-shift
+//              chains per 64 values gather the sign bits (bit = 1 iff y >= 0).
+//              Words leave as 16-byte stores.
+//   warps 10-11 ||k|| from the swizzled key tile already in shared memory:
+//              two rows per thread, sm_100 mixed-precision FMA (bf16 in, fp32
+//              accumulate, 4 accumulators per row). These warps, not the epilogue,
+//              release the key stage together with the MMAs' commit.
 // Every mbarrier wait is bounded. On expiry the kernel records an error
 // flag, drains what it issued, frees TMEM and returns.
 
@@ -35,7 +40,9 @@
 namespace {
 
 constexpr int BM = 128;            // keys per tile (MMA M)
-constexpr int kThreads = 192;      // 6 warps
+constexpr int kEpiWarps = 8;
+constexpr int kNormWarps = 2;
+constexpr int kThreads = (2 + kEpiWarps + kNormWarps) * 32;  // producer, MMA, epilogue, norms
 constexpr int kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
 
@@ -149,8 +156,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Two back-to-back 32-column TMEM loads (64 columns of this thread's row), one wait.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+// Two back-to-back 32-column TMEM loads (64 columns of this thread's row), no wait.
+__device__ __forceinline__ void tmem_ld64_nowait(uint32_t taddr, uint32_t (&r)[64]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
       "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -167,6 +174,10 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
         "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
         "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
       : "r"(taddr + 32u));
+}
+
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  tmem_ld64_nowait(taddr, r);
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
@@ -184,6 +195,31 @@ __device__ __forceinline__ void sign_words2(const uint32_t (&r)[64], uint32_t& w
   }
   w0 = ~(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24));
   w1 = ~(c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+}
+
+// 128 columns (four 32-column loads issued back to back, one wait) -> 4 sign words.
+__device__ __forceinline__ void tmem_ld128_pack(uint32_t taddr, uint32_t (&w)[4]) {
+  uint32_t v0[64], v1[64];
+  tmem_ld64_nowait(taddr, v0);
+  tmem_ld64_nowait(taddr + 64u, v1);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  sign_words2(v0, w[0], w[1]);
+  sign_words2(v1, w[2], w[3]);
+}
+
+__device__ __forceinline__ void tmem_ld64_pack(uint32_t taddr, uint32_t& w0, uint32_t& w1) {
+  uint32_t v[64];
+  tmem_ld64(taddr, v);
+  sign_words2(v, w0, w1);
+}
+
+// acc += lo^2 + hi^2 for the two bf16 halves of u, with sm_100's mixed-precision
+// FMA (bf16 operands widened exactly, fp32 accumulate): no unpacking.
+__device__ __forceinline__ void sq_acc_bf16x2(uint32_t u, float& acc) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tfma.rn.f32.bf16 %0, lo, lo, %0;\n\t"
+      "fma.rn.f32.bf16 %0, hi, hi, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(u));
 }
 
 __device__ __forceinline__ void flag_error(int* err, int code) { atomicOr(err, code); }
@@ -217,11 +253,11 @@ __global__ void __launch_bounds__(kThreads, 1) dense_tc_kernel(const __grid_cons
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);
+      mbar_init(&empty[s], 1 + kNormWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], kEpiWarps);
     }
     mbar_init(sbar, 1);
     mbar_init(dbar, 1);
@@ -301,58 +337,77 @@ __global__ void __launch_bounds__(kThreads, 1) dense_tc_kernel(const __grid_cons
       mma_commit(dbar);
       if (!mbar_wait(dbar, 0)) flag_error(prm.err, 8);
     }
-  } else {
-    // epilogue: thread owns TMEM lane (row) 32*(warp%4) + lane
+  } else if (warp < 2 + kEpiWarps) {
+    // epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (the hardware ties a warp
+    // to its lane quarter), so each thread owns one key row; the two warps on a
+    // quarter take half of the accumulator columns each
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const int W = m >> 5;
     uint32_t u = 0;
-    int s = 0;
-    uint32_t ph = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-      if (!mbar_wait(&full[s], ph)) { flag_error(prm.err, 16); ok = false; break; }
-      // ||k|| from the swizzled tile: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
-      const unsigned char* tile = sK + (size_t)s * kStageBytes;
-      float ss = 0.f;
-#pragma unroll
-      for (int a = 0; a < KA; ++a) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(tile + a * BM * 128 + r * 128 + ((c ^ (r & 7)) << 4));
-          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const float lo = __uint_as_float(wv[h] << 16), hi = __uint_as_float(wv[h] & 0xFFFF0000u);
-            ss = fmaf(lo, lo, ss);
-            ss = fmaf(hi, hi, ss);
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
       const int64_t row = t * BM + r;
-      if (row < prm.n) prm.norms[row] = sqrtf(ss);
       for (int c = 0; c < nchunk; ++c, ++u) {
         const int buf = (int)(u & 1u);
         if (!mbar_wait(&tfull[buf], (u >> 1) & 1u)) { flag_error(prm.err, 16); ok = false; break; }
         tc_fence_after();
         const int N = min(256, m - 256 * c);
-        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * 256);
-        for (int cb = 0; cb < N / 32; cb += 4) {
+        const int hc = N >> 1;  // columns per half: 128 or 64
+        const uint32_t taddr =
+            tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * 256 + half * hc);
+        if (hc == 128) {
           uint32_t wq[4];
-#pragma unroll
-          for (int k = 0; k < 4; k += 2) {
-            uint32_t v[64];
-            tmem_ld64(taddr + (uint32_t)((cb + k) * 32), v);
-            sign_words2(v, wq[k], wq[k + 1]);
-          }
+          tmem_ld128_pack(taddr, wq);
           if (row < prm.n)
-            *reinterpret_cast<uint4*>(prm.bits + row * W + c * 8 + cb) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+            *reinterpret_cast<uint4*>(prm.bits + row * W + c * 8 + half * 4) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+        } else {
+          uint32_t w0, w1;
+          tmem_ld64_pack(taddr, w0, w1);
+          if (row < prm.n) *reinterpret_cast<uint2*>(prm.bits + row * W + c * 8 + half * 2) = make_uint2(w0, w1);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);
+      }
+    }
+  } else {
+    // norm warps: ||k|| of rows 32*nw + lane and 32*nw + lane + 64 from the swizzled key tile
+    // (16-byte chunk c of row r sits at chunk c ^ (r % 8)); then the stage is
+    // released together with the MMAs' commit
+    const int r0 = (warp - 2 - kEpiWarps) * 32 + lane;  // rows r0 and r0 + 64
+    int s = 0;
+    uint32_t ph = 0;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      if (!mbar_wait(&full[s], ph)) { flag_error(prm.err, 32); break; }
+      const unsigned char* tile = sK + (size_t)s * kStageBytes;
+      float acc[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[j][k] = 0.f;
+#pragma unroll
+      for (int a = 0; a < KA; ++a) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int r = r0 + 64 * j;
+            const uint4 v = *reinterpret_cast<const uint4*>(tile + a * BM * 128 + r * 128 + ((c ^ (r & 7)) << 4));
+            sq_acc_bf16x2(v.x, acc[j][0]);
+            sq_acc_bf16x2(v.y, acc[j][1]);
+            sq_acc_bf16x2(v.z, acc[j][2]);
+            sq_acc_bf16x2(v.w, acc[j][3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int64_t row = t * BM + r0 + 64 * j;
+        if (row < prm.n) prm.norms[row] = sqrtf((acc[j][0] + acc[j][1]) + (acc[j][2] + acc[j][3]));
       }
       if (++s == NS) { s = 0; ph ^= 1u; }
     }
