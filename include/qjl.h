@@ -203,6 +203,38 @@ qjl_status qjl_decode_attention(const qjl_projection* proj, const uint32_t* bits
                                 int64_t N, const float* sq, int q_per_group, float softmax_scale,
                                 float* out, void* ws, size_t ws_bytes, void* stream);
 
+/* Fixed scratch size of qjl_decode_attention_noalloc: 4 MiB per device. */
+#define QJL_DECODE_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * qjl_decode_attention without a caller workspace, for callers that may not
+ * allocate device memory while decoding. Examples: a serving engine whose
+ * own pool owns the whole GPU and forbids raw cudaMalloc so that its
+ * accounting stays exact, or a latency-critical loop that cannot afford
+ * cudaMalloc's implicit device-wide synchronisation. The pages have no
+ * counterpart to this call. It exists only to suit such callers.
+ *
+ * Arguments are those of qjl_decode_attention without ws and ws_bytes. The
+ * split-N workspace comes from a file-scope device array of
+ * QJL_DECODE_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
+ * library holds until exit. The call allocates nothing.
+ *   - Returns QJL_ERR_WORKSPACE, launching nothing, when
+ *     qjl_decode_workspace_bytes(groups, q_per_group, N, d) exceeds that size.
+ *   - The first call on each device resolves the array's device address
+ *     (cudaGetSymbolAddress, with that device current). Make that first call
+ *     before any stream capture.
+ *   - All calls share the one array. Calls that overlap on the GPU (for
+ *     example on two streams) race and give undefined results. Serialise
+ *     them. Earlier calls' contents need no clearing: every workspace entry
+ *     is written before it is read.
+ */
+qjl_status qjl_decode_attention_noalloc(const qjl_projection* proj, const uint32_t* bits,
+                                        const float* norms, const uint32_t* codes,
+                                        const uint16_t* scale, const uint16_t* zero,
+                                        int64_t groups, int64_t N, const float* sq,
+                                        int q_per_group, float softmax_scale, float* out,
+                                        void* stream);
+
 /* Static text for a status code. */
 const char* qjl_status_string(qjl_status s);
 
