@@ -260,7 +260,9 @@ __global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 1) scores_stream_kernel
 // takes a zero C operand. Stages are 512 keys (16 KB of bits at m = 256) and
 // two tiles' MMAs are interleaved per consumer warp.
 constexpr int kDecStageKeys = 512;
-constexpr int kDecTilesPerWarp = kDecStageKeys / 16 / kConsumerWarps;  // 8
+constexpr int kDecConsumers = 8;                                         // consumer warps
+constexpr int kDecThreads = (kDecConsumers + 1) * 32;
+constexpr int kDecTilesPerWarp = kDecStageKeys / 16 / kDecConsumers;    // 4
 
 __device__ __forceinline__ void mma_u8s8_zc(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                             uint32_t b0, uint32_t b1) {
@@ -271,14 +273,14 @@ __device__ __forceinline__ void mma_u8s8_zc(int (&d)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
-template <int W>
-__global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 2) scores_decode_kernel(
+template <int W, bool CLS>
+__global__ void __launch_bounds__(kDecThreads, 2) scores_decode_kernel(
     const uint32_t* __restrict__ bits, const float* __restrict__ norms, const float* __restrict__ sq,
     int64_t G, int64_t N, int J, int NS, float est_scale, int64_t items_per_cta, float* __restrict__ scores,
     int* __restrict__ err) {
   using namespace qjl_sync;
   constexpr int SK = kDecStageKeys;
-  constexpr int KT = 2;
+  constexpr int KT = CLS ? 4 : 2;   // tiles whose MMA chains are interleaved per warp
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* s_inv = reinterpret_cast<float*>(smem_raw);
   float* s_mul = s_inv + 64;
@@ -298,13 +300,13 @@ __global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 2) scores_decode_kernel
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&empty[s], kDecConsumers);
     }
     mbar_fence_init();
   }
   __syncthreads();
 
-  if (warp == kConsumerWarps) {
+  if (warp == kDecConsumers) {
     if (lane == 0) {
       int64_t g = i0 / cpg, c = i0 - (i0 / cpg) * cpg;
       int s = 0;
@@ -340,18 +342,27 @@ __global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 2) scores_decode_kernel
   int s = 0;
   uint32_t ph = 0;
   uint2 breg[W];
-  float mul = 0.f, qs32 = 0.f;
+  float mul = 0.f;
+  int qs32 = 0;
   for (int64_t it = i0; it < i1; ++it) {
     const int64_t n0 = c * SK;
     const int cnt = (int)(N - n0 < SK ? N - n0 : SK);
     if (g != cur_g) {
-      named_sync(1, kConsumerWarps * 32);
-      build_tables<W>(sq + g * (int64_t)J * (32 * W), J, 1, est_scale, s_inv, s_mul, s_qsum, Btab, kConsumerWarps,
-                      1);
+      named_sync(1, kDecConsumers * 32);
+      if constexpr (CLS)
+        build_tables_cls<W>(sq + g * (int64_t)(32 * W), est_scale, s_inv, s_mul, s_qsum, Btab, kDecConsumers, 1);
+      else
+        build_tables<W>(sq + g * (int64_t)J * (32 * W), J, 1, est_scale, s_inv, s_mul, s_qsum, Btab, kDecConsumers,
+                        1);
 #pragma unroll
       for (int mu = 0; mu < W; ++mu) breg[mu] = Btab[mu * 32 + lane];
-      mul = q < J ? s_mul[q] * 0.03125f : 0.f;
-      qs32 = q < J ? 32.f * (float)s_qsum[q] : 0.f;
+      if constexpr (CLS) {
+        mul = s_mul[0] * 0.03125f;
+        qs32 = 32 * s_qsum[0];
+      } else {
+        mul = q < J ? s_mul[q] * 0.03125f : 0.f;
+        qs32 = q < J ? 32 * s_qsum[q] : 0;
+      }
       cur_g = g;
     }
     if (!mbar_wait(&full[s], ph)) { atomicOr(err, 4); break; }
@@ -359,21 +370,21 @@ __global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 2) scores_decode_kernel
     const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
     const uint32_t* sb = sbits + (size_t)s * SK * W;
     const float* sn = snorm + (size_t)s * SK;
-    float* gout = scores + (g * J + q) * N + n0;
+    float* gout = scores + (g * J + (CLS ? 0 : q)) * N + n0;
 #pragma unroll 1
     for (int i = 0; i < kDecTilesPerWarp; i += KT) {
-      const int tile0 = warp + i * kConsumerWarps;
+      const int tile0 = warp + i * kDecConsumers;
       if (tile0 * 16 >= cnt) break;
       int rr[KT][2];
       uint32_t w0[KT][W / 4], w1[KT][W / 4];
 #pragma unroll
       for (int t2 = 0; t2 < KT; ++t2) {
-        rr[t2][0] = (tile0 + t2 * kConsumerWarps) * 16 + gq;
+        rr[t2][0] = (tile0 + t2 * kDecConsumers) * 16 + gq;
         rr[t2][1] = rr[t2][0] + 8;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          // rows past cnt read stale stage data; their results are never stored
-          const uint32_t* src = sb + min(rr[t2][r], SK - 1) * W + q * (W / 4);
+          // rows past cnt (always < SK) read stale stage data; their results are never stored
+          const uint32_t* src = sb + rr[t2][r] * W + q * (W / 4);
 #pragma unroll
           for (int kk = 0; kk < W / 8; ++kk) {
             const uint2 v = *reinterpret_cast<const uint2*>(src + 2 * kk);
@@ -382,6 +393,59 @@ __global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 2) scores_decode_kernel
           }
         }
       }
+      if constexpr (CLS) {
+        // all 8 W/8 MMAs of a tile into one fragment; class Ji lands in column pair Ji
+        int acc[KT][4];
+#pragma unroll
+        for (int p = 0; p < W / 8; ++p) {
+#pragma unroll
+          for (int sh = 0; sh < 2; ++sh) {
+#pragma unroll
+            for (int Ji = 0; Ji < 4; ++Ji) {
+              const uint32_t M = 0x01010101u << (2 * Ji);
+              const uint2 bb = breg[8 * p + 2 * Ji + sh];
+#pragma unroll
+              for (int t2 = 0; t2 < KT; ++t2) {
+                const uint32_t a0 = (w0[t2][2 * p] >> sh) & M, a1 = (w1[t2][2 * p] >> sh) & M;
+                const uint32_t a2 = (w0[t2][2 * p + 1] >> sh) & M, a3 = (w1[t2][2 * p + 1] >> sh) & M;
+                if (p == 0 && sh == 0 && Ji == 0) mma_u8s8_zc(acc[t2], a0, a1, a2, a3, bb.x, bb.y);
+                else mma_u8s8(acc[t2], a0, a1, a2, a3, bb.x, bb.y);
+              }
+            }
+          }
+        }
+        // lane (g, q) holds class q: (hi, lo) of rows g and g + 8. Weight class q by
+        // 4^(3-q) so the sum over the four lanes is 64 * sum b Q, exactly.
+        const int sft = 2 * (3 - q);
+        int v[KT][2];
+#pragma unroll
+        for (int t2 = 0; t2 < KT; ++t2)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            int x = (acc[t2][2 * r] * 256 + acc[t2][2 * r + 1]) << sft;
+            x += __shfl_xor_sync(0xffffffffu, x, 1);
+            x += __shfl_xor_sync(0xffffffffu, x, 2);
+            v[t2][r] = x;
+          }
+        // the quad's KT tiles x 2 rows: lane q finishes tile q (both rows) when
+        // KT == 4, or row (q & 1) of tile (q >> 1) when KT == 2
+#pragma unroll
+        for (int k = 0; k < KT / 2; ++k) {
+          const int t2s = (KT == 4) ? q : (q >> 1);
+          const int rs = (KT == 4) ? k : (q & 1);
+          int mine = v[0][0];
+#pragma unroll
+          for (int t2 = 0; t2 < KT; ++t2)
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+              if (t2 == t2s && r == rs) mine = v[t2][r];
+          const int row = (tile0 + t2s * kDecConsumers) * 16 + gq + 8 * rs;
+          if (row < cnt) {
+            const float nrm = nbulk ? sn[row] : __ldg(nsrc + row);
+            gout[row] = mul * nrm * (float)(mine - qs32);
+          }
+        }
+      } else {
       int acc[KT][4][4];
 #pragma unroll
       for (int p = 0; p < W / 8; ++p) {
@@ -411,10 +475,13 @@ __global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 2) scores_decode_kernel
             const int hi = ((acc[t2][0][2 * r] * 4 + acc[t2][1][2 * r]) * 4 + acc[t2][2][2 * r]) * 4 + acc[t2][3][2 * r];
             const int lo = ((acc[t2][0][2 * r + 1] * 4 + acc[t2][1][2 * r + 1]) * 4 + acc[t2][2][2 * r + 1]) * 4 +
                            acc[t2][3][2 * r + 1];
+            // 32 * sum_i (2 b_i - 1) Q_i, exact in int32 (|.| <= 32 m 32639 < 2^31 for m <= 2048)
+            const int Dq = hi * 256 + lo - qs32;
             const float nrm = nbulk ? sn[row] : __ldg(nsrc + row);
-            gout[row] = mul * nrm * (fmaf((float)hi, 256.f, (float)lo) - qs32);
+            gout[row] = mul * nrm * (float)Dq;
           }
         }
+      }
       }
     }
     __syncwarp();
@@ -482,19 +549,20 @@ qjl_status launch_mma(const qjl_projection* P, const uint32_t* bits, const float
   return qjl_check_launch("scores_stream_kernel");
 }
 
-template <int W>
+template <int W, bool CLS>
 qjl_status launch_decode_fast(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t G,
                               int64_t N, const float* sq, int J, float* scores, cudaStream_t st) {
   const int NS = W == 8 ? 4 : 3;
   const size_t smem = 3 * 64 * 4 + (size_t)W * 32 * sizeof(uint2) + (size_t)NS * kDecStageKeys * (W + 1) * 4 +
                       (size_t)2 * NS * 8;
-  auto kern = scores_decode_kernel<W>;
+  static_assert(kDecTilesPerWarp % 4 == 0, "tiles are consumed in groups of 2 or 4");
+  auto kern = scores_decode_kernel<W, CLS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return qjl_check_launch("scores_decode_kernel smem attribute");
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return qjl_check_launch("scores_decode_kernel attributes");
-  const int regs_per_cta = ((fa.numRegs * 32 + 255) / 256) * 256 * (kThreads / 32);
+  const int regs_per_cta = ((fa.numRegs * 32 + 255) / 256) * 256 * (kDecThreads / 32);
   const int per_sm = std::max(1, std::min(65536 / std::max(regs_per_cta, 1), (int)((228u * 1024u) / (smem + 1024))));
   int* err = qjl_error_flag(P->device);
   if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
@@ -503,8 +571,8 @@ qjl_status launch_decode_fast(const qjl_projection* P, const uint32_t* bits, con
   const int64_t grid = std::min<int64_t>(total, slots);
   const int64_t ipc = (total + grid - 1) / grid;
   const int64_t nblk = (total + ipc - 1) / ipc;
-  qjl_log_launch("scores_decode_kernel", nblk, kThreads, smem, per_sm);
-  kern<<<(unsigned)nblk, kThreads, smem, st>>>(bits, norms, sq, G, N, J, NS, P->est_scale, ipc, scores, err);
+  qjl_log_launch("scores_decode_kernel", nblk, kDecThreads, smem, per_sm);
+  kern<<<(unsigned)nblk, kDecThreads, smem, st>>>(bits, norms, sq, G, N, J, NS, P->est_scale, ipc, scores, err);
   return qjl_check_launch("scores_decode_kernel");
 }
 
@@ -527,8 +595,10 @@ qjl_status launch_scores(const qjl_projection* P, const uint32_t* bits, const fl
   }();
   if (choice == 1 && scores_tc_supported(P->m, J)) return launch_scores_tc(P, bits, norms, G, N, sq, J, scores, st);
   if (choice == 0 && J <= 4 && (P->m == 256 || P->m == 512))
-    return P->m == 256 ? launch_decode_fast<8>(P, bits, norms, G, N, sq, J, scores, st)
-                       : launch_decode_fast<16>(P, bits, norms, G, N, sq, J, scores, st);
+    return P->m == 256 ? (J == 1 ? launch_decode_fast<8, true>(P, bits, norms, G, N, sq, J, scores, st)
+                                 : launch_decode_fast<8, false>(P, bits, norms, G, N, sq, J, scores, st))
+                       : (J == 1 ? launch_decode_fast<16, true>(P, bits, norms, G, N, sq, J, scores, st)
+                                 : launch_decode_fast<16, false>(P, bits, norms, G, N, sq, J, scores, st));
   const int NTR = J > 4 ? 2 : 1;
   switch (scores_mma_supported(P->m) ? P->m : 0) {
     case 256: return NTR == 1 ? launch_mma<8, 1>(P, bits, norms, G, N, sq, J, scores, st)

@@ -111,6 +111,59 @@ __device__ __forceinline__ void load_words(const uint32_t* __restrict__ base, in
 }
 
 
+// Single-query variant of build_tables: the n8 B tile's column pairs carry
+// the four bit-weight classes instead of four queries. Column 2c + h holds the
+// hi (h = 0) or lo (h = 1) byte of Q for the coordinates whose A bytes have
+// weight 4^c, and zero elsewhere. All MMAs of a key tile can then accumulate
+// into one fragment, with class c landing in column pair c.
+template <int W>
+__device__ void build_tables_cls(const float* __restrict__ sqg, float est_scale, float* s_inv, float* s_mul,
+                                 int* s_qsum, uint2* Btab, int nwarps, int bar_id) {
+  constexpr int m = 32 * W;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nthreads = 32 * nwarps;
+  if (warp == 0) {
+    float mx = 0.f;
+    for (int i = lane; i < m; i += 32) mx = fmaxf(mx, fabsf(sqg[i]));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float inv = mx > 0.f ? (float)kQmax / mx : 0.f;
+    int qs = 0;
+    for (int i = lane; i < m; i += 32) qs += quant16(sqg[i], inv);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+    if (lane == 0) {
+      s_inv[0] = inv;
+      s_mul[0] = est_scale * (mx > 0.f ? mx / (float)kQmax : 0.f);
+      s_qsum[0] = qs;
+    }
+  }
+  asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthreads) : "memory");
+  const float inv = s_inv[0];
+  for (int idx = threadIdx.x; idx < W * 32; idx += nthreads) {
+    const int ln = idx & 31, mu = idx >> 5;
+    const int n = ln >> 2, qq = ln & 3;
+    const int cls = n >> 1, half = n & 1;
+    const int p = mu >> 3, jb = mu & 7;  // jb = 2 Ji + s
+    uint32_t b[2] = {0u, 0u};
+    if (cls == (jb >> 1)) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int word = qq * (W / 4) + 2 * p + r;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int Q = quant16(sqg[32 * word + 8 * e + jb], inv);
+          const int lo = (int)(int8_t)(Q & 0xFF);
+          const int hi = (Q - lo) >> 8;
+          b[r] |= ((uint32_t)(half ? lo : hi) & 0xFFu) << (8 * e);
+        }
+      }
+    }
+    Btab[idx] = make_uint2(b[0], b[1]);
+  }
+  asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthreads) : "memory");
+}
+
 // One column tile (4 queries) over a 16-key tile. Thread (g = lane/4,
 // q = lane%4) receives 64 * sum_i b_i hi_i (hi) and 64 * sum_i b_i lo_i (lo)
 // for query q of the column tile and key rows g (r = 0) and g + 8 (r = 1).
