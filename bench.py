@@ -37,13 +37,8 @@ sys.path.insert(0, ROOT)
 METRIC = "QJL decode scores keys/s (HBM GB/s vs ~8 TB/s); key-quantize vectors/s"
 WORKLOAD = "decode_llama7b"
 B, H, N, D, M = 8, 32, 32768, 128, 256
-KEYS = B * H * N
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# algorithmic bytes per key for each kernel of the step
-BYTES_QUANT = D * 2 + M // 8 + 4          # bf16 key in, bits + norm out = 292
-BYTES_SCORE = M // 8 + 4 + 4              # bits + norm in, score out = 40
-FLOP_QUANT = 2 * D * M                    # bf16 contraction per key
 
 
 def peaks():
@@ -245,12 +240,142 @@ def profile_case(case, n):
     return 0
 
 
+class Stage:
+    """One library call of a step: name, callable, units it processes, algorithmic bytes (and flops) per unit."""
+
+    def __init__(self, name, fn, units, bytes_per_unit, flops_per_unit=0, kernel=None, src=None, bound="hbm",
+                 launches=1):
+        self.name, self.fn, self.units, self.launches = name, fn, units, launches
+        self.bytes_per_unit, self.flops_per_unit = bytes_per_unit, flops_per_unit
+        self.kernel, self.src, self.bound = kernel, src, bound
+
+
+def build_workload(name, dev, qjl, wl, torch):
+    """Inputs resident on `dev`, the step's stages, the host-side copies for the e2e leg, and a description."""
+    W = {}
+    if name == "decode_llama7b":
+        P = qjl.Projection(2, D, M, "dense", s_bf16=True)
+        G = B * H
+        keys = wl.llama_keys(dev, B=B, H=H, N=N, d=D).reshape(-1, D)
+        q = wl.llama_queries(dev, B=B, H=H, d=D).reshape(-1, D)
+        bits = torch.empty((G * N, M // 32), dtype=torch.int32, device=dev)
+        norms = torch.empty((G * N,), dtype=torch.float32, device=dev)
+        sq = torch.empty((G, M), dtype=torch.float32, device=dev)
+        out = torch.empty((G, 1, N), dtype=torch.float32, device=dev)
+        stages = [
+            Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), G * N,
+                  2 * D + M // 8 + 4, 2 * D * M, "dense_tc_kernel", "dense_tc.cu"),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * M),
+            Stage("scores", lambda: qjl.scores(P, bits.view(G, N, M // 32), norms.view(G, N), sq.view(G, 1, M), out=out),
+                  G * N, M // 8 + 4 + 4, 0, "scores_decode_kernel", "scores.cu"),
+        ]
+        W.update(units=G * N, unit="keys/s", inputs=[keys, q], outputs=[out], dtype="bf16",
+                 desc="%s: B=%d, heads=%d, N=%d, d=%d, m=%d dense bf16 S; quantize all keys, project 1 query/head, "
+                      "score all keys" % (name, B, H, N, D, M))
+    elif name == "gqa_decode":
+        Bq, Hq, Hkv, Nq, m = 16, 32, 8, 131072, 512
+        G, J = Bq * Hkv, Hq // Hkv
+        P = qjl.Projection(3, D, m, "dense", s_bf16=True)
+        keys = wl.gqa_keys(dev, B=Bq, Hkv=Hkv, N=Nq, d=D).reshape(-1, D)
+        q = wl.gqa_queries(dev, B=Bq, Hq=Hq, d=D).reshape(-1, D)
+        bits = torch.empty((G * Nq, m // 32), dtype=torch.int32, device=dev)
+        norms = torch.empty((G * Nq,), dtype=torch.float32, device=dev)
+        sq = torch.empty((G * J, m), dtype=torch.float32, device=dev)
+        out = torch.empty((G, J, Nq), dtype=torch.float32, device=dev)
+        stages = [
+            Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), G * Nq,
+                  2 * D + m // 8 + 4, 2 * D * m, "dense_tc_kernel", "dense_tc.cu", "tensor"),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G * J, 4 * D + 4 * m),
+            Stage("scores", lambda: qjl.scores(P, bits.view(G, Nq, m // 32), norms.view(G, Nq), sq.view(G, J, m),
+                                               out=out), G * Nq, m // 8 + 4 + 4 * J, 0, "scores_decode_kernel",
+                  "scores.cu"),
+        ]
+        W.update(units=G * Nq, unit="keys/s", inputs=[keys, q], outputs=[out], dtype="bf16",
+                 desc="%s: B=16, 32 query heads over 8 KV heads (4 per KV head), N=131072, d=128, m=512 dense bf16 S; "
+                      "quantize, project, score" % name)
+    elif name == "dense_1head":
+        P = qjl.Projection(1, D, M, "dense", s_bf16=False)
+        keys, q = wl.dense_1head(dev)
+        n, J = keys.shape[0], q.shape[0]
+        bits = torch.empty((n, M // 32), dtype=torch.int32, device=dev)
+        norms = torch.empty((n,), dtype=torch.float32, device=dev)
+        sq = torch.empty((J, M), dtype=torch.float32, device=dev)
+        out = torch.empty((1, J, n), dtype=torch.float32, device=dev)
+        stages = [
+            Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), n, 4 * D + M // 8 + 4,
+                  2 * D * M, "dense_simt_kernel", "dense_simt.cu"),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), J, 4 * D + 4 * M),
+            Stage("scores", lambda: qjl.scores(P, bits.view(1, n, M // 32), norms.view(1, n), sq.view(1, J, M), out=out),
+                  n, M // 8 + 4 + 4 * J, 0, "scores_stream_kernel", "scores.cu"),
+        ]
+        W.update(units=n, unit="keys/s", inputs=[keys, q], outputs=[out], dtype="f32",
+                 desc="%s: 4096 fp32 keys, 16 queries, d=128, m=256 fp32 S (launch-bound)" % name)
+    elif name in ("pfqjl_bulk_m256", "pfqjl_bulk_m1024"):
+        m = 256 if name.endswith("256") else 1024
+        d, n, ns, J = 256, 1 << 24, 1 << 20, 64
+        P = qjl.Projection(4, d, m, "pfqjl")
+        keys = wl.bulk_keys(dev, n=n, d=d)
+        q = wl.bulk_queries(dev, nq=J, d=d)
+        bits = torch.empty((n, m // 32), dtype=torch.int32, device=dev)
+        norms = torch.empty((n,), dtype=torch.float32, device=dev)
+        sq = torch.empty((J, m), dtype=torch.float32, device=dev)
+        out = torch.empty((1, J, ns), dtype=torch.float32, device=dev)
+        stages = [
+            Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), n,
+                  2 * d + m // 8 + 4, 0, "fqjl_kernel", "fqjl.cu", "alu"),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), J, 4 * d + 4 * m),
+            Stage("scores", lambda: qjl.scores(P, bits[:ns].view(1, ns, m // 32), norms[:ns].view(1, ns),
+                                               sq.view(1, J, m), out=out), ns, m // 8 + 4 + 4 * J, 0,
+                  "scores_stream_kernel", "scores.cu"),
+        ]
+        W.update(units=n, unit="vectors/s", inputs=[keys, q], outputs=[out], dtype="bf16",
+                 desc="%s: P-FQJL, 2^24 keys d=256 bf16, m=%d; quantize all, project 64 queries, score the first "
+                      "2^20 keys against them" % (name, m))
+    elif name == "dfqjl_decode":
+        Bd, Hd, Nd, m = 32, 32, 16384, 256
+        G = Bd * Hd
+        P = qjl.Projection(5, D, m, "dfqjl", dither_sigma_rel=0.5)
+        keys, vals = wl.decode_kv(dev, B=Bd, H=Hd, N=Nd, d=D)
+        keys, vals = keys.reshape(-1, D), vals.reshape(-1, D)
+        q = wl.decode_queries(dev, B=Bd, H=Hd, d=D).reshape(-1, D)
+        bits = torch.empty((G * Nd, m // 32), dtype=torch.int32, device=dev)
+        norms = torch.empty((G * Nd,), dtype=torch.float32, device=dev)
+        codes = torch.empty((G * Nd, D // 16), dtype=torch.int32, device=dev)
+        sc = torch.empty((G * Nd, D // 32), dtype=torch.float16, device=dev)
+        zr = torch.empty((G * Nd, D // 32), dtype=torch.float16, device=dev)
+        sq = torch.empty((G, m), dtype=torch.float32, device=dev)
+        out = torch.empty((G, 1, D), dtype=torch.float32, device=dev)
+        ws = torch.empty((qjl.decode_workspace_bytes(G, 1, Nd, D),), dtype=torch.uint8, device=dev)
+        smx = 1.0 / math.sqrt(D)
+        stages = [
+            Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), G * Nd,
+                  2 * D + m // 8 + 4, 0, "fqjl_kernel", "fqjl.cu", "alu"),
+            Stage("quantize_values", lambda: qjl.quantize_values_2bit(vals, codes=codes, scale=sc, zero=zr), G * Nd,
+                  2 * D + D // 4 + D // 8, 0, "values_2bit_kernel", "values.cu"),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * m),
+            Stage("decode_attention", lambda: qjl.decode_attention(
+                P, bits.view(G, Nd, m // 32), norms.view(G, Nd), codes.view(G, Nd, D // 16), sc.view(G, Nd, D // 32),
+                zr.view(G, Nd, D // 32), sq.view(G, 1, m), smx, out=out, workspace=ws), G * Nd,
+                m // 8 + 4 + D // 4 + D // 8, 0, "decode_partial_kernel", "decode.cu", launches=2),
+        ]
+        W.update(units=G * Nd, unit="tokens/s", inputs=[keys, vals, q], outputs=[out], dtype="bf16",
+                 desc="%s: D-FQJL sigma_rel 0.5, B=32, 32 heads, N=16384, d=128, m=256; quantize keys and 2-bit "
+                      "values, project queries, fused softmax(QK)V decode" % name)
+    else:
+        raise SystemExit("unknown workload %s" % name)
+    W["stages"] = stages
+    return W
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=["decode_llama7b", "gqa_decode", "dense_1head", "pfqjl_bulk_m256", "pfqjl_bulk_m1024",
+                             "dfqjl_decode"])
     ap.add_argument("--ref-sample", type=int, default=4096)
     ap.add_argument("--cpu-sample", type=int, default=1 << 18)
     ap.add_argument("--profile-case", default=None,
@@ -274,32 +399,22 @@ def main():
     import bit_kv_cache_qjl_b200 as qjl
     from bit_kv_cache_qjl_b200 import workloads as wl
 
-    P = qjl.Projection(2, D, M, "dense", s_bf16=True)
-    keys = wl.llama_keys(dev, B=B, H=H, N=N, d=D).reshape(-1, D)
-    queries = wl.llama_queries(dev, B=B, H=H, d=D).reshape(-1, D)
-    bits = torch.empty((KEYS, M // 32), dtype=torch.int32, device=dev)
-    norms = torch.empty((KEYS,), dtype=torch.float32, device=dev)
-    sq = torch.empty((B * H, M), dtype=torch.float32, device=dev)
-    out = torch.empty((B * H, 1, N), dtype=torch.float32, device=dev)
+    Wk = build_workload(args.workload, dev, qjl, wl, torch)
+    stages = Wk["stages"]
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
+        for i, st in enumerate(stages):
+            if ev is not None:
+                ev[i].record(stream)
+            st.fn()
         if ev is not None:
-            ev[0].record(stream)
-        qjl.quantize_keys(P, keys, bits=bits, norms=norms)
-        if ev is not None:
-            ev[1].record(stream)
-        qjl.project_queries(P, queries, out=sq)
-        if ev is not None:
-            ev[2].record(stream)
-        qjl.scores(P, bits.view(B * H, N, M // 32), norms.view(B * H, N), sq.view(B * H, 1, M), out=out)
-        if ev is not None:
-            ev[3].record(stream)
+            ev[len(stages)].record(stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
@@ -312,24 +427,25 @@ def main():
     barrier(world)
     ms_total = max_over_ranks(t_start.elapsed_time(t_end), world)
     ms_step = ms_total / args.steps
-    k_quant = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    k_proj = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    k_score = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    value = world * KEYS / (ms_step * 1e-3)
+    k_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(len(stages))]
+    units = Wk["units"]
+    value = world * units / (ms_step * 1e-3)
 
     # end to end through the same calls with host buffers (pinned), copies inside the timed region
-    h_keys = torch.empty((KEYS, D), dtype=torch.bfloat16, pin_memory=True)
-    h_keys.copy_(keys)
-    h_q = torch.empty((B * H, D), dtype=torch.float32, pin_memory=True)
-    h_q.copy_(queries)
-    h_out = torch.empty((B * H, 1, N), dtype=torch.float32, pin_memory=True)
+    h_in = []
+    for t in Wk["inputs"]:
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        h_in.append(h)
+    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in Wk["outputs"]]
     torch.cuda.synchronize()
 
     def e2e_step():
-        keys.copy_(h_keys, non_blocking=True)
-        queries.copy_(h_q, non_blocking=True)
+        for t, h in zip(Wk["inputs"], h_in):
+            t.copy_(h, non_blocking=True)
         step()
-        h_out.copy_(out, non_blocking=True)
+        for t, h in zip(Wk["outputs"], h_out):
+            h.copy_(t, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -341,48 +457,54 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
-    h2d = h_keys.numel() * 2 + h_q.numel() * 4
-    d2h = h_out.numel() * 4
+    h2d = sum(h.numel() * h.element_size() for h in h_in)
+    d2h = sum(h.numel() * h.element_size() for h in h_out)
 
     pk, pk_kind = peaks()
     hbm = pk["hbm_gbs"]
     tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-    q_gbs = KEYS * BYTES_QUANT / (k_quant * 1e-3) / 1e9
-    s_gbs = KEYS * BYTES_SCORE / (k_score * 1e-3) / 1e9
-    q_tflops = KEYS * FLOP_QUANT / (k_quant * 1e-3) / 1e12
-    traffic = ncu_traffic("dense_tc_kernel", WORKLOAD, "dense_tc.cu")
+    kernels = {}
+    for st, ms in zip(stages, k_ms):
+        gbs = st.units * st.bytes_per_unit / (ms * 1e-3) / 1e9
+        e = {"ms": ms, "units_per_s": st.units / (ms * 1e-3), "gbs": gbs, "frac_hbm_measured": gbs / hbm,
+             "frac_8tbs": gbs / 8000.0, "bytes_per_unit": st.bytes_per_unit}
+        if st.flops_per_unit:
+            e["tflops"] = st.units * st.flops_per_unit / (ms * 1e-3) / 1e12
+        kernels[st.name] = e
+    dom = max(range(len(stages)), key=lambda i: k_ms[i])
+    ds = stages[dom]
+    d_gbs = kernels[ds.name]["gbs"]
+    roof = {"bound": "hbm", "kernel": "%s (%s)" % (ds.kernel, ds.name), "achieved": d_gbs, "peak": hbm,
+            "unit": "GB/s", "frac": d_gbs / hbm, "peak_kind": pk_kind,
+            "traffic": ncu_traffic(ds.kernel, args.workload, ds.src) if ds.src else None,
+            "bytes_per_launch": ds.units * ds.bytes_per_unit}
+    if ds.flops_per_unit:
+        roof["tensor_tflops"] = kernels[ds.name]["tflops"]
+        roof["tensor_frac_of_sustained"] = kernels[ds.name]["tflops"] / tf
+    if ds.bound == "alu":
+        roof["note"] = ("the FQJL transform is bound by FP32/shuffle issue, not HBM; frac is the HBM fraction of its "
+                        "algorithmic bytes")
     clocks = clk.summary()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu and args.workload == WORKLOAD:
         rate, dt, threads, k = cpu_oracle_rate(args.cpu_sample)
         cpu = {"value": rate, "unit": "keys/s", "cores": threads, "kind": "oracle",
                "sample": "%d keys of the workload (%d head slices of %d keys): oracle quantize + project + "
                          "score, %.1f s" % (k, max(1, k // N), min(N, k), dt)}
 
     line = {
-        "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": Wk["unit"], "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "%s: B=%d, heads=%d, N=%d, d=%d, m=%d dense bf16 S; quantize all keys, project "
-                               "1 query/head, score all keys" % (WORKLOAD, B, H, N, D, M),
-                   "keys_per_step": KEYS * world, "l2": "inputs larger than L2 (2.15 GB keys/step), no flush",
+        "vs_baseline": None, "dtype": Wk["dtype"], "data": "synthetic",
+        "config": {"workload": Wk["desc"], "units_per_step": units * world,
+                   "l2": "inputs larger than L2 (126 MB) in every step, no flush",
                    "parallelism": "replicas (weak)" if world > 1 else "single GPU"},
-        "roofline": {"bound": "hbm", "kernel": "dense_tc_kernel (key quantize)", "achieved": q_gbs,
-                     "peak": hbm, "unit": "GB/s", "frac": q_gbs / hbm, "peak_kind": pk_kind,
-                     "traffic": traffic,
-                     "bytes_per_launch": KEYS * BYTES_QUANT, "tensor_tflops": q_tflops,
-                     "tensor_frac_of_sustained": q_tflops / tf},
-        "kernels": {
-            "quantize_keys": {"ms": k_quant, "vectors_per_s": KEYS / (k_quant * 1e-3), "gbs": q_gbs,
-                              "frac_hbm_measured": q_gbs / hbm, "frac_8tbs": q_gbs / 8000.0},
-            "project_queries": {"ms": k_proj},
-            "scores": {"ms": k_score, "keys_per_s": KEYS / (k_score * 1e-3), "gbs": s_gbs,
-                       "frac_hbm_measured": s_gbs / hbm, "frac_8tbs": s_gbs / 8000.0},
-        },
-        "e2e": {"value": world * KEYS / (e2e_ms * 1e-3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
+        "roofline": roof,
+        "kernels": kernels,
+        "e2e": {"value": world * units / (e2e_ms * 1e-3), "unit": Wk["unit"], "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": sum(st.launches for st in stages) * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

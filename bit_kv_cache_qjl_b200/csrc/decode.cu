@@ -27,11 +27,13 @@
 #include <stdint.h>
 
 #include "qjl_internal.h"
+#include "mbarrier.cuh"
 #include "sign_mma.cuh"
 
 namespace {
 
 using namespace qjl_sign;
+using qjl_sync::named_sync;
 constexpr int kWarps = 4;
 constexpr int kMaxJ = 4;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -211,6 +213,332 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partial_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Streaming fused decode for one query per group (the decode step proper).
+// Each CTA owns one split of one group. A producer lane moves 512-token
+// stages (bits, norms, codes, scales, zeros) into a shared-memory ring with
+// cp.async.bulk. Eight consumer warps take 64 tokens each per stage:
+//   * estimates by the class-in-column s8 MMAs (one fragment per tile, two
+//     xor-shuffles merge the four weight classes; each lane ends with the
+//     logits of 2 tokens);
+//   * an online softmax per warp (base 2);
+//   * p * v_hat accumulated per lane for its d/32 channels, which lie in one
+//     32-channel group: acc_c += (p s) (code_c 4^c) and accz += p z. The
+//     term code_c 4^c comes out exactly as (word & (3 << 2c)) | 2^23 - 2^23,
+//     with no shift and no int-to-float conversion, and the 4^c is divided
+//     out once at the end.
+// The warps are merged in shared memory into one (max, sum, acc[d]) partial.
+constexpr int kDsConsumers = 8;
+constexpr int kDsThreads = (kDsConsumers + 1) * 32;
+constexpr int kDsStage = 512;
+
+__device__ __forceinline__ void mma_u8s8_acc(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_u8s8_zero(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};\n"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
+
+// acc_c += (p s) (code_c 4^c) for this lane's CPL channels and accz += p z.
+// code_c 4^c = float(2^23 | (cwd & (3 << 2c))) - 2^23 exactly (the bits sit in
+// the mantissa), so no shift or int-to-float conversion is needed. Channel
+// pairs go through sm_100's packed fp32 subtract and FMA.
+template <int CPL>
+__device__ __forceinline__ void pv_accum(uint32_t cwd, uint16_t sraw, uint16_t zraw, float pt, float (&acc)[CPL],
+                                         float& accz) {
+  const float pw = pt * __half2float(__ushort_as_half(sraw));
+  accz = fmaf(pt, __half2float(__ushort_as_half(zraw)), accz);
+  if constexpr (CPL == 1) {
+    acc[0] = fmaf(pw, __uint_as_float(0x4B000000u | (cwd & 3u)) - 8388608.f, acc[0]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < CPL; c += 2) {
+      const uint32_t u0 = 0x4B000000u | (cwd & (3u << (2 * c)));
+      const uint32_t u1 = 0x4B000000u | (cwd & (3u << (2 * c + 2)));
+      asm("{\n\t.reg .b64 f, m, w, a;\n\t"
+          "mov.b64 f, {%2, %3};\n\t"
+          "mov.b64 m, {%4, %4};\n\t"
+          "sub.rn.f32x2 f, f, m;\n\t"
+          "mov.b64 w, {%5, %5};\n\t"
+          "mov.b64 a, {%0, %1};\n\t"
+          "fma.rn.f32x2 a, w, f, a;\n\t"
+          "mov.b64 {%0, %1}, a;\n\t}"
+          : "+f"(acc[c]), "+f"(acc[c + 1])
+          : "r"(u0), "r"(u1), "f"(8388608.f), "f"(pw));
+    }
+  }
+}
+
+struct DsLayout {
+  // byte offsets inside one stage
+  uint32_t bits, norms, codes, scale, zero, bytes;
+};
+
+__host__ __device__ inline DsLayout ds_layout(int W, int d) {
+  DsLayout L;
+  L.bits = 0;
+  L.norms = L.bits + kDsStage * W * 4;
+  L.codes = L.norms + kDsStage * 4;
+  L.scale = L.codes + kDsStage * (d / 16) * 4;
+  L.zero = L.scale + kDsStage * (d / 32) * 2;
+  L.bytes = L.zero + kDsStage * (d / 32) * 2;
+  return L;
+}
+
+__device__ __forceinline__ bool bulk_ok(const void* src, uint32_t bytes) {
+  return (((uintptr_t)src & 15u) == 0) && (bytes % 16u == 0);
+}
+
+template <int W, int CPL>
+__global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
+    const uint32_t* __restrict__ bits, const float* __restrict__ norms, const uint32_t* __restrict__ codes,
+    const uint16_t* __restrict__ scale, const uint16_t* __restrict__ zero, const float* __restrict__ sq, int64_t N,
+    int NS, float est_scale, float logit_scale, int64_t tokens_per_cta, float* __restrict__ ws,
+    int* __restrict__ err) {
+  using namespace qjl_sync;
+  constexpr int d = 32 * CPL;
+  constexpr int CW = d / 16;  // code words per token
+  constexpr int GW = d / 32;  // scale / zero halves per token
+  constexpr int KT = 4;       // 16-token tiles per warp per stage
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* s_inv = reinterpret_cast<float*>(smem_raw);
+  float* s_mul = s_inv + 64;
+  int* s_qsum = reinterpret_cast<int*>(s_mul + 64);
+  uint2* Btab = reinterpret_cast<uint2*>(smem_raw + 3 * 64 * 4);
+  float* s_red = reinterpret_cast<float*>(Btab + W * 32);                      // [kDsConsumers][d + 2]
+  unsigned char* ring = reinterpret_cast<unsigned char*>(s_red + kDsConsumers * (d + 2));
+  const DsLayout L = ds_layout(W, d);
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + (size_t)NS * L.bytes);
+  uint64_t* empty = full + NS;
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t gi = blockIdx.y;
+  const int64_t t0 = (int64_t)blockIdx.x * tokens_per_cta;
+  const int64_t t1 = min(N, t0 + tokens_per_cta);
+  const int64_t nst = (t1 - t0 + kDsStage - 1) / kDsStage;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kDsConsumers);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == kDsConsumers) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      for (int64_t k = 0; k < nst; ++k, ++issued) {
+        if (!mbar_wait(&empty[s], ph ^ 1u)) { atomicOr(err, 1); break; }
+        const int64_t n0 = t0 + k * kDsStage;
+        const uint32_t cnt = (uint32_t)(t1 - n0 < kDsStage ? t1 - n0 : kDsStage);
+        const int64_t row = gi * N + n0;
+        unsigned char* st = ring + (size_t)s * L.bytes;
+        const void* src[5] = {bits + row * W, norms + row, codes + row * CW, scale + row * GW, zero + row * GW};
+        const uint32_t nb[5] = {cnt * W * 4, cnt * 4, cnt * CW * 4, cnt * GW * 2, cnt * GW * 2};
+        const uint32_t off[5] = {L.bits, L.norms, L.codes, L.scale, L.zero};
+        uint32_t tx = 0;
+        for (int a = 0; a < 5; ++a)
+          if (bulk_ok(src[a], nb[a])) tx += nb[a];
+        mbar_expect_tx(&full[s], tx);
+        for (int a = 0; a < 5; ++a)
+          if (bulk_ok(src[a], nb[a])) bulk_g2s(st + off[a], src[a], nb[a], &full[s]);
+        if (++s == NS) { s = 0; ph ^= 1u; }
+      }
+      const int used = issued < NS ? (int)issued : NS;
+      for (int j = 0; j < used; ++j) {
+        int stg = s - 1 - j;
+        uint32_t p = ph;
+        if (stg < 0) { stg += NS; p ^= 1u; }
+        if (!mbar_wait(&full[stg], p)) atomicOr(err, 2);
+      }
+    }
+    return;
+  }
+
+  // consumers
+  build_tables_cls<W>(sq + gi * (int64_t)(32 * W), est_scale, s_inv, s_mul, s_qsum, Btab, kDsConsumers, 1);
+  uint2 breg[W];
+#pragma unroll
+  for (int mu = 0; mu < W; ++mu) breg[mu] = Btab[mu * 32 + lane];
+  const float xmul = s_mul[0] * 0.03125f * logit_scale * 1.4426950408889634f;  // to log2-domain logits
+  const int qs32 = 32 * s_qsum[0];
+  const int gq = lane >> 2, q = lane & 3;
+  const int c0 = lane * CPL;
+  const int grp = c0 >> 5, cw = c0 >> 4, cshift = 2 * (c0 & 15);
+
+  float m_run = -INFINITY, l_lane = 0.f, accz = 0.f, acc[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
+  bool ok = true;
+  int s = 0;
+  uint32_t ph = 0;
+  for (int64_t k = 0; k < nst; ++k) {
+    const int64_t n0 = t0 + k * kDsStage;
+    const int cnt = (int)(t1 - n0 < kDsStage ? t1 - n0 : kDsStage);
+    const int64_t row0 = gi * N + n0;
+    if (!mbar_wait(&full[s], ph)) { atomicOr(err, 4); ok = false; break; }
+    const unsigned char* st = ring + (size_t)s * L.bytes;
+    const uint32_t* sb = reinterpret_cast<const uint32_t*>(st + L.bits);
+    const bool nb_norm = bulk_ok(norms + row0, (uint32_t)cnt * 4);
+    const bool nb_codes = bulk_ok(codes + row0 * CW, (uint32_t)cnt * CW * 4);
+    const bool nb_scale = bulk_ok(scale + row0 * GW, (uint32_t)cnt * GW * 2);
+    const bool nb_zero = bulk_ok(zero + row0 * GW, (uint32_t)cnt * GW * 2);
+    const float* snorm = reinterpret_cast<const float*>(st + L.norms);
+    const uint32_t* scodes = reinterpret_cast<const uint32_t*>(st + L.codes);
+    const uint16_t* sscale = reinterpret_cast<const uint16_t*>(st + L.scale);
+    const uint16_t* szero = reinterpret_cast<const uint16_t*>(st + L.zero);
+
+    // ---- estimates of this warp's KT tiles (tiles warp + 8 t2)
+    uint32_t w0[KT][W / 4], w1[KT][W / 4];
+#pragma unroll
+    for (int t2 = 0; t2 < KT; ++t2) {
+      const int rA = (warp + t2 * kDsConsumers) * 16 + gq;
+#pragma unroll
+      for (int kk = 0; kk < W / 8; ++kk) {
+        const uint2 a = *reinterpret_cast<const uint2*>(sb + rA * W + q * (W / 4) + 2 * kk);
+        const uint2 b = *reinterpret_cast<const uint2*>(sb + (rA + 8) * W + q * (W / 4) + 2 * kk);
+        w0[t2][2 * kk] = a.x; w0[t2][2 * kk + 1] = a.y;
+        w1[t2][2 * kk] = b.x; w1[t2][2 * kk + 1] = b.y;
+      }
+    }
+    int accm[KT][4];
+#pragma unroll
+    for (int p = 0; p < W / 8; ++p) {
+#pragma unroll
+      for (int sh = 0; sh < 2; ++sh) {
+#pragma unroll
+        for (int Ji = 0; Ji < 4; ++Ji) {
+          const uint32_t M = 0x01010101u << (2 * Ji);
+          const uint2 bb = breg[8 * p + 2 * Ji + sh];
+#pragma unroll
+          for (int t2 = 0; t2 < KT; ++t2) {
+            const uint32_t a0 = (w0[t2][2 * p] >> sh) & M, a1 = (w1[t2][2 * p] >> sh) & M;
+            const uint32_t a2 = (w0[t2][2 * p + 1] >> sh) & M, a3 = (w1[t2][2 * p + 1] >> sh) & M;
+            if (p == 0 && sh == 0 && Ji == 0) mma_u8s8_zero(accm[t2], a0, a1, a2, a3, bb.x, bb.y);
+            else mma_u8s8_acc(accm[t2], a0, a1, a2, a3, bb.x, bb.y);
+          }
+        }
+      }
+    }
+    // lane q of quad gq ends with tile t2 = q, rows gq (r = 0) and gq + 8 (r = 1)
+    const int sft = 2 * (3 - q);
+    float x[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      int mine = 0;
+#pragma unroll
+      for (int t2 = 0; t2 < KT; ++t2) {
+        int v = (accm[t2][2 * r] * 256 + accm[t2][2 * r + 1]) << sft;
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        if (t2 == q) mine = v;
+      }
+      const int row = (warp + q * kDsConsumers) * 16 + gq + 8 * r;
+      if (row < cnt) {
+        const float nrm = nb_norm ? snorm[row] : __ldg(norms + row0 + row);
+        x[r] = xmul * nrm * (float)(mine - qs32);
+      } else {
+        x[r] = -INFINITY;
+      }
+    }
+    // ---- online softmax over the warp's 64 tokens
+    float mt = fmaxf(x[0], x[1]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+    const float mn = fmaxf(m_run, mt);
+    if (mn != -INFINITY) {
+      const float corr = exp2f(m_run - mn);
+      m_run = mn;
+      l_lane *= corr;
+      accz *= corr;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) acc[c] *= corr;
+      const float p0 = exp2f(x[0] - mn), p1 = exp2f(x[1] - mn);
+      l_lane += p0 + p1;
+      // ---- p * v_hat: token (tile t2, row) is held by lane 4 (row % 8) + t2, register row / 8
+      if (cnt == kDsStage && nb_codes && nb_scale && nb_zero) {
+        // whole stage in shared memory: no per-token bounds or source selection
+        const uint32_t* cp = scodes + cw;
+        const uint16_t* sp = sscale + grp;
+        const uint16_t* zp = szero + grp;
+#pragma unroll 1
+        for (int t2 = 0; t2 < KT; ++t2) {
+          const int tb = (warp + t2 * kDsConsumers) * 16;
+#pragma unroll
+          for (int row = 0; row < 16; ++row) {
+            const int tok = tb + row;
+            const float pt = __shfl_sync(0xffffffffu, row < 8 ? p0 : p1, 4 * (row & 7) + t2);
+            pv_accum<CPL>(cp[tok * CW] >> cshift, sp[tok * GW], zp[tok * GW], pt, acc, accz);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int t2 = 0; t2 < KT; ++t2) {
+#pragma unroll
+          for (int row = 0; row < 16; ++row) {
+            const int tok = (warp + t2 * kDsConsumers) * 16 + row;
+            const float pt = __shfl_sync(0xffffffffu, row < 8 ? p0 : p1, 4 * (row & 7) + t2);
+            if (tok >= cnt) continue;
+            const uint32_t cwd = (nb_codes ? scodes[tok * CW + cw] : __ldg(codes + (row0 + tok) * CW + cw)) >> cshift;
+            const uint16_t sr = nb_scale ? sscale[tok * GW + grp] : __ldg(scale + (row0 + tok) * GW + grp);
+            const uint16_t zr = nb_zero ? szero[tok * GW + grp] : __ldg(zero + (row0 + tok) * GW + grp);
+            pv_accum<CPL>(cwd, sr, zr, pt, acc, accz);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == NS) { s = 0; ph ^= 1u; }
+  }
+  if (!ok) return;
+
+  // ---- merge the consumer warps: (m, l, acc[d]) per warp, then one partial per CTA
+  float l_w = l_lane;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) l_w += __shfl_xor_sync(0xffffffffu, l_w, o);
+  float* red = s_red + warp * (d + 2);
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) red[2 + c0 + c] = acc[c] * (1.0f / (float)(1 << (2 * c))) + accz;
+  if (lane == 0) {
+    red[0] = m_run;
+    red[1] = l_w;
+  }
+  named_sync(1, kDsConsumers * 32);
+  const int64_t split = blockIdx.x;
+  const int64_t nsplit = gridDim.x;
+  for (int idx = threadIdx.x; idx < d + 2; idx += kDsConsumers * 32) {
+    float M = -INFINITY;
+    for (int w = 0; w < kDsConsumers; ++w) M = fmaxf(M, s_red[w * (d + 2)]);
+    float v = 0.f;
+    if (idx == 0) {
+      v = M;
+    } else {
+      for (int w = 0; w < kDsConsumers; ++w) {
+        const float mw = s_red[w * (d + 2)];
+        const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+        v += f * s_red[w * (d + 2) + idx];
+      }
+    }
+    ws[(gi * nsplit + split) * (d + 2) + idx] = v;
+  }
+}
+
 // out[g][j][c] = sum_s acc_s[c] 2^(m_s - M) / sum_s l_s 2^(m_s - M)
 __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ ws, int64_t G,
                                                              int J, int d, int64_t nsplit,
@@ -261,11 +589,52 @@ qjl_status launch_wc(const qjl_projection* P, const uint32_t* bits, const float*
   return qjl_check_launch("decode_combine_kernel");
 }
 
+template <int W, int CPL>
+qjl_status launch_stream(const qjl_projection* P, const uint32_t* bits, const float* norms, const uint32_t* codes,
+                         const uint16_t* scale, const uint16_t* zero, int64_t G, int64_t N, const float* sq,
+                         float softmax_scale, float* out, float* ws, cudaStream_t st) {
+  constexpr int d = 32 * CPL;
+  const DsLayout L = ds_layout(W, d);
+  int NS = 4;  // one CTA per SM: about 168 KB in flight at d = 128, m = 256
+  while (NS > 2 && 3 * 64 * 4 + (size_t)W * 32 * sizeof(uint2) + (size_t)kDsConsumers * (d + 2) * 4 +
+                       (size_t)NS * L.bytes + (size_t)2 * NS * 8 > 220 * 1024)
+    --NS;
+  const size_t smem = 3 * 64 * 4 + (size_t)W * 32 * sizeof(uint2) + (size_t)kDsConsumers * (d + 2) * 4 +
+                      (size_t)NS * L.bytes + (size_t)2 * NS * 8;
+  auto kern = decode_stream_kernel<W, CPL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+    return qjl_check_launch("decode_stream_kernel smem attribute");
+  int* err = qjl_error_flag(P->device);
+  if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  const int64_t splits = decode_splits(G, N);
+  const int64_t ntiles = (N + 15) / 16;
+  const int64_t tpc = 16 * ((ntiles + splits - 1) / splits);  // tokens per CTA, as the tile-based kernel splits
+  const int64_t nsplit = (N + tpc - 1) / tpc;
+  if (nsplit != splits) return qjl_set_error(QJL_ERR_UNSUPPORTED, "internal split mismatch");
+  dim3 grid((unsigned)splits, (unsigned)G);
+  qjl_log_launch("decode_stream_kernel", (int64_t)splits * G, kDsThreads, smem, 1);
+  kern<<<grid, kDsThreads, smem, st>>>(bits, norms, codes, scale, zero, sq, N, NS, P->est_scale, softmax_scale, tpc,
+                                       ws, err);
+  qjl_status s = qjl_check_launch("decode_stream_kernel");
+  if (s != QJL_OK) return s;
+  decode_combine_kernel<<<(unsigned)G, 128, 0, st>>>(ws, G, 1, d, splits, out);
+  return qjl_check_launch("decode_combine_kernel");
+}
+
 template <int W>
 qjl_status launch_w(const qjl_projection* P, const uint32_t* bits, const float* norms,
                     const uint32_t* codes, const uint16_t* scale, const uint16_t* zero, int64_t G,
                     int64_t N, const float* sq, int J, float softmax_scale, float* out, float* ws,
                     cudaStream_t st) {
+  if (J == 1) {
+    switch (P->d) {
+      case 32: return launch_stream<W, 1>(P, bits, norms, codes, scale, zero, G, N, sq, softmax_scale, out, ws, st);
+      case 64: return launch_stream<W, 2>(P, bits, norms, codes, scale, zero, G, N, sq, softmax_scale, out, ws, st);
+      case 128: return launch_stream<W, 4>(P, bits, norms, codes, scale, zero, G, N, sq, softmax_scale, out, ws, st);
+      case 256: return launch_stream<W, 8>(P, bits, norms, codes, scale, zero, G, N, sq, softmax_scale, out, ws, st);
+    }
+  }
   switch (P->d) {
     case 32: return launch_wc<W, 1>(P, bits, norms, codes, scale, zero, G, N, sq, J, softmax_scale, out, ws, st);
     case 64: return launch_wc<W, 2>(P, bits, norms, codes, scale, zero, G, N, sq, J, softmax_scale, out, ws, st);

@@ -64,11 +64,13 @@ def test_values_and_decode_kernels(cuda_ok):
     v = wl.normal((2 * 300, 128), 4, "cuda", torch.bfloat16)
     bits = torch.zeros((2, 300, 8), dtype=torch.int32, device="cuda")
     norms = torch.ones((2, 300), device="cuda")
-    sq = torch.ones((2, 1, 256), device="cuda")
 
-    def run():
+    def run(J):
+        sq = torch.ones((2, J, 256), device="cuda")
         c, s, z = qjl.quantize_values_2bit(v)
         qjl.decode_attention(P, bits, norms, c.view(2, 300, 8), s.view(2, 300, 4), z.view(2, 300, 4), sq, 0.1)
-    names = _kernels(run)
-    for k in ("values_2bit_kernel", "decode_partial_kernel", "decode_combine_kernel"):
+    names = _kernels(lambda: run(1))
+    for k in ("values_2bit_kernel", "decode_stream_kernel", "decode_combine_kernel"):
         assert _has(names, k), (k, names)
+    # several queries per group take the tile-per-warp kernel
+    assert _has(_kernels(lambda: run(2)), "decode_partial_kernel")

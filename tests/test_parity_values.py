@@ -36,3 +36,20 @@ def test_values_constant_groups(cuda_ok):
     torch.cuda.synchronize()
     assert torch.all(codes == 0) and torch.all(scale == 0)
     assert torch.equal(zero.float().cpu(), torch.tensor([[0, 0], [2.5, 2.5], [-1.0, 0.0]]))
+
+
+def test_values_exact_ties(cuda_ok):
+    """Values at exact half-levels (t = 0.5, 1.5, 2.5) go through the exact-division
+    fallback; round-half-even must agree with the oracle bit for bit."""
+    base = torch.tensor([0.0, 3.0, 0.5, 1.5, 2.5, 1.0, 2.0, 0.75], dtype=torch.float32)
+    rows = []
+    for scale in (1.0, 0.5, 2.0, 0.25, 3.0, 0.125):
+        rows.append((base.repeat(4) * scale + (scale * 7 if scale > 1 else 0.0)))
+    v = torch.stack(rows).to(torch.bfloat16).repeat(1, 4).cuda()        # [6, 128]
+    codes, scale, zero = quantize_values_2bit(v)
+    torch.cuda.synchronize()
+    oc, os_, oz = oracle.kivi.quantize_values_2bit(host(v).astype(np.float32))
+    assert np.array_equal(host(codes), oc)
+    assert np.array_equal(scale.cpu().numpy().view(np.uint16), os_.view(np.uint16))
+    # the ties really occur: some codes round half to even
+    assert (oracle.kivi.unpack_codes(oc, 128) == 2).any()
