@@ -356,7 +356,7 @@ def build_workload(name, dev, qjl, wl, torch):
             Stage("decode_attention", lambda: qjl.decode_attention(
                 P, bits.view(G, Nd, m // 32), norms.view(G, Nd), codes.view(G, Nd, D // 16), sc.view(G, Nd, D // 32),
                 zr.view(G, Nd, D // 32), sq.view(G, 1, m), smx, out=out, workspace=ws), G * Nd,
-                m // 8 + 4 + D // 4 + D // 8, 0, "decode_partial_kernel", "decode.cu", launches=2),
+                m // 8 + 4 + D // 4 + D // 8, 0, "decode_stream_kernel", "decode.cu", launches=2),
         ]
         W.update(units=G * Nd, unit="tokens/s", inputs=[keys, vals, q], outputs=[out], dtype="bf16",
                  desc="%s: D-FQJL sigma_rel 0.5, B=32, 32 heads, N=16384, d=128, m=256; quantize keys and 2-bit "
