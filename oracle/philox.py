@@ -35,7 +35,7 @@ MASK32 = 0xFFFFFFFF
 STREAM_GAUSS = 0       # dense S entries, Gaussian diagonal D_g
 STREAM_RADEMACHER = 1  # Rademacher diagonal D_r
 STREAM_PERM = 2        # Fisher-Yates draws for the permutation Pi
-STREAM_DITHER = 3      # D-FQJL dither, one per (token, coordinate)
+STREAM_DITHER = 3      # D-FQJL dither, one block per (token, 4 coordinates)
 
 
 def _u32(x):
@@ -80,6 +80,21 @@ def box_muller(x0, x1):
     u0 = uniform_open01(x0)
     u1 = uniform_open01(x1)
     return np.sqrt(-2.0 * np.log(u0)) * np.cos(2.0 * np.pi * u1)
+
+
+def box_muller_pair23(xr, xa):
+    """Two independent standard normals from two words, on 23-bit draws (fp64).
+
+    The radius draw is u = ((xr >> 9) + 1/2) / 2^23, in (0, 1). The angle draw
+    is v = (xa >> 9) / 2^23, in [0, 1). The pair is sqrt(-2 ln u) times
+    (cos 2 pi v, sin 2 pi v). These are the two outputs of Box and Muller,
+    "A Note on the Generation of Random Normal Deviates" (1958), and they are
+    independent N(0, 1).
+    """
+    u = (np.asarray(xr, dtype=np.uint64) >> np.uint64(9)).astype(np.float64) * 2.0 ** -23 + 2.0 ** -24
+    v = (np.asarray(xa, dtype=np.uint64) >> np.uint64(9)).astype(np.float64) * 2.0 ** -23
+    r = np.sqrt(-2.0 * np.log(u))
+    return r * np.cos(2.0 * np.pi * v), r * np.sin(2.0 * np.pi * v)
 
 
 def gaussian(seed, c0, c1, c2, stream):

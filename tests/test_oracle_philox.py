@@ -133,3 +133,38 @@ def test_dither_depends_on_absolute_token():
     assert np.array_equal(a[1:], b)
     big = P.dither(9, 16, 32, [(1 << 32) + 10])
     assert not np.array_equal(big[0], a[0])
+
+
+def test_dither_is_standard_normal_per_coordinate():
+    xi = P.dither(21, 64, 128, np.arange(4000))
+    for j in range(4):     # each of the four coordinates one block yields
+        col = xi[:, j::4].ravel()
+        assert scipy.stats.kstest(col, "norm").pvalue > 1e-4
+    # variance 1 to within the sampling error of 512000 draws
+    assert abs(xi.var() - 1.0) < 0.01
+
+
+def test_dither_pairs_are_independent_normals():
+    """A Box-Muller pair is two independent N(0,1): its squared radius is
+    chi-square with 2 degrees of freedom, and any rotation of the pair is
+    again standard normal. Pairs from different words of one block do not
+    correlate."""
+    xi = P.dither(22, 32, 64, np.arange(5000)).reshape(-1, 4)
+    for a, b in ((0, 1), (2, 3)):
+        r2 = xi[:, a] ** 2 + xi[:, b] ** 2
+        assert scipy.stats.kstest(r2, "chi2", args=(2,)).pvalue > 1e-4
+        rot = (xi[:, a] + xi[:, b]) / math.sqrt(2.0)
+        assert scipy.stats.kstest(rot, "norm").pvalue > 1e-4
+    c = np.corrcoef(xi.T)
+    assert np.max(np.abs(c - np.eye(4))) < 0.02
+
+
+def test_dither_prefix_and_block_structure():
+    """Coordinates come in fours from one block: the dither of the first m'
+    coordinates does not depend on m, and neither on d."""
+    a = P.dither(23, 32, 64, [5, 6])
+    b = P.dither(23, 64, 256, [5, 6])
+    assert np.array_equal(a, b[:, :64])
+    assert np.all(np.isfinite(b))
+    # the radius draw is never 0 or 1: |xi| is bounded by sqrt(-2 ln 2^-24)
+    assert np.max(np.abs(P.dither(24, 128, 1024, np.arange(500)))) < math.sqrt(2 * 24 * math.log(2)) + 1e-9
