@@ -1,0 +1,571 @@
+// D-FQJL / P-FQJL key sketch: bits and norms by two fast Walsh-Hadamard
+// transforms per block.
+//
+// "Fast Quantized Johnson - Lindenstrauss Transforms" ("In short", "Key
+// concepts", "The paper" abstract): the dense Gaussian projection is replaced
+// by two randomized Hadamard transforms with a Gaussian diagonal in the second
+// stage, at O(d log d) per vector. P-FQJL puts a uniform random permutation
+// between the Hadamard stages. D-FQJL adds Gaussian dither before the sign
+// ("Transcript: The paper's improvements"). For block b of the m/d stacked
+// blocks, with H the unnormalised Sylvester matrix:
+//   y = H D_g Pi H D_r x            (default; sqrt(d) H_n D_g Pi H_n D_r x times sqrt(d))
+//   y = D_g H Pi H D_r x            (dg_outer, the literal order)
+// and the stored bit is [y + sqrt(d) sigma_rel ||x|| xi >= 0] (the positive
+// factor sqrt(d) between y and the normalised map does not move a sign).
+// The dither xi for coordinate e = b*d + i of token t comes four coordinates
+// to a Philox4x32-10 block at counter (e/4, t_lo, t_hi, 3): Box-Muller on
+// 23-bit draws, cos and sin outputs, from words (0,1) and (2,3).
+//
+// Work split. A thread holds E = min(d, 128) elements of one key in registers
+// as E/2 packed pairs V[t] = (v_t, v_{t+E/2}), so most butterflies are sm_100
+// packed-fp32 add/sub. L = d/E lanes share a key (1 for d <= 128, else 2, 4
+// or 8), K = 32/L keys per warp. Butterflies on register bits need no data
+// movement. Butterflies on lane bits are one shfl_xor and one packed FMA.
+// Two element orders are used:
+//   layout A (first transform)  : i = (s>>1)*2E + 2r + (s&1)   (i = r if L = 1)
+//   layout B (second transform) : i = s*E + r
+// where s is the lane within the key and r the register index. Layout A lets
+// the L lanes of a key read the same staged words (broadcast, no bank
+// conflict). Layout B gives each lane E consecutive output bits, which
+// funnel-shift into whole words. The permutation gather between the two
+// transforms also switches layout. It goes through a per-warp shared buffer
+// in which element j of key slot k sits at word K*(j + 2*(j / 2E)) + k. The
+// writes from layout A are conflict-free; the gather reads are at
+// precomputed offsets.
+//
+// Keys reach shared memory by cp.async.bulk (the API requires 16-byte aligned
+// rows), one copy per key row segment, into segments padded by 16 bytes so
+// that the register loads are conflict-free. Each warp prefetches its next
+// batch of K keys while it transforms the current one. Per-block tables (D_r and D_g as register
+// pairs, gather offsets) are staged once per CTA.
+//
+// No output bit can come from a -0: D_g is applied as fma(u, g, +0), which
+// maps an exact zero product to +0, and sums of values that are not -0 are
+// not -0. So the sign bit of y is exactly [y < 0].
+
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "mbarrier.cuh"
+#include "philox.h"
+#include "qjl_internal.h"
+
+namespace {
+
+using qjl_sync::bulk_g2s;
+using qjl_sync::mbar_expect_tx;
+using qjl_sync::mbar_fence_init;
+using qjl_sync::mbar_init;
+using qjl_sync::mbar_wait;
+using qjl_sync::smem_u32;
+
+constexpr int kMaxWarps = 8;
+constexpr size_t kTableBudget = 24 * 1024;   // shared bytes for the per-block tables of one launch
+constexpr size_t kSmemLimit = 227 * 1024;
+
+enum { MODE_P = 0, MODE_D = 1 };
+
+// ---- packed fp32 pair arithmetic (sm_100 f32x2) ----------------------------------------------
+
+// (a, b) <- (a + b, a - b), both lanes of the pair
+__device__ __forceinline__ void bfly2(float2& a, float2& b) {
+  asm("{\n\t.reg .b64 x, y, s, d;\n\t"
+      "mov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "add.rn.f32x2 s, x, y;\n\tsub.rn.f32x2 d, x, y;\n\t"
+      "mov.b64 {%0, %1}, s;\n\tmov.b64 {%2, %3}, d;\n\t}"
+      : "+f"(a.x), "+f"(a.y), "+f"(b.x), "+f"(b.y));
+}
+
+// a <- a * b
+__device__ __forceinline__ void mul2(float2& a, float2 b) {
+  asm("{\n\t.reg .b64 x, y;\n\t"
+      "mov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "mul.rn.f32x2 x, x, y;\n\t"
+      "mov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a.x), "+f"(a.y)
+      : "f"(b.x), "f"(b.y));
+}
+
+// a <- fma(a, b, +0): the product, with an exact zero always +0
+__device__ __forceinline__ void mulz2(float2& a, float2 b) {
+  asm("{\n\t.reg .b64 x, y, z;\n\t"
+      "mov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\tmov.b64 z, {%4, %4};\n\t"
+      "fma.rn.f32x2 x, x, y, z;\n\t"
+      "mov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a.x), "+f"(a.y)
+      : "f"(b.x), "f"(b.y), "f"(0.f));
+}
+
+// a <- fma(sg, a, p) with the same sign sg on both lanes
+__device__ __forceinline__ void sfma2(float2& a, float sg, float2 p) {
+  asm("{\n\t.reg .b64 x, s, q;\n\t"
+      "mov.b64 x, {%0, %1};\n\tmov.b64 s, {%2, %2};\n\tmov.b64 q, {%3, %4};\n\t"
+      "fma.rn.f32x2 x, s, x, q;\n\t"
+      "mov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a.x), "+f"(a.y)
+      : "f"(sg), "f"(p.x), "f"(p.y));
+}
+
+// acc += a * a (pairwise)
+__device__ __forceinline__ void sq_acc2(float2& acc, float2 a) {
+  asm("{\n\t.reg .b64 x, c;\n\t"
+      "mov.b64 x, {%2, %3};\n\tmov.b64 c, {%0, %1};\n\t"
+      "fma.rn.f32x2 c, x, x, c;\n\t"
+      "mov.b64 {%0, %1}, c;\n\t}"
+      : "+f"(acc.x), "+f"(acc.y)
+      : "f"(a.x), "f"(a.y));
+}
+
+// ---- transform ----------------------------------------------------------------------------------
+
+// Unnormalised Walsh-Hadamard transform over the d elements of each key, whatever the layout:
+// register-bit stages (pairs, then within a pair), then lane-bit stages.
+template <int E, int L>
+__device__ __forceinline__ void fwht(float2 (&V)[E / 2], int lane) {
+#pragma unroll
+  for (int h = 1; h < E / 2; h <<= 1) {
+#pragma unroll
+    for (int t = 0; t < E / 2; ++t)
+      if (!(t & h)) bfly2(V[t], V[t + h]);
+  }
+#pragma unroll
+  for (int t = 0; t < E / 2; ++t) {
+    const float a = V[t].x, b = V[t].y;
+    V[t].x = a + b;
+    V[t].y = a - b;
+  }
+#pragma unroll
+  for (int g = 1; g < L; g <<= 1) {
+    // lower lane: a + b = fma(+1, a, b); upper lane: a - b = fma(-1, b, a)
+    const float sg = (lane & g) ? -1.f : 1.f;
+#pragma unroll
+    for (int t = 0; t < E / 2; ++t) {
+      float2 p;
+      p.x = __shfl_xor_sync(0xffffffffu, V[t].x, g);
+      p.y = __shfl_xor_sync(0xffffffffu, V[t].y, g);
+      sfma2(V[t], sg, p);
+    }
+  }
+}
+
+// ---- dither ------------------------------------------------------------------------------------
+
+// Box-Muller on 23-bit draws, scaled by amp: (amp r cos 2 pi v, amp r sin 2 pi v) with
+// u = ((xr >> 9) + 1/2) 2^-23 and v = (xa >> 9) 2^-23. Both draws are exact fp32 values:
+// u = (1 + k 2^-23) - (1 - 2^-24) is an exact subtraction. The angle is taken as 2 pi (1 + v),
+// which has the same sine and cosine.
+__device__ __forceinline__ void box_muller23(uint32_t xr, uint32_t xa, float amp, float& c, float& s) {
+  const float u = __uint_as_float((xr >> 9) | 0x3f800000u) - __uint_as_float(0x3f7fffffu);
+  const float f = __uint_as_float((xa >> 9) | 0x3f800000u);
+  float l, rs, sn, cs;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(u));
+  const float t = -1.38629436f * l;  // -2 ln u > 0
+  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(rs) : "f"(t));
+  const float r = t * rs * amp;
+  const float th = 6.28318548f * f;
+  asm("sin.approx.ftz.f32 %0, %1;" : "=f"(sn) : "f"(th));
+  asm("cos.approx.ftz.f32 %0, %1;" : "=f"(cs) : "f"(th));
+  c = r * cs;
+  s = r * sn;
+}
+
+// ---- staging ------------------------------------------------------------------------------------
+
+template <int E, int L, int ES>
+struct Geo {
+  static constexpr int K = 32 / L;                          // keys per warp
+  static constexpr int SEGE = (L == 1) ? E : 2 * E;         // elements per staged row segment
+  static constexpr int NSEG = (L == 1) ? 1 : L / 2;         // segments per key row
+  static constexpr int SEGB = SEGE * ES;                    // bytes per segment
+  static constexpr int SEGP = SEGB + 16;                    // padded segment pitch
+  static constexpr int ROWP = NSEG * SEGP;                  // padded row pitch
+  static constexpr int XBUF = K * ROWP;                     // staged keys per warp
+  static constexpr int GBUF = (32 * E + 32) * 4;            // gather buffer per warp
+};
+
+struct KeysArgs {
+  const void* x;
+  int64_t n, ld;
+  int d, m, b0, b1;           // this launch covers blocks [b0, b1)
+  const float* tab;           // device tables of all blocks, 3d words per block
+  float amp_rel;              // sqrt(d) * sigma_rel (D-FQJL), else 0
+  int dg_outer;
+  uint32_t k0, k1;
+  uint64_t first_token;
+  uint32_t* bits;
+  float* norms;
+  int W;                      // words per key row of bits
+  int* err;
+};
+
+template <int E, int L, int ES>
+__device__ __forceinline__ void stage_rows(const KeysArgs& a, int64_t row0, int nvalid, unsigned char* xb,
+                                           uint64_t* bar, int lane) {
+  using G = Geo<E, L, ES>;
+  // order this warp's earlier generic-proxy reads of the buffer before the async-proxy writes
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+  if (lane == 0) mbar_expect_tx(bar, (uint32_t)(nvalid * G::NSEG * G::SEGB));
+  __syncwarp();
+  if (lane < nvalid * G::NSEG) {
+    const int k = lane / G::NSEG, j = lane % G::NSEG;
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(a.x);
+    bulk_g2s(xb + k * G::ROWP + j * G::SEGP, src + ((row0 + k) * a.ld) * ES + (int64_t)j * G::SEGB, G::SEGB, bar);
+  }
+}
+
+// Registers of layout A from the staged row of this lane's key.
+template <int E, int L, int ES>
+__device__ __forceinline__ void load_x(const unsigned char* xrow, int s, float2 (&V)[E / 2]) {
+  using G = Geo<E, L, ES>;
+  if (L == 1) {
+    if (ES == 2) {
+#pragma unroll
+      for (int t = 0; t < E / 2; t += 8) {
+        const uint4 a = *reinterpret_cast<const uint4*>(xrow + 2 * t);
+        const uint4 c = *reinterpret_cast<const uint4*>(xrow + 2 * (t + E / 2));
+        const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          V[t + 2 * k].x = __uint_as_float(wa[k] << 16);
+          V[t + 2 * k + 1].x = __uint_as_float(wa[k] & 0xffff0000u);
+          V[t + 2 * k].y = __uint_as_float(wc[k] << 16);
+          V[t + 2 * k + 1].y = __uint_as_float(wc[k] & 0xffff0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < E / 2; t += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(xrow + 4 * t);
+        const float4 c = *reinterpret_cast<const float4*>(xrow + 4 * (t + E / 2));
+        V[t].x = a.x; V[t + 1].x = a.y; V[t + 2].x = a.z; V[t + 3].x = a.w;
+        V[t].y = c.x; V[t + 1].y = c.y; V[t + 2].y = c.z; V[t + 3].y = c.w;
+      }
+    }
+  } else {
+    const unsigned char* seg = xrow + (s >> 1) * G::SEGP;
+    const int lo = s & 1;
+    if (ES == 2) {
+      // element 2r + lo is half `lo` of word r of the segment
+      const uint32_t sel = lo ? 0x3244u : 0x1044u;
+#pragma unroll
+      for (int t = 0; t < E / 2; t += 4) {
+        const uint4 a = *reinterpret_cast<const uint4*>(seg + 4 * t);
+        const uint4 c = *reinterpret_cast<const uint4*>(seg + 4 * (t + E / 2));
+        V[t].x = __uint_as_float(__byte_perm(a.x, 0u, sel));
+        V[t + 1].x = __uint_as_float(__byte_perm(a.y, 0u, sel));
+        V[t + 2].x = __uint_as_float(__byte_perm(a.z, 0u, sel));
+        V[t + 3].x = __uint_as_float(__byte_perm(a.w, 0u, sel));
+        V[t].y = __uint_as_float(__byte_perm(c.x, 0u, sel));
+        V[t + 1].y = __uint_as_float(__byte_perm(c.y, 0u, sel));
+        V[t + 2].y = __uint_as_float(__byte_perm(c.z, 0u, sel));
+        V[t + 3].y = __uint_as_float(__byte_perm(c.w, 0u, sel));
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < E / 2; t += 2) {
+        const float4 a = *reinterpret_cast<const float4*>(seg + 8 * t);
+        const float4 c = *reinterpret_cast<const float4*>(seg + 8 * (t + E / 2));
+        V[t].x = lo ? a.y : a.x;
+        V[t + 1].x = lo ? a.w : a.z;
+        V[t].y = lo ? c.y : c.x;
+        V[t + 1].y = lo ? c.w : c.z;
+      }
+    }
+  }
+}
+
+// ---- kernel -------------------------------------------------------------------------------------
+
+template <int E, int L, int ES, int MODE>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const KeysArgs a) {
+  using G = Geo<E, L, ES>;
+  constexpr int K = G::K;
+  constexpr bool BUF = (MODE == MODE_P) || (L > 1);
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int nw = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kp = lane / L, s = lane % L;
+  const int d = a.d, nbl = a.b1 - a.b0;
+
+  // shared layout: tables | per-warp staged keys | per-warp gather buffers | per-warp barriers
+  float* tab = reinterpret_cast<float*>(smem);
+  unsigned char* xb = smem + (size_t)nbl * 3 * d * 4 + (size_t)warp * G::XBUF;
+  float* gb = reinterpret_cast<float*>(smem + (size_t)nbl * 3 * d * 4 + (size_t)nw * G::XBUF +
+                                       (BUF ? (size_t)warp * G::GBUF : 0));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)nbl * 3 * d * 4 + (size_t)nw * G::XBUF +
+                                              (BUF ? (size_t)nw * G::GBUF : 0)) + warp;
+
+  {
+    const float4* src = reinterpret_cast<const float4*>(a.tab + (size_t)a.b0 * 3 * d);
+    float4* dst = reinterpret_cast<float4*>(tab);
+    for (int i = threadIdx.x; i < nbl * 3 * d / 4; i += blockDim.x) dst[i] = __ldg(src + i);
+  }
+  if (lane == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  const int64_t nbatch = (a.n + K - 1) / K;
+  const int64_t stride = (int64_t)gridDim.x * nw;
+  int64_t q = (int64_t)blockIdx.x * nw + warp;
+  uint32_t phase = 0;
+  if (q < nbatch) stage_rows<E, L, ES>(a, q * K, (int)(a.n - q * K < K ? a.n - q * K : K), xb, bar, lane);
+
+  for (; q < nbatch; q += stride) {
+    const int64_t row = q * K + kp;
+    const bool valid = row < a.n;
+    if (!mbar_wait(bar, phase)) {
+      if (lane == 0) atomicExch(a.err, 1);
+      return;
+    }
+    phase ^= 1u;
+    const uint64_t tok = a.first_token + (uint64_t)row;
+    float norm = 0.f;
+
+    for (int bl = 0; bl < nbl; ++bl) {
+      const int b = a.b0 + bl;
+      const float* tb = tab + (size_t)bl * 3 * d;
+      float2 V[E / 2];
+      load_x<E, L, ES>(xb + kp * G::ROWP, s, V);
+      if (bl == 0) {
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < E / 2; ++t) sq_acc2(acc, V[t]);
+        float ss = acc.x + acc.y;
+#pragma unroll
+        for (int g = 1; g < L; g <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, g);
+        norm = sqrtf(ss);
+      }
+      if (bl == nbl - 1) {
+        // the staged rows are no longer needed: fetch the next batch while this one finishes
+        __syncwarp();
+        const int64_t qn = q + stride;
+        if (qn < nbatch) stage_rows<E, L, ES>(a, qn * K, (int)(a.n - qn * K < K ? a.n - qn * K : K), xb, bar, lane);
+      }
+      // D_r, then the first transform (layout A)
+      {
+        const float2* dr = reinterpret_cast<const float2*>(tb) + s * (E / 2);
+#pragma unroll
+        for (int t = 0; t < E / 2; t += 2) {
+          const float4 p = *reinterpret_cast<const float4*>(dr + t);
+          mul2(V[t], make_float2(p.x, p.y));
+          mul2(V[t + 1], make_float2(p.z, p.w));
+        }
+      }
+      fwht<E, L>(V, lane);
+      // permutation gather (and the switch to layout B)
+      if (BUF) {
+        constexpr int RS = (L == 1) ? K : 2 * K;  // word stride of consecutive r in layout A
+        float* wb = gb + ((L == 1) ? kp : K * ((s >> 1) * (2 * E + 2) + (s & 1)) + kp);
+#pragma unroll
+        for (int t = 0; t < E / 2; ++t) {
+          wb[RS * t] = V[t].x;
+          wb[RS * (t + E / 2)] = V[t].y;
+        }
+        __syncwarp();
+        const int* ro = reinterpret_cast<const int*>(tb + 2 * d) + s * E;
+        const unsigned char* rb = reinterpret_cast<const unsigned char*>(gb + kp);
+#pragma unroll
+        for (int t = 0; t < E / 2; t += 4) {
+          const int4 o1 = *reinterpret_cast<const int4*>(ro + t);
+          const int4 o2 = *reinterpret_cast<const int4*>(ro + t + E / 2);
+          V[t].x = *reinterpret_cast<const float*>(rb + o1.x);
+          V[t + 1].x = *reinterpret_cast<const float*>(rb + o1.y);
+          V[t + 2].x = *reinterpret_cast<const float*>(rb + o1.z);
+          V[t + 3].x = *reinterpret_cast<const float*>(rb + o1.w);
+          V[t].y = *reinterpret_cast<const float*>(rb + o2.x);
+          V[t + 1].y = *reinterpret_cast<const float*>(rb + o2.y);
+          V[t + 2].y = *reinterpret_cast<const float*>(rb + o2.z);
+          V[t + 3].y = *reinterpret_cast<const float*>(rb + o2.w);
+        }
+        __syncwarp();
+      }
+      const float2* gp = reinterpret_cast<const float2*>(tb + d) + s * (E / 2);
+      if (!a.dg_outer) {
+#pragma unroll
+        for (int t = 0; t < E / 2; t += 2) {
+          const float4 g = *reinterpret_cast<const float4*>(gp + t);
+          mulz2(V[t], make_float2(g.x, g.y));
+          mulz2(V[t + 1], make_float2(g.z, g.w));
+        }
+      }
+      fwht<E, L>(V, lane);
+      if (a.dg_outer) {
+#pragma unroll
+        for (int t = 0; t < E / 2; t += 2) {
+          const float4 g = *reinterpret_cast<const float4*>(gp + t);
+          mulz2(V[t], make_float2(g.x, g.y));
+          mulz2(V[t + 1], make_float2(g.z, g.w));
+        }
+      }
+      if (MODE == MODE_D) {
+        const float amp = a.amp_rel * norm;
+        if (amp != 0.f) {
+          const uint32_t cb = (uint32_t)((b * d + s * E) >> 2);
+          const uint32_t tlo = (uint32_t)tok, thi = (uint32_t)(tok >> 32);
+#pragma unroll
+          for (int c = 0; c < E / 4; ++c) {
+            const qjl::U32x4 w = qjl::philox({cb + c, tlo, thi, qjl::kStreamDither}, a.k0, a.k1);
+            float c0, s0, c1, s1;
+            box_muller23(w.x, w.y, amp, c0, s0);
+            box_muller23(w.z, w.w, amp, c1, s1);
+            const float xi[4] = {c0, s0, c1, s1};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int r = 4 * c + j;
+              if (r < E / 2) V[r].x += xi[j];
+              else V[r - E / 2].y += xi[j];
+            }
+          }
+        }
+      }
+      // sign bits: element s*E + r is bit r % 32 of word (b*d + s*E + r) / 32
+      if (valid) {
+        uint32_t* out = a.bits + row * (int64_t)a.W + ((b * d + s * E) >> 5);
+#pragma unroll
+        for (int w = 0; w < E / 32; ++w) {
+          uint32_t acc = 0;
+#pragma unroll
+          for (int k = 31; k >= 0; --k) {
+            const int r = 32 * w + k;
+            const float y = (r < E / 2) ? V[r].x : V[r - E / 2].y;
+            acc = __funnelshift_l(__float_as_uint(y), acc, 1);
+          }
+          out[w] = ~acc;
+        }
+      }
+    }
+    if (valid && s == 0 && a.norms) a.norms[row] = norm;
+  }
+}
+
+// ---- host side ----------------------------------------------------------------------------------
+
+struct Layout {
+  int E, L, K;
+};
+
+Layout layout_for(int d) {
+  Layout g;
+  g.E = d < 128 ? d : 128;
+  g.L = d / g.E;
+  g.K = 32 / g.L;
+  return g;
+}
+
+template <int E, int L, int ES, int MODE>
+qjl_status launch_t(const qjl_projection* P, KeysArgs a, int64_t n, cudaStream_t st) {
+  using G = Geo<E, L, ES>;
+  constexpr bool BUF = (MODE == MODE_P) || (L > 1);
+  auto kern = fqjl_keys_kernel<E, L, ES, MODE>;
+  const int d = P->d, nb = P->m / d;
+  const int per_launch = std::max(1, (int)std::min<size_t>(nb, kTableBudget / ((size_t)3 * d * 4)));
+  const size_t per_warp = G::XBUF + (BUF ? G::GBUF : 0) + 8;
+  int dev = P->device;
+  for (int b0 = 0; b0 < nb; b0 += per_launch) {
+    const int b1 = std::min(nb, b0 + per_launch);
+    const size_t tab = (size_t)(b1 - b0) * 3 * d * 4;
+    int nw = kMaxWarps;
+    while (nw > 1 && tab + nw * per_warp > kSmemLimit) --nw;
+    const size_t smem = tab + nw * per_warp;
+    if (smem > kSmemLimit) return qjl_set_error(QJL_ERR_UNSUPPORTED, "FQJL key kernel: shared memory");
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return qjl_check_launch("fqjl_keys_kernel smem attribute");
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nw * 32, smem) != cudaSuccess || per_sm < 1) {
+      cudaGetLastError();
+      per_sm = 1;
+    }
+    const int64_t nbatch = (n + G::K - 1) / G::K;
+    const int64_t want = (nbatch + nw - 1) / nw;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)qjl_num_sms(dev) * per_sm));
+    a.b0 = b0;
+    a.b1 = b1;
+    if (b0 > 0) a.norms = nullptr;
+    qjl_log_launch("fqjl_keys_kernel", grid, nw * 32, smem, per_sm);
+    kern<<<grid, nw * 32, smem, st>>>(a);
+    const qjl_status s = qjl_check_launch("fqjl_keys_kernel");
+    if (s != QJL_OK) return s;
+  }
+  return QJL_OK;
+}
+
+template <int E, int L>
+qjl_status launch_el(const qjl_projection* P, const KeysArgs& a, int dtype, int64_t n, cudaStream_t st) {
+  const bool dmode = P->kind == QJL_DFQJL;
+  if (dtype == QJL_F32)
+    return dmode ? launch_t<E, L, 4, MODE_D>(P, a, n, st) : launch_t<E, L, 4, MODE_P>(P, a, n, st);
+  return dmode ? launch_t<E, L, 2, MODE_D>(P, a, n, st) : launch_t<E, L, 2, MODE_P>(P, a, n, st);
+}
+
+}  // namespace
+
+// Per-block tables of the key kernel, 3d words per block: D_r as layout-A register pairs, D_g as
+// layout-B register pairs, and for each layout-B element the byte offset of its gather source in
+// the warp's buffer (the permutation for P-FQJL, the identity otherwise).
+std::vector<float> fqjl_key_tables(int d, int m, const float* D_r, const int32_t* perm, const float* D_g) {
+  const Layout g = layout_for(d);
+  const int E = g.E, L = g.L, K = g.K, nb = m / d;
+  std::vector<float> t((size_t)nb * 3 * d);
+  auto elemA = [&](int r, int s) { return L == 1 ? r : (s >> 1) * 2 * E + 2 * r + (s & 1); };
+  for (int b = 0; b < nb; ++b) {
+    float* dr = t.data() + (size_t)b * 3 * d;
+    float* gp = dr + d;
+    int32_t* ro = reinterpret_cast<int32_t*>(dr + 2 * d);
+    const float* Dr = D_r + (size_t)b * d;
+    const float* Dg = D_g + (size_t)b * d;
+    const int32_t* pi = perm + (size_t)b * d;
+    for (int s = 0; s < L; ++s) {
+      for (int u = 0; u < E / 2; ++u) {
+        dr[s * E + 2 * u] = Dr[elemA(u, s)];
+        dr[s * E + 2 * u + 1] = Dr[elemA(u + E / 2, s)];
+        gp[s * E + 2 * u] = Dg[s * E + u];
+        gp[s * E + 2 * u + 1] = Dg[s * E + u + E / 2];
+      }
+      for (int r = 0; r < E; ++r) {
+        const int j = pi[s * E + r];
+        ro[s * E + r] = 4 * K * (j + 2 * (j / (2 * E)));
+      }
+    }
+  }
+  return t;
+}
+
+bool fqjl_keys_supported(const qjl_projection* P) { return P->d >= 32 && P->d <= 1024 && P->ktab; }
+
+qjl_status launch_fqjl_keys(const qjl_projection* P, const void* x, int dtype, int64_t n, int64_t ld,
+                            uint64_t first_token, uint32_t* bits, float* norms, cudaStream_t st) {
+  if (n <= 0) return QJL_OK;
+  KeysArgs a{};
+  a.x = x;
+  a.n = n;
+  a.ld = ld;
+  a.d = P->d;
+  a.m = P->m;
+  a.tab = P->ktab;
+  a.amp_rel = P->kind == QJL_DFQJL ? sqrtf((float)P->d) * P->dither_sigma : 0.f;
+  a.dg_outer = P->opt.dg_outer;
+  a.k0 = (uint32_t)P->seed;
+  a.k1 = (uint32_t)(P->seed >> 32);
+  a.first_token = first_token;
+  a.bits = bits;
+  a.norms = norms;
+  a.W = P->m / 32;
+  a.err = qjl_error_flag(P->device);
+  if (!a.err) return qjl_set_error(QJL_ERR_CUDA, "cannot allocate the device error flag");
+  switch (P->d) {
+    case 32: return launch_el<32, 1>(P, a, dtype, n, st);
+    case 64: return launch_el<64, 1>(P, a, dtype, n, st);
+    case 128: return launch_el<128, 1>(P, a, dtype, n, st);
+    case 256: return launch_el<128, 2>(P, a, dtype, n, st);
+    case 512: return launch_el<128, 4>(P, a, dtype, n, st);
+    case 1024: return launch_el<128, 8>(P, a, dtype, n, st);
+  }
+  return qjl_set_error(QJL_ERR_UNSUPPORTED, "FQJL key kernel supports d in {32,...,1024}");
+}

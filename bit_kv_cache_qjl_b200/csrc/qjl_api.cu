@@ -134,6 +134,7 @@ void free_projection(qjl_projection* P) {
   cudaFree(P->D_r);
   cudaFree(P->perm);
   cudaFree(P->D_g);
+  cudaFree(P->ktab);
   free(P->h_S);
   free(P->h_D_r);
   free(P->h_perm);
@@ -261,6 +262,10 @@ qjl_status qjl_make_projection(uint64_t seed, int d, int m, qjl_kind kind, const
     st = dev_upload(&P->D_r, P->h_D_r, cnt);
     if (st == QJL_OK) st = dev_upload(&P->D_g, P->h_D_g, cnt);
     if (st == QJL_OK) st = dev_upload(&P->perm, P->h_perm, cnt);
+    if (st == QJL_OK) {
+      const std::vector<float> kt = fqjl_key_tables(d, m, P->h_D_r, P->h_perm, P->h_D_g);
+      st = dev_upload(&P->ktab, kt.data(), kt.size());
+    }
   }
   if (st != QJL_OK) {
     free_projection(P);
@@ -326,7 +331,7 @@ qjl_status qjl_quantize_keys(const qjl_projection* P, const void* keys, qjl_dtyp
     if (dense_tc_supported(P, dtype, keys, ld)) return launch_dense_tc(P, keys, n, ld, bits, norms, st);
     return launch_dense_simt(P, keys, dtype, n, ld, bits, norms, nullptr, st);
   }
-  return launch_fqjl(P, keys, dtype, n, ld, first_token, bits, norms, nullptr, st);
+  return launch_fqjl_keys(P, keys, dtype, n, ld, first_token, bits, norms, st);
 }
 
 qjl_status qjl_project_queries(const qjl_projection* P, const float* q, int64_t nq, int64_t ld,
@@ -343,7 +348,7 @@ qjl_status qjl_project_queries(const qjl_projection* P, const float* q, int64_t 
   if (!g.ok) return qjl_set_error(QJL_ERR_CUDA, "cannot select the projection's device");
   cudaStream_t st = (cudaStream_t)stream;
   if (P->kind == QJL_DENSE) return launch_project_dense(P, q, nq, ld, sq, st);
-  return launch_fqjl(P, q, QJL_F32, nq, ld, 0, nullptr, nullptr, sq, st);
+  return launch_fqjl_queries(P, q, nq, ld, sq, st);
 }
 
 qjl_status qjl_scores(const qjl_projection* P, const uint32_t* bits, const float* norms,

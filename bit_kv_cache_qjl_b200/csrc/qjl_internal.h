@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <vector>
 
 #include "../../include/qjl.h"
 
@@ -21,6 +22,7 @@ struct qjl_projection {
   float* D_r = nullptr;
   int32_t* perm = nullptr;
   float* D_g = nullptr;
+  float* ktab = nullptr;        // key-kernel tables, 3d words per block (fqjl_key_tables)
   // host copies for export
   float* h_S = nullptr;
   float* h_D_r = nullptr;
@@ -41,9 +43,11 @@ qjl_status launch_project_dense(const qjl_projection* P, const float* q, int64_t
 bool dense_tc_supported(const qjl_projection* P, int dtype, const void* keys, int64_t ld);
 qjl_status launch_dense_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld,
                            uint32_t* bits, float* norms, cudaStream_t st);
-qjl_status launch_fqjl(const qjl_projection* P, const void* keys, int dtype, int64_t n,
-                       int64_t ld, uint64_t first_token, uint32_t* bits, float* norms,
-                       float* proj_out, cudaStream_t st);
+qjl_status launch_fqjl_queries(const qjl_projection* P, const float* q, int64_t nq, int64_t ld,
+                               float* out, cudaStream_t st);
+std::vector<float> fqjl_key_tables(int d, int m, const float* D_r, const int32_t* perm, const float* D_g);
+qjl_status launch_fqjl_keys(const qjl_projection* P, const void* keys, int dtype, int64_t n, int64_t ld,
+                            uint64_t first_token, uint32_t* bits, float* norms, cudaStream_t st);
 bool scores_mma_supported(int m);
 bool scores_tc_supported(int m, int J);
 qjl_status launch_scores_tc(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t groups,

@@ -41,10 +41,12 @@ def test_fp32_keys_use_simt_kernel(cuda_ok):
     assert _has(_kernels(lambda: qjl.quantize_keys(P, keys)), "dense_simt_kernel")
 
 
-def test_fqjl_kernel(cuda_ok):
+def test_fqjl_kernels(cuda_ok):
     P = qjl.Projection(4, 256, 1024, "pfqjl")
     keys = wl.normal((512, 256), 1, "cuda", torch.bfloat16)
-    assert _has(_kernels(lambda: qjl.quantize_keys(P, keys)), "fqjl_kernel")
+    assert _has(_kernels(lambda: qjl.quantize_keys(P, keys)), "fqjl_keys_kernel")
+    q = wl.normal((3, 256), 2, "cuda")
+    assert _has(_kernels(lambda: qjl.project_queries(P, q)), "fqjl_query_kernel")
 
 
 def test_scores_and_projection_kernels(cuda_ok):

@@ -81,6 +81,18 @@ def test_dense_bf16_keys_fp32_matrix_simt(cuda_ok):
     ("pfqjl", 32, 64, 77, torch.float32, 0),
     ("dfqjl", 1024, 2048, 40, torch.bfloat16, 3),
     ("pfqjl", 512, 512, 33, torch.float32, 0),
+    # every thread layout of the transform kernel (d = 32 ... 1024), both dtypes, ragged batches
+    ("pfqjl", 64, 128, 129, torch.bfloat16, 0),
+    ("dfqjl", 32, 64, 65, torch.bfloat16, 5),
+    ("dfqjl", 64, 64, 31, torch.float32, 9),
+    ("dfqjl", 256, 512, 301, torch.bfloat16, 7),
+    ("pfqjl", 256, 256, 17, torch.float32, 0),
+    ("dfqjl", 512, 1024, 45, torch.float32, 0),
+    ("pfqjl", 1024, 1024, 9, torch.float32, 0),
+    ("pfqjl", 128, 128, 1, torch.bfloat16, 0),
+    # more blocks than one launch's table budget: several launches over block ranges
+    ("pfqjl", 1024, 4096, 37, torch.bfloat16, 0),
+    ("dfqjl", 128, 4096, 70, torch.float32, 11),
 ])
 def test_fqjl(cuda_ok, kind, d, m, n, dtype, ft):
     P = Projection(4, d, m, kind)
@@ -90,6 +102,43 @@ def test_fqjl(cuda_ok, kind, d, m, n, dtype, ft):
 def test_fqjl_literal_order(cuda_ok):
     P = Projection(4, 128, 256, "pfqjl", dg_outer=True)
     _run(P, wl.normal((500, 128), 8, "cuda", torch.bfloat16))
+    P = Projection(4, 256, 512, "dfqjl", dg_outer=True)
+    _run(P, wl.normal((70, 256), 18, "cuda", torch.bfloat16), first_token=3)
+
+
+def test_dfqjl_without_dither(cuda_ok):
+    P = Projection(6, 128, 256, "dfqjl", dither_sigma_rel=0.0)
+    _run(P, wl.normal((100, 128), 19, "cuda", torch.bfloat16))
+
+
+@pytest.mark.parametrize("kind,d", [("pfqjl", 128), ("dfqjl", 128), ("pfqjl", 256), ("dfqjl", 512)])
+def test_fqjl_zero_keys(cuda_ok, kind, d):
+    """A zero key: the map is +0 everywhere, so every bit is 1 (sign(0) = +1), dither or not."""
+    P = Projection(4, d, 2 * d, kind)
+    keys = torch.zeros((40, d), dtype=torch.bfloat16, device="cuda")
+    keys[7] = -0.0
+    bits, norms = quantize_keys(P, keys)
+    torch.cuda.synchronize()
+    assert torch.all(norms == 0)
+    assert torch.all(bits == -1)
+
+
+def test_fqjl_strided_rows(cuda_ok):
+    import ctypes
+    from bit_kv_cache_qjl_b200 import lib
+    P = Projection(4, 256, 512, "pfqjl")
+    big = wl.normal((90, 320), 21, "cuda", torch.bfloat16)
+    keys = big[:, :256]
+    b2 = torch.empty((90, 16), dtype=torch.int32, device="cuda")
+    n2 = torch.empty((90,), device="cuda")
+    st = lib().qjl_quantize_keys(P.handle, ctypes.c_void_p(keys.data_ptr()), 1, 90, 320, 4,
+                                 ctypes.c_void_p(b2.data_ptr()), ctypes.c_void_p(n2.data_ptr()),
+                                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    ow, onorm, y = oracle.qjl.quantize_keys(oracle_projection(P), host(keys), 4)
+    check_bits(host(b2), ow, y, onorm, 512)
+    np.testing.assert_allclose(host(n2), onorm, rtol=1e-5)
 
 
 def test_outlier_keys_dense(cuda_ok):
