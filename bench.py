@@ -212,6 +212,11 @@ def profile_case(case, n):
         P = qjl.Projection(4, 256, m, "pfqjl")
         keys = wl.bulk_keys(dev, n=n, d=256)
         run = lambda: qjl.quantize_keys(P, keys)
+    elif case == "dfqjl":
+        P = qjl.Projection(5, D, M, "dfqjl", dither_sigma_rel=0.5)
+        keys, _ = wl.decode_kv(dev, B=1, H=max(1, n // 16384), N=min(16384, n), d=D)
+        keys = keys.reshape(-1, D)
+        run = lambda: qjl.quantize_keys(P, keys)
     elif case == "scores":
         P = qjl.Projection(2, D, M, "dense")
         G = max(1, n // N)
@@ -379,7 +384,7 @@ def main():
     ap.add_argument("--ref-sample", type=int, default=4096)
     ap.add_argument("--cpu-sample", type=int, default=1 << 18)
     ap.add_argument("--profile-case", default=None,
-                    choices=["quantize", "scores", "fqjl", "fqjl1024", "values", "decode"],
+                    choices=["quantize", "scores", "fqjl", "fqjl1024", "dfqjl", "values", "decode"],
                     help="run one small case of a single kernel (3 launches after 2 warm-ups) for ncu")
     ap.add_argument("--profile-keys", type=int, default=1 << 20)
     ap.add_argument("--e2e-steps", type=int, default=5)

@@ -19,25 +19,21 @@
 // Work split. A thread holds E = min(d, 128) elements of one key in registers
 // as E/2 packed pairs V[t] = (v_t, v_{t+E/2}), so most butterflies are sm_100
 // packed-fp32 add/sub. L = d/E lanes share a key (1 for d <= 128, else 2, 4
-// or 8), K = 32/L keys per warp. Butterflies on register bits need no data
-// movement. Butterflies on lane bits are one shfl_xor and one packed FMA.
-// Two element orders are used:
-//   layout A (first transform)  : i = (s>>1)*2E + 2r + (s&1)   (i = r if L = 1)
-//   layout B (second transform) : i = s*E + r
-// where s is the lane within the key and r the register index. Layout A lets
-// the L lanes of a key read the same staged words (broadcast, no bank
-// conflict). Layout B gives each lane E consecutive output bits, which
-// funnel-shift into whole words. The permutation gather between the two
-// transforms also switches layout. It goes through a per-warp shared buffer
-// in which element j of key slot k sits at word K*(j + 2*(j / 2E)) + k. The
-// writes from layout A are conflict-free; the gather reads are at
+// or 8), K = 32/L keys per warp, and lane s of a key holds elements
+// i = s*E + r, r = 0..E-1. Butterflies on register bits need no data
+// movement. Butterflies on lane bits are one shfl_xor and one packed FMA per
+// pair. Each lane thus ends with E consecutive output bits, which
+// funnel-shift into whole words. The P-FQJL permutation is a gather through
+// a per-warp shared buffer, in which element j of key slot k sits at word
+// K*(j + j/E) + k: the writes are conflict-free and the gather reads go to
 // precomputed offsets.
 //
 // Keys reach shared memory by cp.async.bulk (the API requires 16-byte aligned
 // rows), one copy per key row segment, into segments padded by 16 bytes so
-// that the register loads are conflict-free. Each warp prefetches its next
-// batch of K keys while it transforms the current one. Per-block tables (D_r and D_g as register
-// pairs, gather offsets) are staged once per CTA.
+// that the register loads are conflict-free. Each warp fetches its next batch
+// of K keys while other warps compute, one batch in flight per warp. Per-block tables (D_r
+// and D_g as register pairs, gather offsets) are staged once per CTA, with the
+// lanes' segments 16 bytes apart so that they sit in different banks.
 //
 // No output bit can come from a -0: D_g is applied as fma(u, g, +0), which
 // maps an exact zero product to +0, and sums of values that are not -0 are
@@ -178,13 +174,13 @@ __device__ __forceinline__ void box_muller23(uint32_t xr, uint32_t xa, float amp
 template <int E, int L, int ES>
 struct Geo {
   static constexpr int K = 32 / L;                          // keys per warp
-  static constexpr int SEGE = (L == 1) ? E : 2 * E;         // elements per staged row segment
-  static constexpr int NSEG = (L == 1) ? 1 : L / 2;         // segments per key row
-  static constexpr int SEGB = SEGE * ES;                    // bytes per segment
+  static constexpr int SEGB = E * ES;                       // bytes of one lane's segment of a key row
   static constexpr int SEGP = SEGB + 16;                    // padded segment pitch
-  static constexpr int ROWP = NSEG * SEGP;                  // padded row pitch
+  static constexpr int ROWP = L * SEGP;                     // padded row pitch
   static constexpr int XBUF = K * ROWP;                     // staged keys per warp
   static constexpr int GBUF = (32 * E + 32) * 4;            // gather buffer per warp
+  static constexpr int TSEG = E + 4;                        // words per lane segment of a table
+  static constexpr int TBLK = 3 * L * TSEG;                 // table words per block
 };
 
 struct KeysArgs {
@@ -209,73 +205,58 @@ __device__ __forceinline__ void stage_rows(const KeysArgs& a, int64_t row0, int 
   // order this warp's earlier generic-proxy reads of the buffer before the async-proxy writes
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncwarp();
-  if (lane == 0) mbar_expect_tx(bar, (uint32_t)(nvalid * G::NSEG * G::SEGB));
+  if (lane == 0) mbar_expect_tx(bar, (uint32_t)(nvalid * L * G::SEGB));
   __syncwarp();
-  if (lane < nvalid * G::NSEG) {
-    const int k = lane / G::NSEG, j = lane % G::NSEG;
+  if (lane < nvalid * L) {
+    const int k = lane / L, j = lane % L;
     const unsigned char* src = reinterpret_cast<const unsigned char*>(a.x);
     bulk_g2s(xb + k * G::ROWP + j * G::SEGP, src + ((row0 + k) * a.ld) * ES + (int64_t)j * G::SEGB, G::SEGB, bar);
   }
 }
 
-// Registers of layout A from the staged row of this lane's key.
+// This lane's E elements of its key, from the staged row, as register pairs.
 template <int E, int L, int ES>
 __device__ __forceinline__ void load_x(const unsigned char* xrow, int s, float2 (&V)[E / 2]) {
   using G = Geo<E, L, ES>;
-  if (L == 1) {
-    if (ES == 2) {
+  const unsigned char* seg = xrow + s * G::SEGP;
+  if (ES == 2) {
 #pragma unroll
-      for (int t = 0; t < E / 2; t += 8) {
-        const uint4 a = *reinterpret_cast<const uint4*>(xrow + 2 * t);
-        const uint4 c = *reinterpret_cast<const uint4*>(xrow + 2 * (t + E / 2));
-        const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wc[4] = {c.x, c.y, c.z, c.w};
+    for (int t = 0; t < E / 2; t += 8) {
+      const uint4 a = *reinterpret_cast<const uint4*>(seg + 2 * t);
+      const uint4 c = *reinterpret_cast<const uint4*>(seg + 2 * (t + E / 2));
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wc[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          V[t + 2 * k].x = __uint_as_float(wa[k] << 16);
-          V[t + 2 * k + 1].x = __uint_as_float(wa[k] & 0xffff0000u);
-          V[t + 2 * k].y = __uint_as_float(wc[k] << 16);
-          V[t + 2 * k + 1].y = __uint_as_float(wc[k] & 0xffff0000u);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int t = 0; t < E / 2; t += 4) {
-        const float4 a = *reinterpret_cast<const float4*>(xrow + 4 * t);
-        const float4 c = *reinterpret_cast<const float4*>(xrow + 4 * (t + E / 2));
-        V[t].x = a.x; V[t + 1].x = a.y; V[t + 2].x = a.z; V[t + 3].x = a.w;
-        V[t].y = c.x; V[t + 1].y = c.y; V[t + 2].y = c.z; V[t + 3].y = c.w;
+      for (int k = 0; k < 4; ++k) {
+        V[t + 2 * k].x = __uint_as_float(wa[k] << 16);
+        V[t + 2 * k + 1].x = __uint_as_float(wa[k] & 0xffff0000u);
+        V[t + 2 * k].y = __uint_as_float(wc[k] << 16);
+        V[t + 2 * k + 1].y = __uint_as_float(wc[k] & 0xffff0000u);
       }
     }
   } else {
-    const unsigned char* seg = xrow + (s >> 1) * G::SEGP;
-    const int lo = s & 1;
-    if (ES == 2) {
-      // element 2r + lo is half `lo` of word r of the segment
-      const uint32_t sel = lo ? 0x3244u : 0x1044u;
 #pragma unroll
-      for (int t = 0; t < E / 2; t += 4) {
-        const uint4 a = *reinterpret_cast<const uint4*>(seg + 4 * t);
-        const uint4 c = *reinterpret_cast<const uint4*>(seg + 4 * (t + E / 2));
-        V[t].x = __uint_as_float(__byte_perm(a.x, 0u, sel));
-        V[t + 1].x = __uint_as_float(__byte_perm(a.y, 0u, sel));
-        V[t + 2].x = __uint_as_float(__byte_perm(a.z, 0u, sel));
-        V[t + 3].x = __uint_as_float(__byte_perm(a.w, 0u, sel));
-        V[t].y = __uint_as_float(__byte_perm(c.x, 0u, sel));
-        V[t + 1].y = __uint_as_float(__byte_perm(c.y, 0u, sel));
-        V[t + 2].y = __uint_as_float(__byte_perm(c.z, 0u, sel));
-        V[t + 3].y = __uint_as_float(__byte_perm(c.w, 0u, sel));
-      }
-    } else {
-#pragma unroll
-      for (int t = 0; t < E / 2; t += 2) {
-        const float4 a = *reinterpret_cast<const float4*>(seg + 8 * t);
-        const float4 c = *reinterpret_cast<const float4*>(seg + 8 * (t + E / 2));
-        V[t].x = lo ? a.y : a.x;
-        V[t + 1].x = lo ? a.w : a.z;
-        V[t].y = lo ? c.y : c.x;
-        V[t + 1].y = lo ? c.w : c.z;
-      }
+    for (int t = 0; t < E / 2; t += 4) {
+      const float4 a = *reinterpret_cast<const float4*>(seg + 4 * t);
+      const float4 c = *reinterpret_cast<const float4*>(seg + 4 * (t + E / 2));
+      V[t].x = a.x; V[t + 1].x = a.y; V[t + 2].x = a.z; V[t + 3].x = a.w;
+      V[t].y = c.x; V[t + 1].y = c.y; V[t + 2].y = c.z; V[t + 3].y = c.w;
     }
+  }
+}
+
+// Philox4x32-10 on four counters at once, rounds interleaved for instruction-level parallelism.
+__device__ __forceinline__ void philox_x4(qjl::U32x4 (&c)[4], uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t hA, lA, hB, lB;
+      qjl::mul_hi_lo(0xD2511F53u, c[j].x, hA, lA);
+      qjl::mul_hi_lo(0xCD9E8D57u, c[j].z, hB, lB);
+      c[j] = qjl::U32x4{hB ^ c[j].y ^ k0, lB, hA ^ c[j].w ^ k1, lA};
+    }
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
   }
 }
 
@@ -285,25 +266,25 @@ template <int E, int L, int ES, int MODE>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const KeysArgs a) {
   using G = Geo<E, L, ES>;
   constexpr int K = G::K;
-  constexpr bool BUF = (MODE == MODE_P) || (L > 1);
+  constexpr bool BUF = (MODE == MODE_P);
   extern __shared__ __align__(16) unsigned char smem[];
   const int nw = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kp = lane / L, s = lane % L;
   const int d = a.d, nbl = a.b1 - a.b0;
+  const size_t tab_bytes = (size_t)nbl * G::TBLK * 4;
 
   // shared layout: tables | per-warp staged keys | per-warp gather buffers | per-warp barriers
   float* tab = reinterpret_cast<float*>(smem);
-  unsigned char* xb = smem + (size_t)nbl * 3 * d * 4 + (size_t)warp * G::XBUF;
-  float* gb = reinterpret_cast<float*>(smem + (size_t)nbl * 3 * d * 4 + (size_t)nw * G::XBUF +
-                                       (BUF ? (size_t)warp * G::GBUF : 0));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)nbl * 3 * d * 4 + (size_t)nw * G::XBUF +
+  unsigned char* xb = smem + tab_bytes + (size_t)warp * G::XBUF;
+  float* gb = reinterpret_cast<float*>(smem + tab_bytes + (size_t)nw * G::XBUF + (BUF ? (size_t)warp * G::GBUF : 0));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + tab_bytes + (size_t)nw * G::XBUF +
                                               (BUF ? (size_t)nw * G::GBUF : 0)) + warp;
 
   {
-    const float4* src = reinterpret_cast<const float4*>(a.tab + (size_t)a.b0 * 3 * d);
+    const float4* src = reinterpret_cast<const float4*>(a.tab + (size_t)a.b0 * G::TBLK);
     float4* dst = reinterpret_cast<float4*>(tab);
-    for (int i = threadIdx.x; i < nbl * 3 * d / 4; i += blockDim.x) dst[i] = __ldg(src + i);
+    for (int i = threadIdx.x; i < nbl * G::TBLK / 4; i += blockDim.x) dst[i] = __ldg(src + i);
   }
   if (lane == 0) {
     mbar_init(bar, 1);
@@ -311,26 +292,28 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
   }
   __syncthreads();
 
+  // this warp's batches are q0, q0 + stride, ...; the barrier completes one phase per batch
   const int64_t nbatch = (a.n + K - 1) / K;
   const int64_t stride = (int64_t)gridDim.x * nw;
   int64_t q = (int64_t)blockIdx.x * nw + warp;
-  uint32_t phase = 0;
   if (q < nbatch) stage_rows<E, L, ES>(a, q * K, (int)(a.n - q * K < K ? a.n - q * K : K), xb, bar, lane);
 
-  for (; q < nbatch; q += stride) {
+  for (uint32_t phase = 0; q < nbatch; q += stride, phase ^= 1u) {
     const int64_t row = q * K + kp;
     const bool valid = row < a.n;
-    if (!mbar_wait(bar, phase)) {
+    if (!__all_sync(0xffffffffu, mbar_wait(bar, phase))) {
+      // the batch never landed (the whole warp agrees): flag it, give the copy one more
+      // bounded wait, and stop
       if (lane == 0) atomicExch(a.err, 1);
+      mbar_wait(bar, phase);
       return;
     }
-    phase ^= 1u;
     const uint64_t tok = a.first_token + (uint64_t)row;
     float norm = 0.f;
 
     for (int bl = 0; bl < nbl; ++bl) {
       const int b = a.b0 + bl;
-      const float* tb = tab + (size_t)bl * 3 * d;
+      const float* tb = tab + (size_t)bl * G::TBLK;
       float2 V[E / 2];
       load_x<E, L, ES>(xb + kp * G::ROWP, s, V);
       if (bl == 0) {
@@ -342,15 +325,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
         for (int g = 1; g < L; g <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, g);
         norm = sqrtf(ss);
       }
-      if (bl == nbl - 1) {
-        // the staged rows are no longer needed: fetch the next batch while this one finishes
-        __syncwarp();
-        const int64_t qn = q + stride;
-        if (qn < nbatch) stage_rows<E, L, ES>(a, qn * K, (int)(a.n - qn * K < K ? a.n - qn * K : K), xb, bar, lane);
-      }
-      // D_r, then the first transform (layout A)
+      // D_r, then the first transform
       {
-        const float2* dr = reinterpret_cast<const float2*>(tb) + s * (E / 2);
+        const float2* dr = reinterpret_cast<const float2*>(tb + s * G::TSEG);
 #pragma unroll
         for (int t = 0; t < E / 2; t += 2) {
           const float4 p = *reinterpret_cast<const float4*>(dr + t);
@@ -359,17 +336,16 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
         }
       }
       fwht<E, L>(V, lane);
-      // permutation gather (and the switch to layout B)
+      // permutation gather: element j of key slot kp at word K*(j + j/E) + kp
       if (BUF) {
-        constexpr int RS = (L == 1) ? K : 2 * K;  // word stride of consecutive r in layout A
-        float* wb = gb + ((L == 1) ? kp : K * ((s >> 1) * (2 * E + 2) + (s & 1)) + kp);
+        float* wb = gb + K * s * (E + 1) + kp;
 #pragma unroll
         for (int t = 0; t < E / 2; ++t) {
-          wb[RS * t] = V[t].x;
-          wb[RS * (t + E / 2)] = V[t].y;
+          wb[K * t] = V[t].x;
+          wb[K * (t + E / 2)] = V[t].y;
         }
         __syncwarp();
-        const int* ro = reinterpret_cast<const int*>(tb + 2 * d) + s * E;
+        const int* ro = reinterpret_cast<const int*>(tb + 2 * L * G::TSEG + s * G::TSEG);
         const unsigned char* rb = reinterpret_cast<const unsigned char*>(gb + kp);
 #pragma unroll
         for (int t = 0; t < E / 2; t += 4) {
@@ -386,7 +362,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
         }
         __syncwarp();
       }
-      const float2* gp = reinterpret_cast<const float2*>(tb + d) + s * (E / 2);
+      const float2* gp = reinterpret_cast<const float2*>(tb + L * G::TSEG + s * G::TSEG);
       if (!a.dg_outer) {
 #pragma unroll
         for (int t = 0; t < E / 2; t += 2) {
@@ -410,22 +386,27 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
           const uint32_t cb = (uint32_t)((b * d + s * E) >> 2);
           const uint32_t tlo = (uint32_t)tok, thi = (uint32_t)(tok >> 32);
 #pragma unroll
-          for (int c = 0; c < E / 4; ++c) {
-            const qjl::U32x4 w = qjl::philox({cb + c, tlo, thi, qjl::kStreamDither}, a.k0, a.k1);
-            float c0, s0, c1, s1;
-            box_muller23(w.x, w.y, amp, c0, s0);
-            box_muller23(w.z, w.w, amp, c1, s1);
-            const float xi[4] = {c0, s0, c1, s1};
+          for (int c = 0; c < E / 4; c += 4) {
+            qjl::U32x4 w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w[j] = qjl::U32x4{cb + c + j, tlo, thi, qjl::kStreamDither};
+            philox_x4(w, a.k0, a.k1);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const int r = 4 * c + j;
-              if (r < E / 2) V[r].x += xi[j];
-              else V[r - E / 2].y += xi[j];
+              float xi[4];
+              box_muller23(w[j].x, w[j].y, amp, xi[0], xi[1]);
+              box_muller23(w[j].z, w[j].w, amp, xi[2], xi[3]);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int r = 4 * (c + j) + e;
+                if (r < E / 2) V[r].x += xi[e];
+                else V[r - E / 2].y += xi[e];
+              }
             }
           }
         }
       }
-      // sign bits: element s*E + r is bit r % 32 of word (b*d + s*E + r) / 32
+      // sign bits: element s*E + r is bit r % 32 of word (b*d + s*E + r) / 32 of the key's row
       if (valid) {
         uint32_t* out = a.bits + row * (int64_t)a.W + ((b * d + s * E) >> 5);
 #pragma unroll
@@ -442,6 +423,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
       }
     }
     if (valid && s == 0 && a.norms) a.norms[row] = norm;
+    // fetch the next batch into the same buffer (issuing it at the end of the batch measured
+    // faster than right after the last read of the staged rows)
+    __syncwarp();
+    const int64_t qn = q + stride;
+    if (qn < nbatch) stage_rows<E, L, ES>(a, qn * K, (int)(a.n - qn * K < K ? a.n - qn * K : K), xb, bar, lane);
   }
 }
 
@@ -462,15 +448,15 @@ Layout layout_for(int d) {
 template <int E, int L, int ES, int MODE>
 qjl_status launch_t(const qjl_projection* P, KeysArgs a, int64_t n, cudaStream_t st) {
   using G = Geo<E, L, ES>;
-  constexpr bool BUF = (MODE == MODE_P) || (L > 1);
+  constexpr bool BUF = (MODE == MODE_P);
   auto kern = fqjl_keys_kernel<E, L, ES, MODE>;
   const int d = P->d, nb = P->m / d;
-  const int per_launch = std::max(1, (int)std::min<size_t>(nb, kTableBudget / ((size_t)3 * d * 4)));
-  const size_t per_warp = G::XBUF + (BUF ? G::GBUF : 0) + 8;
+  const int per_launch = std::max(1, (int)std::min<size_t>(nb, kTableBudget / ((size_t)G::TBLK * 4)));
+  const size_t per_warp = G::XBUF + 8 + (BUF ? G::GBUF : 0);
   int dev = P->device;
   for (int b0 = 0; b0 < nb; b0 += per_launch) {
     const int b1 = std::min(nb, b0 + per_launch);
-    const size_t tab = (size_t)(b1 - b0) * 3 * d * 4;
+    const size_t tab = (size_t)(b1 - b0) * G::TBLK * 4;
     int nw = kMaxWarps;
     while (nw > 1 && tab + nw * per_warp > kSmemLimit) --nw;
     const size_t smem = tab + nw * per_warp;
@@ -506,31 +492,33 @@ qjl_status launch_el(const qjl_projection* P, const KeysArgs& a, int dtype, int6
 
 }  // namespace
 
-// Per-block tables of the key kernel, 3d words per block: D_r as layout-A register pairs, D_g as
-// layout-B register pairs, and for each layout-B element the byte offset of its gather source in
-// the warp's buffer (the permutation for P-FQJL, the identity otherwise).
+// Per-block tables of the key kernel. For each lane segment s (elements s*E .. s*E + E - 1) a
+// block holds three runs of E + 4 words: D_r as register pairs (d_{sE+t}, d_{sE+t+E/2}), D_g as
+// register pairs, and for each element i = s*E + r the byte offset of its gather source
+// j = pi(i) in the warp's buffer, 4 K (j + j/E) (the identity for D-FQJL). The 4-word pad puts
+// the segments of different lanes in different banks.
 std::vector<float> fqjl_key_tables(int d, int m, const float* D_r, const int32_t* perm, const float* D_g) {
   const Layout g = layout_for(d);
-  const int E = g.E, L = g.L, K = g.K, nb = m / d;
-  std::vector<float> t((size_t)nb * 3 * d);
-  auto elemA = [&](int r, int s) { return L == 1 ? r : (s >> 1) * 2 * E + 2 * r + (s & 1); };
+  const int E = g.E, L = g.L, K = g.K, nb = m / d, tseg = E + 4, tblk = 3 * L * tseg;
+  std::vector<float> t((size_t)nb * tblk, 0.f);
   for (int b = 0; b < nb; ++b) {
-    float* dr = t.data() + (size_t)b * 3 * d;
-    float* gp = dr + d;
-    int32_t* ro = reinterpret_cast<int32_t*>(dr + 2 * d);
+    float* blk = t.data() + (size_t)b * tblk;
     const float* Dr = D_r + (size_t)b * d;
     const float* Dg = D_g + (size_t)b * d;
     const int32_t* pi = perm + (size_t)b * d;
     for (int s = 0; s < L; ++s) {
+      float* dr = blk + s * tseg;
+      float* gp = blk + (L + s) * tseg;
+      int32_t* ro = reinterpret_cast<int32_t*>(blk + (2 * L + s) * tseg);
       for (int u = 0; u < E / 2; ++u) {
-        dr[s * E + 2 * u] = Dr[elemA(u, s)];
-        dr[s * E + 2 * u + 1] = Dr[elemA(u + E / 2, s)];
-        gp[s * E + 2 * u] = Dg[s * E + u];
-        gp[s * E + 2 * u + 1] = Dg[s * E + u + E / 2];
+        dr[2 * u] = Dr[s * E + u];
+        dr[2 * u + 1] = Dr[s * E + u + E / 2];
+        gp[2 * u] = Dg[s * E + u];
+        gp[2 * u + 1] = Dg[s * E + u + E / 2];
       }
       for (int r = 0; r < E; ++r) {
         const int j = pi[s * E + r];
-        ro[s * E + r] = 4 * K * (j + 2 * (j / (2 * E)));
+        ro[r] = 4 * K * (j + j / E);
       }
     }
   }

@@ -22,7 +22,7 @@ struct qjl_projection {
   float* D_r = nullptr;
   int32_t* perm = nullptr;
   float* D_g = nullptr;
-  float* ktab = nullptr;        // key-kernel tables, 3d words per block (fqjl_key_tables)
+  float* ktab = nullptr;        // key-kernel tables, per block (fqjl_key_tables)
   // host copies for export
   float* h_S = nullptr;
   float* h_D_r = nullptr;
