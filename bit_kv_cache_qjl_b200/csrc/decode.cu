@@ -250,22 +250,28 @@ __device__ __forceinline__ void mma_u8s8_zero(int (&d)[4], uint32_t a0, uint32_t
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
-// acc_c += (p s) (code_c 4^c) for this lane's CPL channels and accz += p z.
-// code_c 4^c = float(2^23 | (cwd & (3 << 2c))) - 2^23 exactly (the bits sit in
-// the mantissa), so no shift or int-to-float conversion is needed. Channel
-// pairs go through sm_100's packed fp32 subtract and FMA.
-template <int CPL>
-__device__ __forceinline__ void pv_accum(uint32_t cwd, uint16_t sraw, uint16_t zraw, float pt, float (&acc)[CPL],
-                                         float& accz) {
+// acc_j += (p s) (code_j 4^(j % 8)) for this lane's PL channels of one token, and accz += p z.
+// The lane's channels are c0 .. c0 + PL - 1 (one 32-channel group). The code words are read in
+// 8-channel chunks (16 bits each), so code_j 4^(j % 8) = float(2^23 | (chunk & (3 << 2(j % 8))))
+// - 2^23 exactly: the bits stay in the mantissa, and no int-to-float conversion is needed.
+// Channel pairs go through sm_100's packed fp32 subtract and FMA.
+template <int PL>
+__device__ __forceinline__ void pv_accum(const uint32_t* cw, int c0, uint16_t sraw, uint16_t zraw, float pt,
+                                         float (&acc)[PL], float& accz) {
   const float pw = pt * __half2float(__ushort_as_half(sraw));
   accz = fmaf(pt, __half2float(__ushort_as_half(zraw)), accz);
-  if constexpr (CPL == 1) {
-    acc[0] = fmaf(pw, __uint_as_float(0x4B000000u | (cwd & 3u)) - 8388608.f, acc[0]);
-  } else {
+  constexpr int NCH = PL < 8 ? 1 : PL / 8;     // 8-channel chunks
+  constexpr int CL = PL < 8 ? PL : 8;          // channels per chunk
 #pragma unroll
-    for (int c = 0; c < CPL; c += 2) {
-      const uint32_t u0 = 0x4B000000u | (cwd & (3u << (2 * c)));
-      const uint32_t u1 = 0x4B000000u | (cwd & (3u << (2 * c + 2)));
+  for (int h = 0; h < NCH; ++h) {
+    // chunk h covers channels c0 + 8h ..; it sits in word (c0 + 8h) / 16 at bit 2 ((c0 + 8h) % 16)
+    const uint32_t chunk = PL < 16 ? cw[0] >> (2 * ((c0 + 8 * h) & 15)) : cw[h >> 1] >> (16 * (h & 1));
+#pragma unroll
+    for (int k = 0; k < CL; k += 2) {
+      const uint32_t u0 = 0x4B000000u | (chunk & (3u << (2 * k)));
+      const uint32_t u1 = 0x4B000000u | (chunk & (3u << (2 * k + 2)));
+      float& a0 = acc[8 * h + k];
+      float& a1 = acc[8 * h + k + 1];
       asm("{\n\t.reg .b64 f, m, w, a;\n\t"
           "mov.b64 f, {%2, %3};\n\t"
           "mov.b64 m, {%4, %4};\n\t"
@@ -274,7 +280,7 @@ __device__ __forceinline__ void pv_accum(uint32_t cwd, uint16_t sraw, uint16_t z
           "mov.b64 a, {%0, %1};\n\t"
           "fma.rn.f32x2 a, w, f, a;\n\t"
           "mov.b64 {%0, %1}, a;\n\t}"
-          : "+f"(acc[c]), "+f"(acc[c + 1])
+          : "+f"(a0), "+f"(a1)
           : "r"(u0), "r"(u1), "f"(8388608.f), "f"(pw));
     }
   }
@@ -378,12 +384,18 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
   const float xmul = s_mul[0] * 0.03125f * logit_scale * 1.4426950408889634f;  // to log2-domain logits
   const int qs32 = 32 * s_qsum[0];
   const int gq = lane >> 2, q = lane & 3;
-  const int c0 = lane * CPL;
-  const int grp = c0 >> 5, cw = c0 >> 4, cshift = 2 * (c0 & 15);
+  // value accumulation: lane = 8 tg + cs takes channels c0 = cs PL .. c0 + PL - 1 of the tokens
+  // of group tg. At step j a warp covers four consecutive rows 4 (j & 3) + tg of its tile j / 4,
+  // so the four groups read adjacent tokens (conflict-free) and all fetch their probability from
+  // the same register (p0 for rows < 8, p1 above) of the MMA-layout lanes.
+  constexpr int PL = d / 8;
+  const int tg = lane >> 3, cs = lane & 7;
+  const int c0 = cs * PL;
+  const int grp = c0 >> 5, cwi = c0 >> 4;
 
-  float m_run = -INFINITY, l_lane = 0.f, accz = 0.f, acc[CPL];
+  float m_run = -INFINITY, l_lane = 0.f, accz = 0.f, acc[PL];
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
+  for (int c = 0; c < PL; ++c) acc[c] = 0.f;
   bool ok = true;
   int s = 0;
   uint32_t ph = 0;
@@ -467,38 +479,33 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
       l_lane *= corr;
       accz *= corr;
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) acc[c] *= corr;
+      for (int c = 0; c < PL; ++c) acc[c] *= corr;
       const float p0 = exp2f(x[0] - mn), p1 = exp2f(x[1] - mn);
       l_lane += p0 + p1;
-      // ---- p * v_hat: token (tile t2, row) is held by lane 4 (row % 8) + t2, register row / 8
+      // ---- p * v_hat: the token at (tile t2, row) has its p in lane 4 (row % 8) + t2, register row / 8
       if (cnt == kDsStage && nb_codes && nb_scale && nb_zero) {
         // whole stage in shared memory: no per-token bounds or source selection
-        const uint32_t* cp = scodes + cw;
-        const uint16_t* sp = sscale + grp;
-        const uint16_t* zp = szero + grp;
-#pragma unroll 1
-        for (int t2 = 0; t2 < KT; ++t2) {
-          const int tb = (warp + t2 * kDsConsumers) * 16;
 #pragma unroll
-          for (int row = 0; row < 16; ++row) {
-            const int tok = tb + row;
-            const float pt = __shfl_sync(0xffffffffu, row < 8 ? p0 : p1, 4 * (row & 7) + t2);
-            pv_accum<CPL>(cp[tok * CW] >> cshift, sp[tok * GW], zp[tok * GW], pt, acc, accz);
-          }
+        for (int j = 0; j < 16; ++j) {
+          const int t2 = j >> 2, row = 4 * (j & 3) + tg;
+          const int tok = (warp + t2 * kDsConsumers) * 16 + row;
+          const float pt = __shfl_sync(0xffffffffu, (j & 3) < 2 ? p0 : p1, 4 * (row & 7) + t2);
+          pv_accum<PL>(scodes + tok * CW + cwi, c0, sscale[tok * GW + grp], szero[tok * GW + grp], pt, acc, accz);
         }
       } else {
 #pragma unroll 1
-        for (int t2 = 0; t2 < KT; ++t2) {
+        for (int j = 0; j < 16; ++j) {
+          const int t2 = j >> 2, row = 4 * (j & 3) + tg;
+          const int tok = (warp + t2 * kDsConsumers) * 16 + row;
+          const float pt = __shfl_sync(0xffffffffu, (j & 3) < 2 ? p0 : p1, 4 * (row & 7) + t2);
+          if (tok >= cnt) continue;
+          uint32_t cwd[PL < 16 ? 1 : PL / 16];
 #pragma unroll
-          for (int row = 0; row < 16; ++row) {
-            const int tok = (warp + t2 * kDsConsumers) * 16 + row;
-            const float pt = __shfl_sync(0xffffffffu, row < 8 ? p0 : p1, 4 * (row & 7) + t2);
-            if (tok >= cnt) continue;
-            const uint32_t cwd = (nb_codes ? scodes[tok * CW + cw] : __ldg(codes + (row0 + tok) * CW + cw)) >> cshift;
-            const uint16_t sr = nb_scale ? sscale[tok * GW + grp] : __ldg(scale + (row0 + tok) * GW + grp);
-            const uint16_t zr = nb_zero ? szero[tok * GW + grp] : __ldg(zero + (row0 + tok) * GW + grp);
-            pv_accum<CPL>(cwd, sr, zr, pt, acc, accz);
-          }
+          for (int i = 0; i < (PL < 16 ? 1 : PL / 16); ++i)
+            cwd[i] = nb_codes ? scodes[tok * CW + cwi + i] : __ldg(codes + (row0 + tok) * CW + cwi + i);
+          const uint16_t sr = nb_scale ? sscale[tok * GW + grp] : __ldg(scale + (row0 + tok) * GW + grp);
+          const uint16_t zr = nb_zero ? szero[tok * GW + grp] : __ldg(zero + (row0 + tok) * GW + grp);
+          pv_accum<PL>(cwd, c0, sr, zr, pt, acc, accz);
         }
       }
     }
@@ -512,9 +519,19 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
   float l_w = l_lane;
 #pragma unroll
   for (int o = 16; o; o >>= 1) l_w += __shfl_xor_sync(0xffffffffu, l_w, o);
-  float* red = s_red + warp * (d + 2);
+  // the four token groups hold the same channels: add them (lanes cs, cs + 8, cs + 16, cs + 24)
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) red[2 + c0 + c] = acc[c] * (1.0f / (float)(1 << (2 * c))) + accz;
+  for (int c = 0; c < PL; ++c) {
+    acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 8);
+    acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], 16);
+  }
+  accz += __shfl_xor_sync(0xffffffffu, accz, 8);
+  accz += __shfl_xor_sync(0xffffffffu, accz, 16);
+  float* red = s_red + warp * (d + 2);
+  if (tg == 0) {
+#pragma unroll
+    for (int c = 0; c < PL; ++c) red[2 + c0 + c] = acc[c] * (1.0f / (float)(1 << (2 * (c & 7)))) + accz;
+  }
   if (lane == 0) {
     red[0] = m_run;
     red[1] = l_w;
