@@ -38,6 +38,15 @@ METRIC = "QJL decode scores keys/s (HBM GB/s vs ~8 TB/s); key-quantize vectors/s
 WORKLOAD = "decode_llama7b"
 B, H, N, D, M = 8, 32, 32768, 128, 256
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# FP32 issue ceiling of the ALU-bound transform: 148 SMs x 128 FP32 lanes x 1.965 GHz (max SM clock),
+# one add or multiply per lane per clock.
+FP32_TFLOPS = 148 * 128 * 1.965e9 / 1e12
+
+
+def fqjl_flops_per_key(d, m):
+    """Algorithmic fp32 operations of the FQJL map per key: per block, D_r and D_g (d multiplies
+    each) and two Walsh-Hadamard transforms (d log2 d additions each)."""
+    return 2 * m * (int(math.log2(d)) + 1)
 
 
 
@@ -118,7 +127,9 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(mhz)}
 
 
-def dist_setup():
+def dist_setup(backend=None):
+    """One process per GPU under torchrun: (world, rank, local rank). NCCL on GPUs; gloo when no
+    GPU is visible (the CPU tests of the multi-rank path)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -126,18 +137,24 @@ def dist_setup():
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
 
 
 def max_over_ranks(x, world):
+    """The max of a per-rank scalar over all ranks (the job's time is the slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -146,6 +163,11 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+def job_throughput(units_per_rank, world, ms_step_max):
+    """Whole-job units per second: every rank processed units_per_rank in the slowest rank's time."""
+    return world * units_per_rank / (ms_step_max * 1e-3)
 
 
 def cpu_oracle_rate(sample_keys, seconds_hint=None):
@@ -327,7 +349,7 @@ def build_workload(name, dev, qjl, wl, torch):
         out = torch.empty((1, J, ns), dtype=torch.float32, device=dev)
         stages = [
             Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), n,
-                  2 * d + m // 8 + 4, 0, "fqjl_kernel", "fqjl.cu", "alu"),
+                  2 * d + m // 8 + 4, fqjl_flops_per_key(d, m), "fqjl_keys_kernel", "fqjl_keys.cu", "alu"),
             Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), J, 4 * d + 4 * m),
             Stage("scores", lambda: qjl.scores(P, bits[:ns].view(1, ns, m // 32), norms[:ns].view(1, ns),
                                                sq.view(1, J, m), out=out), ns, m // 8 + 4 + 4 * J, 0,
@@ -354,7 +376,7 @@ def build_workload(name, dev, qjl, wl, torch):
         smx = 1.0 / math.sqrt(D)
         stages = [
             Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), G * Nd,
-                  2 * D + m // 8 + 4, 0, "fqjl_kernel", "fqjl.cu", "alu"),
+                  2 * D + m // 8 + 4, fqjl_flops_per_key(D, m), "fqjl_keys_kernel", "fqjl_keys.cu", "alu"),
             Stage("quantize_values", lambda: qjl.quantize_values_2bit(vals, codes=codes, scale=sc, zero=zr), G * Nd,
                   2 * D + D // 4 + D // 8, 0, "values_2bit_kernel", "values.cu"),
             Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * m),
@@ -434,7 +456,7 @@ def main():
     ms_step = ms_total / args.steps
     k_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(len(stages))]
     units = Wk["units"]
-    value = world * units / (ms_step * 1e-3)
+    value = job_throughput(units, world, ms_step)
 
     # end to end through the same calls with host buffers (pinned), copies inside the timed region
     h_in = []
@@ -483,12 +505,21 @@ def main():
             "unit": "GB/s", "frac": d_gbs / hbm, "peak_kind": pk_kind,
             "traffic": ncu_traffic(ds.kernel, args.workload, ds.src) if ds.src else None,
             "bytes_per_launch": ds.units * ds.bytes_per_unit}
-    if ds.flops_per_unit:
+    if ds.bound == "alu":
+        # the Walsh-Hadamard transform is bound by fp32 issue, not by HBM: report its fp32 operation
+        # rate against the FP32 lane ceiling, and keep the HBM fraction beside it
+        tfl = kernels[ds.name]["tflops"]
+        roof.update({"bound": "alu", "achieved": tfl, "peak": FP32_TFLOPS, "unit": "TFLOP/s",
+                     "frac": tfl / FP32_TFLOPS, "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 1.965 GHz",
+                     "flops_per_launch": ds.units * ds.flops_per_unit, "hbm_gbs": d_gbs, "hbm_frac": d_gbs / hbm})
+    elif ds.bound == "tensor":
+        tfl = kernels[ds.name]["tflops"]
+        roof.update({"bound": "tensor", "achieved": tfl, "peak": tf, "unit": "TFLOP/s", "frac": tfl / tf,
+                     "peak_kind": pk_kind + " (bf16, sustained)", "flops_per_launch": ds.units * ds.flops_per_unit,
+                     "hbm_gbs": d_gbs, "hbm_frac": d_gbs / hbm})
+    elif ds.flops_per_unit:
         roof["tensor_tflops"] = kernels[ds.name]["tflops"]
         roof["tensor_frac_of_sustained"] = kernels[ds.name]["tflops"] / tf
-    if ds.bound == "alu":
-        roof["note"] = ("the FQJL transform is bound by FP32/shuffle issue, not HBM; frac is the HBM fraction of its "
-                        "algorithmic bytes")
     clocks = clk.summary()
 
     cpu = None
