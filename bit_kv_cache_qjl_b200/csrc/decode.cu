@@ -396,14 +396,15 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
   float m_run = -INFINITY, l_lane = 0.f, accz = 0.f, acc[PL];
 #pragma unroll
   for (int c = 0; c < PL; ++c) acc[c] = 0.f;
-  bool ok = true;
+  bool dead = false;  // a timed-out wait: keep the loop's barriers, skip the work
   int s = 0;
   uint32_t ph = 0;
   for (int64_t k = 0; k < nst; ++k) {
     const int64_t n0 = t0 + k * kDsStage;
     const int cnt = (int)(t1 - n0 < kDsStage ? t1 - n0 : kDsStage);
     const int64_t row0 = gi * N + n0;
-    if (!mbar_wait(&full[s], ph)) { atomicOr(err, 4); ok = false; break; }
+    if (!dead && !__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { atomicOr(err, 4); dead = true; }
+    if (!dead) {
     const unsigned char* st = ring + (size_t)s * L.bytes;
     const uint32_t* sb = reinterpret_cast<const uint32_t*>(st + L.bits);
     const bool nb_norm = bulk_ok(norms + row0, (uint32_t)cnt * 4);
@@ -509,11 +510,11 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
         }
       }
     }
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
     if (++s == NS) { s = 0; ph ^= 1u; }
   }
-  if (!ok) return;
 
   // ---- merge the consumer warps: (m, l, acc[d]) per warp, then one partial per CTA
   float l_w = l_lane;

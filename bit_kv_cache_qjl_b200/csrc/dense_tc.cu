@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_tc_kernel(const __grid_cons
       const int64_t row = t * BM + r;
       for (int c = 0; c < nchunk; ++c, ++u) {
         const int buf = (int)(u & 1u);
-        if (!mbar_wait(&tfull[buf], (u >> 1) & 1u)) { flag_error(prm.err, 16); ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (u >> 1) & 1u))) { flag_error(prm.err, 16); ok = false; break; }
         tc_fence_after();
         const int N = min(256, m - 256 * c);
         const int hc = N >> 1;  // columns per half: 128 or 64
@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_tc_kernel(const __grid_cons
     int s = 0;
     uint32_t ph = 0;
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      if (!mbar_wait(&full[s], ph)) { flag_error(prm.err, 32); break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { flag_error(prm.err, 32); break; }
       const unsigned char* tile = sK + (size_t)s * kStageBytes;
       float acc[2][4];
 #pragma unroll

@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 1) scores_stream_kernel
   int64_t g = i0 / cpg, c = i0 - (i0 / cpg) * cpg;
   int s = 0;
   uint32_t ph = 0;
+  bool dead = false;  // a timed-out wait: keep the loop's barriers, skip the work
   for (int64_t it = i0; it < i1; ++it) {
     const int64_t n0 = c * kStageKeys;
     const int cnt = (int)(N - n0 < kStageKeys ? N - n0 : kStageKeys);
@@ -236,7 +237,8 @@ __global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 1) scores_stream_kernel
                       kConsumerWarps, 1);
       cur_g = g;
     }
-    if (!mbar_wait(&full[s], ph)) { atomicOr(err, 4); break; }
+    if (!dead && !__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { atomicOr(err, 4); dead = true; }
+    if (!dead) {
     const float* nsrc = norms + g * N + n0;
     const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
     const uint32_t* sb = sbits + (size_t)s * kStageKeys * W;
@@ -247,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 1) scores_stream_kernel
     for (int i = 0; i < kTilesPerWarp; i += KT)
       consume_tiles<W, NTR, KT>(warp + i * kConsumerWarps, sb, sn, nsrc, nbulk, cnt, Btab, s_mul, s_qsum, npass, J,
                                 N, g, n0, scores);
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
     if (++c == cpg) { c = 0; ++g; }
@@ -344,6 +347,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_decode_kernel(
   uint2 breg[W];
   float mul = 0.f;
   int qs32 = 0;
+  bool dead = false;  // a timed-out wait: keep the loop's barriers, skip the work
   for (int64_t it = i0; it < i1; ++it) {
     const int64_t n0 = c * SK;
     const int cnt = (int)(N - n0 < SK ? N - n0 : SK);
@@ -365,7 +369,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_decode_kernel(
       }
       cur_g = g;
     }
-    if (!mbar_wait(&full[s], ph)) { atomicOr(err, 4); break; }
+    if (!dead && !__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { atomicOr(err, 4); dead = true; }
+    if (!dead) {
     const float* nsrc = norms + g * N + n0;
     const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
     const uint32_t* sb = sbits + (size_t)s * SK * W;
@@ -483,6 +488,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_decode_kernel(
         }
       }
       }
+    }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);

@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(
     int npend = 0;
 
     auto epilogue = [&](const Pend& p) {
-      if (!mbar_wait(&dfull[p.buf], p.par)) { atomicOr(err, 16); ok = false; return; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&dfull[p.buf], p.par))) { atomicOr(err, 16); ok = false; return; }
       tc_fence_after();
       uint32_t dv[NC];
       tmem_ld<NC>(tmem_base + lane_off + d_col0 + (uint32_t)(p.buf * DS), dv);
@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(
                            s_mul + 4 * tb, s_qs + 4 * tb);
         cur_g = g;
       }
-      if (!mbar_wait(&full[s], ph)) { atomicOr(err, 32); break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { atomicOr(err, 32); break; }
       const uint32_t* sb = sbits + (size_t)s * kTileKeys * W + (size_t)r * W;
       uint32_t words[W];
 #pragma unroll
