@@ -440,8 +440,10 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
           const uint2 bb = breg[8 * p + 2 * Ji + sh];
 #pragma unroll
           for (int t2 = 0; t2 < KT; ++t2) {
-            const uint32_t a0 = (w0[t2][2 * p] >> sh) & M, a1 = (w1[t2][2 * p] >> sh) & M;
-            const uint32_t a2 = (w0[t2][2 * p + 1] >> sh) & M, a3 = (w1[t2][2 * p + 1] >> sh) & M;
+            // the odd bit of each pair straight from the word (weight 2 * 4^Ji; B holds Q / 2)
+            const uint32_t Ms = M << sh;
+            const uint32_t a0 = w0[t2][2 * p] & Ms, a1 = w1[t2][2 * p] & Ms;
+            const uint32_t a2 = w0[t2][2 * p + 1] & Ms, a3 = w1[t2][2 * p + 1] & Ms;
             if (p == 0 && sh == 0 && Ji == 0) mma_u8s8_zero(accm[t2], a0, a1, a2, a3, bb.x, bb.y);
             else mma_u8s8_acc(accm[t2], a0, a1, a2, a3, bb.x, bb.y);
           }

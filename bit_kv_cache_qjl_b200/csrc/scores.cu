@@ -21,7 +21,9 @@
 //     64 * sum b Q. The estimate is (2 sum b Q - sum Q) * scale, formed in
 //     int64 before one rounding to fp32.
 // The sign sums are exact. The only error is the 16-bit rounding of Sq:
-// at most m * max|Sq| / 65278 before scaling.
+// at most m * max|Sq| / 65278 before scaling. The single-query kernels use an
+// even grid instead (build_tables_cls), so the odd bits need no shift. Their
+// bound is m * max|Sq| / 32638.
 //
 // Layout: bits [G][N][W] uint32, norms [G][N], sq [G][J][m], scores [G][J][N].
 // Grid: (splits, G). Each CTA covers a contiguous range of 16-key tiles of
@@ -411,8 +413,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_decode_kernel(
               const uint2 bb = breg[8 * p + 2 * Ji + sh];
 #pragma unroll
               for (int t2 = 0; t2 < KT; ++t2) {
-                const uint32_t a0 = (w0[t2][2 * p] >> sh) & M, a1 = (w1[t2][2 * p] >> sh) & M;
-                const uint32_t a2 = (w0[t2][2 * p + 1] >> sh) & M, a3 = (w1[t2][2 * p + 1] >> sh) & M;
+                // the odd bit of each pair straight from the word (weight 2 * 4^Ji; B holds Q / 2)
+                const uint32_t Ms = M << sh;
+                const uint32_t a0 = w0[t2][2 * p] & Ms, a1 = w1[t2][2 * p] & Ms;
+                const uint32_t a2 = w0[t2][2 * p + 1] & Ms, a3 = w1[t2][2 * p + 1] & Ms;
                 if (p == 0 && sh == 0 && Ji == 0) mma_u8s8_zc(acc[t2], a0, a1, a2, a3, bb.x, bb.y);
                 else mma_u8s8(acc[t2], a0, a1, a2, a3, bb.x, bb.y);
               }

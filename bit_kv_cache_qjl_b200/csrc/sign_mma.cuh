@@ -12,6 +12,7 @@
 namespace qjl_sign {
 
 constexpr int kQmax = 32639;  // 127 * 256 + 127: both int8 halves stay in range
+constexpr int kQmaxE = 32638; // the even grid of the single-query tables (127 * 256 + 126)
 
 __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -25,6 +26,12 @@ __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, 
 __device__ __forceinline__ int quant16(float v, float inv) {
   const float q = rintf(v * inv);
   return (int)fminf(fmaxf(q, (float)-kQmax), (float)kQmax);
+}
+
+// 2 rint(v inv / 2), clamped to +-kQmaxE: an even 16-bit code
+__device__ __forceinline__ int quant16e(float v, float inv) {
+  const float q = rintf(v * inv * 0.5f);
+  return 2 * (int)fminf(fmaxf(q, (float)-(kQmaxE / 2)), (float)(kQmaxE / 2));
 }
 
 // Fills per-query scale data and the B fragments for group `gi`.
@@ -116,6 +123,12 @@ __device__ __forceinline__ void load_words(const uint32_t* __restrict__ base, in
 // hi (h = 0) or lo (h = 1) byte of Q for the coordinates whose A bytes have
 // weight 4^c, and zero elsewhere. All MMAs of a key tile can then accumulate
 // into one fragment, with class c landing in column pair c.
+//
+// Here Q lies on the even grid, Q = 2 rint(Sq kQmaxE / (2 max|Sq|)). So the
+// MMAs for the odd bit of each 2-bit pair (s = 1) can take A straight from the
+// unshifted word: their A bytes are worth 2 * 4^c, and their B entries hold
+// Q / 2, exactly. That saves one shift per A register. The rounding step of Sq
+// is twice the 16-bit one's.
 template <int W>
 __device__ void build_tables_cls(const float* __restrict__ sqg, float est_scale, float* s_inv, float* s_mul,
                                  int* s_qsum, uint2* Btab, int nwarps, int bar_id) {
@@ -127,14 +140,14 @@ __device__ void build_tables_cls(const float* __restrict__ sqg, float est_scale,
     for (int i = lane; i < m; i += 32) mx = fmaxf(mx, fabsf(sqg[i]));
 #pragma unroll
     for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float inv = mx > 0.f ? (float)kQmax / mx : 0.f;
+    const float inv = mx > 0.f ? (float)kQmaxE / mx : 0.f;
     int qs = 0;
-    for (int i = lane; i < m; i += 32) qs += quant16(sqg[i], inv);
+    for (int i = lane; i < m; i += 32) qs += quant16e(sqg[i], inv);
 #pragma unroll
     for (int o = 16; o; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
     if (lane == 0) {
       s_inv[0] = inv;
-      s_mul[0] = est_scale * (mx > 0.f ? mx / (float)kQmax : 0.f);
+      s_mul[0] = est_scale * (mx > 0.f ? mx / (float)kQmaxE : 0.f);
       s_qsum[0] = qs;
     }
   }
@@ -152,7 +165,8 @@ __device__ void build_tables_cls(const float* __restrict__ sqg, float est_scale,
         const int word = qq * (W / 4) + 2 * p + r;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int Q = quant16(sqg[32 * word + 8 * e + jb], inv);
+          // odd bits (jb & 1): A carries twice the weight, so B holds Q / 2
+          const int Q = quant16e(sqg[32 * word + 8 * e + jb], inv) >> (jb & 1);
           const int lo = (int)(int8_t)(Q & 0xFF);
           const int hi = (Q - lo) >> 8;
           b[r] |= ((uint32_t)(half ? lo : hi) & 0xFFu) << (8 * e);
