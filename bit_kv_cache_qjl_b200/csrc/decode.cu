@@ -302,6 +302,37 @@ __host__ __device__ inline DsLayout ds_layout(int W, int d) {
   return L;
 }
 
+// Work split of the one-query streaming kernel: the flattened (group, 16-token tile) space is cut
+// into ncta equal slices, one persistent CTA each (at least 64 tiles per CTA), so every SM runs
+// one uninterrupted ring. A CTA writes one partial per group its slice touches: at most maxseg.
+constexpr int64_t kStreamCTAs = 148;
+
+struct StreamPlan {
+  int64_t ntg, TT, ncta, maxseg;   // tiles per group, all tiles, CTAs, partial slots per CTA
+};
+
+__host__ __device__ inline StreamPlan stream_plan(int64_t G, int64_t N) {
+  StreamPlan p;
+  p.ntg = (N + 15) / 16;
+  p.TT = G * p.ntg;
+  const int64_t c = p.TT / 64;
+  p.ncta = c < 1 ? 1 : (c > kStreamCTAs ? kStreamCTAs : c);
+  const int64_t per = (p.TT + p.ncta - 1) / p.ncta;
+  p.maxseg = (per + p.ntg - 1) / p.ntg + 1;
+  return p;
+}
+
+// first tile of CTA c (c = ncta gives TT)
+__host__ __device__ inline int64_t stream_tile0(const StreamPlan& p, int64_t c) { return c * p.TT / p.ncta; }
+
+// the CTA whose slice holds tile t
+__host__ __device__ inline int64_t stream_cta_of(const StreamPlan& p, int64_t t) {
+  int64_t c = t * p.ncta / p.TT;
+  while (c + 1 < p.ncta && stream_tile0(p, c + 1) <= t) ++c;
+  while (c > 0 && stream_tile0(p, c) > t) --c;
+  return c;
+}
+
 __device__ __forceinline__ bool bulk_ok(const void* src, uint32_t bytes) {
   return (((uintptr_t)src & 15u) == 0) && (bytes % 16u == 0);
 }
@@ -309,9 +340,8 @@ __device__ __forceinline__ bool bulk_ok(const void* src, uint32_t bytes) {
 template <int W, int CPL>
 __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
     const uint32_t* __restrict__ bits, const float* __restrict__ norms, const uint32_t* __restrict__ codes,
-    const uint16_t* __restrict__ scale, const uint16_t* __restrict__ zero, const float* __restrict__ sq, int64_t N,
-    int NS, float est_scale, float logit_scale, int64_t tokens_per_cta, float* __restrict__ ws,
-    int* __restrict__ err) {
+    const uint16_t* __restrict__ scale, const uint16_t* __restrict__ zero, const float* __restrict__ sq, int64_t G,
+    int64_t N, int NS, float est_scale, float logit_scale, float* __restrict__ ws, int* __restrict__ err) {
   using namespace qjl_sync;
   constexpr int d = 32 * CPL;
   constexpr int CW = d / 16;  // code words per token
@@ -329,10 +359,10 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
   uint64_t* empty = full + NS;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t gi = blockIdx.y;
-  const int64_t t0 = (int64_t)blockIdx.x * tokens_per_cta;
-  const int64_t t1 = min(N, t0 + tokens_per_cta);
-  const int64_t nst = (t1 - t0 + kDsStage - 1) / kDsStage;
+  // this CTA's slice of the flattened (group, 16-token tile) space, cut into one segment per group
+  const StreamPlan plan = stream_plan(G, N);
+  const int64_t tb = stream_tile0(plan, blockIdx.x), te = stream_tile0(plan, blockIdx.x + 1);
+  const int64_t g_first = tb / plan.ntg, g_last = (te - 1) / plan.ntg;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -348,23 +378,30 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
       int s = 0;
       uint32_t ph = 0;
       int64_t issued = 0;
-      for (int64_t k = 0; k < nst; ++k, ++issued) {
-        if (!mbar_wait(&empty[s], ph ^ 1u)) { atomicOr(err, 1); break; }
-        const int64_t n0 = t0 + k * kDsStage;
-        const uint32_t cnt = (uint32_t)(t1 - n0 < kDsStage ? t1 - n0 : kDsStage);
-        const int64_t row = gi * N + n0;
-        unsigned char* st = ring + (size_t)s * L.bytes;
-        const void* src[5] = {bits + row * W, norms + row, codes + row * CW, scale + row * GW, zero + row * GW};
-        const uint32_t nb[5] = {cnt * W * 4, cnt * 4, cnt * CW * 4, cnt * GW * 2, cnt * GW * 2};
-        const uint32_t off[5] = {L.bits, L.norms, L.codes, L.scale, L.zero};
-        uint32_t tx = 0;
-        for (int a = 0; a < 5; ++a)
-          if (bulk_ok(src[a], nb[a])) tx += nb[a];
-        mbar_expect_tx(&full[s], tx);
-        for (int a = 0; a < 5; ++a)
-          if (bulk_ok(src[a], nb[a])) bulk_g2s(st + off[a], src[a], nb[a], &full[s]);
-        if (++s == NS) { s = 0; ph ^= 1u; }
+      bool stop = false;
+      for (int64_t gi = g_first; gi <= g_last && !stop; ++gi) {
+        const int64_t t0 = 16 * (max(tb, gi * plan.ntg) - gi * plan.ntg);
+        const int64_t t1 = min(N, 16 * (min(te, (gi + 1) * plan.ntg) - gi * plan.ntg));
+        const int64_t nst = (t1 - t0 + kDsStage - 1) / kDsStage;
+        for (int64_t k = 0; k < nst; ++k, ++issued) {
+          if (!mbar_wait(&empty[s], ph ^ 1u)) { atomicOr(err, 1); stop = true; break; }
+          const int64_t n0 = t0 + k * kDsStage;
+          const uint32_t cnt = (uint32_t)(t1 - n0 < kDsStage ? t1 - n0 : kDsStage);
+          const int64_t row = gi * N + n0;
+          unsigned char* st = ring + (size_t)s * L.bytes;
+          const void* src[5] = {bits + row * W, norms + row, codes + row * CW, scale + row * GW, zero + row * GW};
+          const uint32_t nb[5] = {cnt * W * 4, cnt * 4, cnt * CW * 4, cnt * GW * 2, cnt * GW * 2};
+          const uint32_t off[5] = {L.bits, L.norms, L.codes, L.scale, L.zero};
+          uint32_t tx = 0;
+          for (int a = 0; a < 5; ++a)
+            if (bulk_ok(src[a], nb[a])) tx += nb[a];
+          mbar_expect_tx(&full[s], tx);
+          for (int a = 0; a < 5; ++a)
+            if (bulk_ok(src[a], nb[a])) bulk_g2s(st + off[a], src[a], nb[a], &full[s]);
+          if (++s == NS) { s = 0; ph ^= 1u; }
+        }
       }
+      // do not leave while copies are in flight
       const int used = issued < NS ? (int)issued : NS;
       for (int j = 0; j < used; ++j) {
         int stg = s - 1 - j;
@@ -376,7 +413,14 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
     return;
   }
 
-  // consumers
+  // consumers: one segment (one group) at a time; the ring carries on across segments
+  int s = 0;
+  uint32_t ph = 0;
+  bool dead = false;  // a timed-out wait: keep the loop's barriers, skip the work
+  for (int64_t gi = g_first; gi <= g_last; ++gi) {
+  const int64_t t0 = 16 * (max(tb, gi * plan.ntg) - gi * plan.ntg);
+  const int64_t t1 = min(N, 16 * (min(te, (gi + 1) * plan.ntg) - gi * plan.ntg));
+  const int64_t nst = (t1 - t0 + kDsStage - 1) / kDsStage;
   build_tables_cls<W>(sq + gi * (int64_t)(32 * W), est_scale, s_inv, s_mul, s_qsum, Btab, kDsConsumers, 1);
   uint2 breg[W];
 #pragma unroll
@@ -396,9 +440,6 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
   float m_run = -INFINITY, l_lane = 0.f, accz = 0.f, acc[PL];
 #pragma unroll
   for (int c = 0; c < PL; ++c) acc[c] = 0.f;
-  bool dead = false;  // a timed-out wait: keep the loop's barriers, skip the work
-  int s = 0;
-  uint32_t ph = 0;
   for (int64_t k = 0; k < nst; ++k) {
     const int64_t n0 = t0 + k * kDsStage;
     const int cnt = (int)(t1 - n0 < kDsStage ? t1 - n0 : kDsStage);
@@ -540,8 +581,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
     red[1] = l_w;
   }
   named_sync(1, kDsConsumers * 32);
-  const int64_t split = blockIdx.x;
-  const int64_t nsplit = gridDim.x;
+  const int64_t slot = (int64_t)blockIdx.x * plan.maxseg + (gi - g_first);
   for (int idx = threadIdx.x; idx < d + 2; idx += kDsConsumers * 32) {
     float M = -INFINITY;
     for (int w = 0; w < kDsConsumers; ++w) M = fmaxf(M, s_red[w * (d + 2)]);
@@ -555,7 +595,37 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
         v += f * s_red[w * (d + 2) + idx];
       }
     }
-    ws[(gi * nsplit + split) * (d + 2) + idx] = v;
+    ws[slot * (d + 2) + idx] = v;
+  }
+  }  // segments
+}
+
+// The one-query partials of group g: the CTAs whose tile ranges meet g's tiles, each in slot
+// (c, g - first group of c). out[g][c] = sum acc 2^(m - M) / sum l 2^(m - M).
+__global__ void __launch_bounds__(128) decode_combine_stream_kernel(const float* __restrict__ ws, int64_t G, int64_t N,
+                                                                    int d, float* __restrict__ out) {
+  const int64_t g = blockIdx.x;
+  if (g >= G) return;
+  const StreamPlan plan = stream_plan(G, N);
+  const int64_t c_lo = stream_cta_of(plan, g * plan.ntg), c_hi = stream_cta_of(plan, (g + 1) * plan.ntg - 1);
+  auto entry = [&](int64_t c) {
+    return ws + (c * plan.maxseg + (g - stream_tile0(plan, c) / plan.ntg)) * (d + 2);
+  };
+  float M = -INFINITY;
+  for (int64_t c = c_lo; c <= c_hi; ++c) M = fmaxf(M, entry(c)[0]);
+  float Lsum = 0.f;
+  for (int64_t c = c_lo; c <= c_hi; ++c) {
+    const float* e = entry(c);
+    Lsum += (e[0] == -INFINITY) ? 0.f : e[1] * exp2f(e[0] - M);
+  }
+  const float invL = 1.f / Lsum;
+  for (int ch = threadIdx.x; ch < d; ch += blockDim.x) {
+    float v = 0.f;
+    for (int64_t c = c_lo; c <= c_hi; ++c) {
+      const float* e = entry(c);
+      if (e[0] != -INFINITY) v += e[2 + ch] * exp2f(e[0] - M);
+    }
+    out[g * d + ch] = v * invL;
   }
 }
 
@@ -627,19 +697,14 @@ qjl_status launch_stream(const qjl_projection* P, const uint32_t* bits, const fl
     return qjl_check_launch("decode_stream_kernel smem attribute");
   int* err = qjl_error_flag(P->device);
   if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
-  const int64_t splits = decode_splits(G, N);
-  const int64_t ntiles = (N + 15) / 16;
-  const int64_t tpc = 16 * ((ntiles + splits - 1) / splits);  // tokens per CTA, as the tile-based kernel splits
-  const int64_t nsplit = (N + tpc - 1) / tpc;
-  if (nsplit != splits) return qjl_set_error(QJL_ERR_UNSUPPORTED, "internal split mismatch");
-  dim3 grid((unsigned)splits, (unsigned)G);
-  qjl_log_launch("decode_stream_kernel", (int64_t)splits * G, kDsThreads, smem, 1);
-  kern<<<grid, kDsThreads, smem, st>>>(bits, norms, codes, scale, zero, sq, N, NS, P->est_scale, softmax_scale, tpc,
-                                       ws, err);
+  const StreamPlan plan = stream_plan(G, N);
+  qjl_log_launch("decode_stream_kernel", plan.ncta, kDsThreads, smem, 1);
+  kern<<<(unsigned)plan.ncta, kDsThreads, smem, st>>>(bits, norms, codes, scale, zero, sq, G, N, NS, P->est_scale,
+                                                      softmax_scale, ws, err);
   qjl_status s = qjl_check_launch("decode_stream_kernel");
   if (s != QJL_OK) return s;
-  decode_combine_kernel<<<(unsigned)G, 128, 0, st>>>(ws, G, 1, d, splits, out);
-  return qjl_check_launch("decode_combine_kernel");
+  decode_combine_stream_kernel<<<(unsigned)G, 128, 0, st>>>(ws, G, N, d, out);
+  return qjl_check_launch("decode_combine_stream_kernel");
 }
 
 template <int W>
@@ -667,6 +732,11 @@ qjl_status launch_w(const qjl_projection* P, const uint32_t* bits, const float* 
 }  // namespace
 
 size_t decode_workspace_bytes(int64_t G, int J, int64_t N, int d) {
+  if (J == 1) {
+    // the one-query kernel: maxseg partial slots per persistent CTA
+    const StreamPlan p = stream_plan(G, N);
+    return (size_t)p.ncta * (size_t)p.maxseg * (size_t)(d + 2) * sizeof(float);
+  }
   return (size_t)G * (size_t)decode_splits(G, N) * (size_t)J * (size_t)(d + 2) * sizeof(float);
 }
 

@@ -72,7 +72,8 @@ def test_values_and_decode_kernels(cuda_ok):
         c, s, z = qjl.quantize_values_2bit(v)
         qjl.decode_attention(P, bits, norms, c.view(2, 300, 8), s.view(2, 300, 4), z.view(2, 300, 4), sq, 0.1)
     names = _kernels(lambda: run(1))
-    for k in ("values_2bit_kernel", "decode_stream_kernel", "decode_combine_kernel"):
+    for k in ("values_2bit_kernel", "decode_stream_kernel", "decode_combine_stream_kernel"):
         assert _has(names, k), (k, names)
-    # several queries per group take the tile-per-warp kernel
-    assert _has(_kernels(lambda: run(2)), "decode_partial_kernel")
+    # several queries per group take the tile-per-warp kernel and the split combine
+    names = _kernels(lambda: run(2))
+    assert _has(names, "decode_partial_kernel") and _has(names, "decode_combine_kernel"), names
