@@ -404,7 +404,7 @@ def main():
                     choices=["decode_llama7b", "gqa_decode", "dense_1head", "pfqjl_bulk_m256", "pfqjl_bulk_m1024",
                              "dfqjl_decode"])
     ap.add_argument("--ref-sample", type=int, default=4096)
-    ap.add_argument("--cpu-sample", type=int, default=1 << 18)
+    ap.add_argument("--cpu-sample", type=int, default=1 << 21)
     ap.add_argument("--profile-case", default=None,
                     choices=["quantize", "scores", "fqjl", "fqjl1024", "dfqjl", "values", "decode"],
                     help="run one small case of a single kernel (3 launches after 2 warm-ups) for ncu")
