@@ -5,30 +5,29 @@
 // whole cache is loaded per generated token), so the kernel must stay at the
 // HBM roof, where each SM has under two clocks per 40-byte key. A plain
 // bit-serial sign-dot costs several instructions per bit, and on sm_100a the
-// 1-bit mma.sync is emulated, so the sign sums run on the s8 tensor-core
-// path instead:
+// 1-bit and 4-bit mma.sync forms are emulated, so the sign sums run on the
+// u8 x s8 tensor-core path (mma.sync m16n8k32). A u8 A element carries at
+// most one new bit per byte against arbitrary weights, so a 32-bit sign word
+// needs eight A registers (32 k-slots); two ways of building them are used:
 //
-//   * Sq is rounded per (group, query) to 16-bit fixed point,
-//     Q = rint(Sq * 32639 / max|Sq|), and split as Q = 256 hi + lo with
-//     int8 halves. Columns 2j and 2j+1 of an n8 B tile hold hi and lo of
-//     query j, so one tile serves 4 queries.
-//   * A 16-key x 32-k A tile takes 32 bits from each key. A register is
-//     (word >> s) & (0x01010101 << J): four bits (8e + J + s), e = 0..3, of
-//     one word, each worth 2^J. That is one AND per 4 bits, with no
-//     unpacking. The k order is free as long as the B tile uses the same
-//     order, so B is laid out to match.
-//   * Four accumulators (J = 0, 2, 4, 6) are merged exactly in int32 as
-//     64 * sum b Q. The estimate is (2 sum b Q - sum Q) * scale, formed in
-//     int64 before one rounding to fp32.
-// The sign sums are exact. The only error is the 16-bit rounding of Sq:
-// at most m * max|Sq| / 65278 before scaling. The single-query kernels use an
-// even grid instead (build_tables_cls), so the odd bits need no shift. Their
-// bound is m * max|Sq| / 32638.
+//   * Shift windows (one or two queries per group, build_tables_dig in
+//     sign_mma.cuh): the eight registers are the word shifted right by
+//     s = 0..7, unmasked, and B holds Q times the inverse of the windows'
+//     unit-triangular weight matrix, modulo 2^32, as four int8 digits in four
+//     columns. Seven shifts per word, and Sq keeps 31 - log2(m) bits.
+//   * Weight classes (three or four queries, build_tables): Sq is rounded to
+//     16-bit fixed point and split into int8 hi/lo columns, so one n8 tile
+//     serves four queries. A register is (word >> s) & (0x01010101 << 2c):
+//     four bits worth 4^c, one AND per 4 bits. Four accumulators (c = 0..3)
+//     are merged exactly in int32. Its only error is the 16-bit rounding of
+//     Sq, at most m * max|Sq| / 65278 before scaling.
+// In both, the sign sums are exact integers; the estimate is
+// (2 sum b Q - sum Q) times the scale, converted to fp32 once.
 //
 // Layout: bits [G][N][W] uint32, norms [G][N], sq [G][J][m], scores [G][J][N].
-// Grid: (splits, G). Each CTA covers a contiguous range of 16-key tiles of
-// one group, and each warp streams every 8th tile with the next tile's words
-// prefetched into registers.
+// Keys stream through a shared-memory ring filled by cp.async.bulk from one
+// producer lane; persistent CTAs each take a contiguous range of (group,
+// stage) items.
 
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -278,14 +277,14 @@ __device__ __forceinline__ void mma_u8s8_zc(int (&d)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
-template <int W, bool CLS>
+template <int W>
 __global__ void __launch_bounds__(kDecThreads, 2) scores_decode_kernel(
     const uint32_t* __restrict__ bits, const float* __restrict__ norms, const float* __restrict__ sq,
     int64_t G, int64_t N, int J, int NS, float est_scale, int64_t items_per_cta, float* __restrict__ scores,
     int* __restrict__ err) {
   using namespace qjl_sync;
   constexpr int SK = kDecStageKeys;
-  constexpr int KT = CLS ? 4 : 2;   // tiles whose MMA chains are interleaved per warp
+  constexpr int KT = 2;   // tiles whose MMA chains are interleaved per warp
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* s_inv = reinterpret_cast<float*>(smem_raw);
   float* s_mul = s_inv + 64;
@@ -355,20 +354,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_decode_kernel(
     const int cnt = (int)(N - n0 < SK ? N - n0 : SK);
     if (g != cur_g) {
       named_sync(1, kDecConsumers * 32);
-      if constexpr (CLS)
-        build_tables_cls<W>(sq + g * (int64_t)(32 * W), est_scale, s_inv, s_mul, s_qsum, Btab, kDecConsumers, 1);
-      else
-        build_tables<W>(sq + g * (int64_t)J * (32 * W), J, 1, est_scale, s_inv, s_mul, s_qsum, Btab, kDecConsumers,
-                        1);
+      build_tables<W>(sq + g * (int64_t)J * (32 * W), J, 1, est_scale, s_inv, s_mul, s_qsum, Btab, kDecConsumers,
+                      1);
 #pragma unroll
       for (int mu = 0; mu < W; ++mu) breg[mu] = Btab[mu * 32 + lane];
-      if constexpr (CLS) {
-        mul = s_mul[0] * 0.03125f;
-        qs32 = 32 * s_qsum[0];
-      } else {
-        mul = q < J ? s_mul[q] * 0.03125f : 0.f;
-        qs32 = q < J ? 32 * s_qsum[q] : 0;
-      }
+      mul = q < J ? s_mul[q] * 0.03125f : 0.f;
+      qs32 = q < J ? 32 * s_qsum[q] : 0;
       cur_g = g;
     }
     if (!dead && !__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { atomicOr(err, 4); dead = true; }
@@ -377,7 +368,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_decode_kernel(
     const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
     const uint32_t* sb = sbits + (size_t)s * SK * W;
     const float* sn = snorm + (size_t)s * SK;
-    float* gout = scores + (g * J + (CLS ? 0 : q)) * N + n0;
+    float* gout = scores + (g * J + q) * N + n0;
 #pragma unroll 1
     for (int i = 0; i < kDecTilesPerWarp; i += KT) {
       const int tile0 = warp + i * kDecConsumers;
@@ -400,61 +391,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_decode_kernel(
           }
         }
       }
-      if constexpr (CLS) {
-        // all 8 W/8 MMAs of a tile into one fragment; class Ji lands in column pair Ji
-        int acc[KT][4];
-#pragma unroll
-        for (int p = 0; p < W / 8; ++p) {
-#pragma unroll
-          for (int sh = 0; sh < 2; ++sh) {
-#pragma unroll
-            for (int Ji = 0; Ji < 4; ++Ji) {
-              const uint32_t M = 0x01010101u << (2 * Ji);
-              const uint2 bb = breg[8 * p + 2 * Ji + sh];
-#pragma unroll
-              for (int t2 = 0; t2 < KT; ++t2) {
-                // the odd bit of each pair straight from the word (weight 2 * 4^Ji; B holds Q / 2)
-                const uint32_t Ms = M << sh;
-                const uint32_t a0 = w0[t2][2 * p] & Ms, a1 = w1[t2][2 * p] & Ms;
-                const uint32_t a2 = w0[t2][2 * p + 1] & Ms, a3 = w1[t2][2 * p + 1] & Ms;
-                if (p == 0 && sh == 0 && Ji == 0) mma_u8s8_zc(acc[t2], a0, a1, a2, a3, bb.x, bb.y);
-                else mma_u8s8(acc[t2], a0, a1, a2, a3, bb.x, bb.y);
-              }
-            }
-          }
-        }
-        // lane (g, q) holds class q: (hi, lo) of rows g and g + 8. Weight class q by
-        // 4^(3-q) so the sum over the four lanes is 64 * sum b Q, exactly.
-        const int sft = 2 * (3 - q);
-        int v[KT][2];
-#pragma unroll
-        for (int t2 = 0; t2 < KT; ++t2)
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            int x = (acc[t2][2 * r] * 256 + acc[t2][2 * r + 1]) << sft;
-            x += __shfl_xor_sync(0xffffffffu, x, 1);
-            x += __shfl_xor_sync(0xffffffffu, x, 2);
-            v[t2][r] = x;
-          }
-        // the quad's KT tiles x 2 rows: lane q finishes tile q (both rows) when
-        // KT == 4, or row (q & 1) of tile (q >> 1) when KT == 2
-#pragma unroll
-        for (int k = 0; k < KT / 2; ++k) {
-          const int t2s = (KT == 4) ? q : (q >> 1);
-          const int rs = (KT == 4) ? k : (q & 1);
-          int mine = v[0][0];
-#pragma unroll
-          for (int t2 = 0; t2 < KT; ++t2)
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-              if (t2 == t2s && r == rs) mine = v[t2][r];
-          const int row = (tile0 + t2s * kDecConsumers) * 16 + gq + 8 * rs;
-          if (row < cnt) {
-            const float nrm = nbulk ? sn[row] : __ldg(nsrc + row);
-            gout[row] = mul * nrm * (float)(mine - qs32);
-          }
-        }
-      } else {
       int acc[KT][4][4];
 #pragma unroll
       for (int p = 0; p < W / 8; ++p) {
@@ -491,12 +427,237 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_decode_kernel(
           }
         }
       }
-      }
     }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
     if (++c == cpg) { c = 0; ++g; }
+    if (++s == NS) { s = 0; ph ^= 1u; }
+  }
+}
+
+// Decode scores with shift-window digit sums (build_tables_dig): the A
+// fragments are the sign words shifted right by s = 0..7, unmasked, so a
+// 16-key tile costs 7 shifts per word and W MMAs per column tile of two
+// queries. The stage ring and producer are those of scores_decode_kernel,
+// with SKT keys per stage. With DUP (one query per group) both halves of the
+// B tile carry the same digits, and lanes q = 2, 3 finish the odd tiles while
+// lanes 0, 1 finish the even ones.
+
+// Finishes KT tiles: lane (gq, q) holds digits (2 par, 2 par + 1) of rows gq and
+// gq + 8. P_r is its part of sum b Q for row r, and the pair (q, q ^ 1)
+// completes row par. CHECK guards rows past cnt and unaligned norms.
+template <int NT, bool DUP, int KT, bool CHECK>
+__device__ __forceinline__ void digit_epilogue(const int (&acc)[KT][NT][4], int tile0, int gq, int par, int half,
+                                               int cnt, bool nbulk, const float* __restrict__ sn,
+                                               const float* __restrict__ nsrc, const float (&mul)[NT],
+                                               const uint32_t (&qs)[NT], int J, int64_t N,
+                                               float* __restrict__ gout) {
+  const uint32_t hm = par ? 65536u : 1u;  // lanes with odd q hold digits 2, 3
+  if constexpr (DUP) {
+#pragma unroll
+    for (int k = 0; k < KT / 2; ++k) {
+      int cc[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) cc[j] = half ? acc[2 * k + 1][0][j] : acc[2 * k][0][j];
+      const uint32_t P0 = (uint32_t)cc[0] * hm + (uint32_t)cc[1] * (hm << 8);
+      const uint32_t P1 = (uint32_t)cc[2] * hm + (uint32_t)cc[3] * (hm << 8);
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, par ? P0 : P1, 1);
+      const uint32_t tot = (par ? P1 : P0) + recv;
+      const int row = (tile0 + (2 * k + half) * kDecConsumers) * 16 + gq + 8 * par;
+      if (!CHECK || row < cnt) {
+        const float nrm = (!CHECK || nbulk) ? sn[row] : __ldg(nsrc + row);
+        gout[row] = mul[0] * nrm * (float)(int)(2u * tot - qs[0]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int jq = 2 * nt + half;
+#pragma unroll
+      for (int t = 0; t < KT; ++t) {
+        const uint32_t P0 = (uint32_t)acc[t][nt][0] * hm + (uint32_t)acc[t][nt][1] * (hm << 8);
+        const uint32_t P1 = (uint32_t)acc[t][nt][2] * hm + (uint32_t)acc[t][nt][3] * (hm << 8);
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, par ? P0 : P1, 1);
+        const uint32_t tot = (par ? P1 : P0) + recv;
+        const int row = (tile0 + t * kDecConsumers) * 16 + gq + 8 * par;
+        if (jq < J && (!CHECK || row < cnt)) {
+          const float nrm = (!CHECK || nbulk) ? sn[row] : __ldg(nsrc + row);
+          gout[jq * N + row] = mul[nt] * nrm * (float)(int)(2u * tot - qs[nt]);
+        }
+      }
+    }
+  }
+}
+
+template <int W, int NT, bool DUP, int KT, int SKT>
+__global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
+    const uint32_t* __restrict__ bits, const float* __restrict__ norms, const float* __restrict__ sq,
+    int64_t G, int64_t N, int J, int NS, float est_scale, int64_t items_per_cta, float* __restrict__ scores,
+    int* __restrict__ err) {
+  using namespace qjl_sync;
+  constexpr int SK = SKT;
+  constexpr int TPW = SK / 16 / kDecConsumers;  // tiles per consumer warp per stage
+  static_assert(!DUP || NT == 1, "DUP is the one-query layout");
+  static_assert(TPW % KT == 0 && (KT == 2 || KT == 4), "KT tiles per batch");
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* s_inv = reinterpret_cast<float*>(smem_raw);
+  float* s_mul = s_inv + 64;
+  int* s_qsum = reinterpret_cast<int*>(s_mul + 64);
+  uint2* Btab = reinterpret_cast<uint2*>(smem_raw + 3 * 64 * 4 + 256);       // [NT][W][32]
+  uint32_t* sbits = reinterpret_cast<uint32_t*>(Btab + (size_t)NT * W * 32);  // [NS][SK * W]
+  float* snorm = reinterpret_cast<float*>(sbits + (size_t)NS * SK * W);     // [NS][SK]
+  uint64_t* full = reinterpret_cast<uint64_t*>(snorm + (size_t)NS * SK);
+  uint64_t* empty = full + NS;
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t cpg = (N + SK - 1) / SK;
+  const int64_t total = G * cpg;
+  const int64_t i0 = (int64_t)blockIdx.x * items_per_cta;
+  const int64_t i1 = min(total, i0 + items_per_cta);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kDecConsumers);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == kDecConsumers) {
+    if (lane == 0) {
+      int64_t g = i0 / cpg, c = i0 - (i0 / cpg) * cpg;
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      for (int64_t it = i0; it < i1; ++it, ++issued) {
+        if (!mbar_wait(&empty[s], ph ^ 1u)) { atomicOr(err, 1); break; }
+        const int64_t n0 = c * SK;
+        const int cnt = (int)(N - n0 < SK ? N - n0 : SK);
+        const float* nsrc = norms + g * N + n0;
+        const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
+        const uint32_t bbytes = (uint32_t)cnt * W * 4;
+        mbar_expect_tx(&full[s], bbytes + (nbulk ? (uint32_t)cnt * 4 : 0u));
+        bulk_g2s(sbits + (size_t)s * SK * W, bits + (g * N + n0) * W, bbytes, &full[s]);
+        if (nbulk) bulk_g2s(snorm + (size_t)s * SK, nsrc, (uint32_t)cnt * 4, &full[s]);
+        if (++c == cpg) { c = 0; ++g; }
+        if (++s == NS) { s = 0; ph ^= 1u; }
+      }
+      const int used = issued < NS ? (int)issued : NS;
+      for (int j = 0; j < used; ++j) {
+        int st = s - 1 - j;
+        uint32_t p = ph;
+        if (st < 0) { st += NS; p ^= 1u; }
+        if (!mbar_wait(&full[st], p)) atomicOr(err, 2);
+      }
+    }
+    return;
+  }
+
+  const int gq = lane >> 2, q = lane & 3, par = q & 1, half = q >> 1;
+  // stage bookkeeping kept incremental and 32-bit where it can be: chunk c of
+  // group g, with the norms and output pointers advanced by SK per stage
+  int64_t g = i0 / cpg;
+  int c = (int)(i0 - g * cpg);
+  const int cpg32 = (int)cpg;
+  const int last_cnt = (int)(N - (cpg - 1) * SK);
+  const bool groups_aligned = ((((uintptr_t)norms) & 15u) == 0) && (N % 4 == 0);
+  const float* nsrc = norms + g * N + (int64_t)c * SK;
+  float* gout = scores + g * (int64_t)J * N + (int64_t)c * SK;
+  int64_t cur_g = -1;
+  int s = 0;
+  uint32_t ph = 0;
+  uint2 breg[NT == 1 ? W : 1];
+  float mul[NT];
+  uint32_t qs[NT];
+  bool dead = false;  // a timed-out wait: keep the loop's barriers, skip the work
+  const int nitems = (int)(i1 - i0);
+  for (int item = 0; item < nitems; ++item) {
+    const int cnt = c == cpg32 - 1 ? last_cnt : SK;
+    if (g != cur_g) {
+      named_sync(1, kDecConsumers * 32);
+      build_tables_dig<W>(sq + g * (int64_t)J * (32 * W), J, NT, DUP, est_scale, s_inv, s_mul, s_qsum, Btab,
+                          kDecConsumers, 1);
+      if constexpr (NT == 1) {
+#pragma unroll
+        for (int mu = 0; mu < W; ++mu) breg[mu] = Btab[mu * 32 + lane];
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int jq = DUP ? 0 : 2 * nt + half;
+        mul[nt] = jq < J ? s_mul[jq] : 0.f;
+        qs[nt] = jq < J ? (uint32_t)s_qsum[jq] : 0u;
+      }
+      cur_g = g;
+    }
+    if (!dead && !__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { atomicOr(err, 4); dead = true; }
+    if (!dead) {
+      // the producer bulk-copied the norms exactly when they were 16-byte aligned
+      // and a multiple of 4; otherwise they are read from global memory
+      const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
+      const bool whole = groups_aligned && cnt == SK;
+      const uint32_t* sb = sbits + (size_t)s * SK * W;
+      const float* sn = snorm + (size_t)s * SK;
+#pragma unroll 1
+      for (int i = 0; i < TPW; i += KT) {
+        const int tile0 = warp + i * kDecConsumers;
+        if (tile0 * 16 >= cnt) break;
+        uint32_t w0[KT][W / 4], w1[KT][W / 4];
+#pragma unroll
+        for (int t = 0; t < KT; ++t) {
+          // rows past cnt (always < SK) read stale stage data; their results are never stored
+          const int r0 = (tile0 + t * kDecConsumers) * 16 + gq;
+#pragma unroll
+          for (int kk = 0; kk < W / 8; ++kk) {
+            const uint2 a = *reinterpret_cast<const uint2*>(sb + r0 * W + q * (W / 4) + 2 * kk);
+            const uint2 b = *reinterpret_cast<const uint2*>(sb + (r0 + 8) * W + q * (W / 4) + 2 * kk);
+            w0[t][2 * kk] = a.x; w0[t][2 * kk + 1] = a.y;
+            w1[t][2 * kk] = b.x; w1[t][2 * kk + 1] = b.y;
+          }
+        }
+        int acc[KT][NT][4];
+#pragma unroll
+        for (int p = 0; p < W / 8; ++p) {
+#pragma unroll
+          for (int sh = 0; sh < 8; ++sh) {
+            uint32_t x[KT][4];
+#pragma unroll
+            for (int t = 0; t < KT; ++t) {
+              x[t][0] = w0[t][2 * p] >> sh;
+              x[t][1] = w1[t][2 * p] >> sh;
+              x[t][2] = w0[t][2 * p + 1] >> sh;
+              x[t][3] = w1[t][2 * p + 1] >> sh;
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const uint2 bb = NT == 1 ? breg[(8 * p + sh) % (NT == 1 ? W : 1)]
+                                       : Btab[(nt * W + 8 * p + sh) * 32 + lane];
+#pragma unroll
+              for (int t = 0; t < KT; ++t) {
+                if (p == 0 && sh == 0) mma_u8s8_zc(acc[t][nt], x[t][0], x[t][1], x[t][2], x[t][3], bb.x, bb.y);
+                else mma_u8s8(acc[t][nt], x[t][0], x[t][1], x[t][2], x[t][3], bb.x, bb.y);
+              }
+            }
+          }
+        }
+        if (whole)
+          digit_epilogue<NT, DUP, KT, false>(acc, tile0, gq, par, half, cnt, nbulk, sn, nsrc, mul, qs, J, N, gout);
+        else
+          digit_epilogue<NT, DUP, KT, true>(acc, tile0, gq, par, half, cnt, nbulk, sn, nsrc, mul, qs, J, N, gout);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (++c == cpg32) {
+      c = 0;
+      ++g;
+      nsrc = norms + g * N;
+      gout = scores + g * (int64_t)J * N;
+    } else {
+      nsrc += SK;
+      gout += SK;
+    }
     if (++s == NS) { s = 0; ph ^= 1u; }
   }
 }
@@ -559,14 +720,14 @@ qjl_status launch_mma(const qjl_projection* P, const uint32_t* bits, const float
   return qjl_check_launch("scores_stream_kernel");
 }
 
-template <int W, bool CLS>
+template <int W>
 qjl_status launch_decode_fast(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t G,
                               int64_t N, const float* sq, int J, float* scores, cudaStream_t st) {
   const int NS = W == 8 ? 4 : 3;
   const size_t smem = 3 * 64 * 4 + (size_t)W * 32 * sizeof(uint2) + (size_t)NS * kDecStageKeys * (W + 1) * 4 +
                       (size_t)2 * NS * 8;
   static_assert(kDecTilesPerWarp % 4 == 0, "tiles are consumed in groups of 2 or 4");
-  auto kern = scores_decode_kernel<W, CLS>;
+  auto kern = scores_decode_kernel<W>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return qjl_check_launch("scores_decode_kernel smem attribute");
@@ -586,17 +747,55 @@ qjl_status launch_decode_fast(const qjl_projection* P, const uint32_t* bits, con
   return qjl_check_launch("scores_decode_kernel");
 }
 
+template <int W, int NT, bool DUP, int KT, int SKT>
+qjl_status launch_digit(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t G, int64_t N,
+                        const float* sq, int J, float* scores, cudaStream_t st) {
+  // ring depth: as many stages as keep two CTAs per SM within shared memory
+  const int NS = SKT * (W + 1) * 4 * 4 <= 80 * 1024 ? 4 : (SKT * (W + 1) * 4 * 3 <= 110 * 1024 ? 3 : 2);
+  const size_t smem = 3 * 64 * 4 + 256 + (size_t)NT * W * 32 * sizeof(uint2) + (size_t)NS * SKT * (W + 1) * 4 +
+                      (size_t)2 * NS * 8;
+  auto kern = scores_digit_kernel<W, NT, DUP, KT, SKT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+    return qjl_check_launch("scores_digit_kernel smem attribute");
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, smem) != cudaSuccess || per_sm < 1)
+    return qjl_check_launch("scores_digit_kernel occupancy");
+  int* err = qjl_error_flag(P->device);
+  if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  const int64_t total = G * ((N + SKT - 1) / SKT);
+  const int64_t slots = (int64_t)qjl_num_sms(P->device) * per_sm;
+  const int64_t grid = std::min<int64_t>(total, slots);
+  const int64_t ipc = (total + grid - 1) / grid;
+  const int64_t nblk = (total + ipc - 1) / ipc;
+  qjl_log_launch("scores_digit_kernel", nblk, kDecThreads, smem, per_sm);
+  kern<<<(unsigned)nblk, kDecThreads, smem, st>>>(bits, norms, sq, G, N, J, NS, P->est_scale, ipc, scores, err);
+  return qjl_check_launch("scores_digit_kernel");
+}
+
+// One or two queries per group: 1024-key stages; four tiles per batch at
+// m = 256, two at m = 512 (registers).
+template <int W>
+qjl_status launch_digit_w(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t G, int64_t N,
+                          const float* sq, int J, float* scores, cudaStream_t st) {
+  constexpr int KT = W == 8 ? 4 : 2;
+  return J == 1 ? launch_digit<W, 1, true, KT, 1024>(P, bits, norms, G, N, sq, J, scores, st)
+                : launch_digit<W, 1, false, KT, 1024>(P, bits, norms, G, N, sq, J, scores, st);
+}
+
 }  // namespace
 
 bool scores_mma_supported(int m) { return m == 256 || m == 512 || m == 1024; }
 
 qjl_status launch_scores(const qjl_projection* P, const uint32_t* bits, const float* norms,
                          int64_t G, int64_t N, const float* sq, int J, float* scores, cudaStream_t st) {
-  // J <= 4 at m = 256 or 512 takes the register-resident decode kernel. The
-  // tcgen05 variant (QJL_SCORES_KERNEL=tc) computes the same sums on the 5th-gen
-  // tensor cores, but at about 48 cycles per 128x8x32 MMA its A-operand reads
-  // (one byte per sign bit) cap it below the mma.sync path; it is kept for
-  // comparison. QJL_SCORES_KERNEL=stream selects the generic streaming kernel.
+  // At m = 256 or 512, one or two queries per group take the shift-window
+  // digit kernel and three or four the class kernel (half the MMAs of two
+  // digit column tiles). The tcgen05 variant (QJL_SCORES_KERNEL=tc) computes
+  // the same sums on the 5th-gen tensor cores, but at about 48 cycles per
+  // 128x8x32 MMA its A-operand reads (one byte per sign bit) cap it below the
+  // mma.sync path; it is kept for comparison. QJL_SCORES_KERNEL=stream selects
+  // the generic streaming kernel.
   static const int choice = [] {
     const char* v = getenv("QJL_SCORES_KERNEL");
     if (v && strcmp(v, "tc") == 0) return 1;
@@ -604,11 +803,12 @@ qjl_status launch_scores(const qjl_projection* P, const uint32_t* bits, const fl
     return 0;
   }();
   if (choice == 1 && scores_tc_supported(P->m, J)) return launch_scores_tc(P, bits, norms, G, N, sq, J, scores, st);
+  if (choice == 0 && J <= 2 && (P->m == 256 || P->m == 512))
+    return P->m == 256 ? launch_digit_w<8>(P, bits, norms, G, N, sq, J, scores, st)
+                       : launch_digit_w<16>(P, bits, norms, G, N, sq, J, scores, st);
   if (choice == 0 && J <= 4 && (P->m == 256 || P->m == 512))
-    return P->m == 256 ? (J == 1 ? launch_decode_fast<8, true>(P, bits, norms, G, N, sq, J, scores, st)
-                                 : launch_decode_fast<8, false>(P, bits, norms, G, N, sq, J, scores, st))
-                       : (J == 1 ? launch_decode_fast<16, true>(P, bits, norms, G, N, sq, J, scores, st)
-                                 : launch_decode_fast<16, false>(P, bits, norms, G, N, sq, J, scores, st));
+    return P->m == 256 ? launch_decode_fast<8>(P, bits, norms, G, N, sq, J, scores, st)
+                       : launch_decode_fast<16>(P, bits, norms, G, N, sq, J, scores, st);
   const int NTR = J > 4 ? 2 : 1;
   switch (scores_mma_supported(P->m) ? P->m : 0) {
     case 256: return NTR == 1 ? launch_mma<8, 1>(P, bits, norms, G, N, sq, J, scores, st)

@@ -1,15 +1,23 @@
 // Sign-bit dot products on the s8 tensor-core path (mma.sync m16n8k32).
 //
-// Shared by the score kernel and the fused decode kernel. The scheme is
-// described at the top of scores.cu: 16-bit fixed-point Sq split into int8
-// hi/lo columns, and sign bits fed as u8 A fragments of value 2^J, one AND
-// per 4 bits. A 16-key tile needs W MMAs per column tile of 4 queries.
+// Shared by the score kernel and the fused decode kernel. Two schemes, both
+// described at the top of scores.cu: weight classes (16-bit fixed-point Sq
+// split into int8 hi/lo columns, sign bits fed as u8 A fragments of value
+// 4^c, one AND per 4 bits; W MMAs per 16-key tile per column tile of four
+// queries) and shift windows (unmasked shifted words as A, B as four int8
+// digits of a residue modulo 2^32; W MMAs per tile per two queries).
 #pragma once
 
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace qjl_sign {
+
+// Named barrier `id` over `threads` threads, or __syncthreads for id 0.
+__device__ __forceinline__ void named_barrier_or_sync(int id, int threads) {
+  if (id) asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+  else __syncthreads();
+}
 
 constexpr int kQmax = 32639;  // 127 * 256 + 127: both int8 halves stay in range
 constexpr int kQmaxE = 32638; // the even grid of the single-query tables (127 * 256 + 126)
@@ -209,6 +217,109 @@ __device__ __forceinline__ void tile_sums(const uint32_t (&w0)[W / 4], const uin
     hi[r] = ((acc[0][2 * r] * 4 + acc[1][2 * r]) * 4 + acc[2][2 * r]) * 4 + acc[3][2 * r];
     lo[r] = ((acc[0][2 * r + 1] * 4 + acc[1][2 * r + 1]) * 4 + acc[2][2 * r + 1]) * 4 + acc[3][2 * r + 1];
   }
+}
+
+
+// ---------------------------------------------------------------------------
+// Shift-window ("digit") sign sums: no masking of the sign words.
+//
+// The A operand of the u8 MMA is the bit word shifted right by s, s = 0..7,
+// unmasked: byte e of (w >> s) is the 8-bit window sum_t 2^t b_{8e+s+t}. Over
+// the eight shifts every bit i of the word is the lowest bit of exactly one
+// window (the one starting at i), so the windows' weights form a unit
+// lower-triangular system. Giving window i the B value
+//   B_i = sum_k 256^k (Q_{i-8k} - 2 Q_{i-8k-1})   (mod 2^32, Q_{<0} = 0)
+// makes sum_windows A B = sum_i b_i Q_i (mod 2^32): the generating function of
+// the window weights is (1 - 256 x^8) / (1 - 2x), and B is Q times its inverse.
+// B is a 32-bit residue, carried as four signed base-256 digits in four B
+// columns; the int32 column sums are combined as D0 + 2^8 D1 + 2^16 D2 + 2^24
+// D3 in wrapping 32-bit arithmetic. As long as sum_i |Q_i| < 2^31 the residue
+// is the exact sum, so Q can take 31 - log2(m) bits (2^23 - 1 at m = 256):
+// the rounding of Sq to that grid is the only error.
+//
+// Per MMA the eight columns hold the digits of two queries (columns 4c'..4c'+3
+// for query c' of the column tile). A thread (g, q) of the C fragment holds
+// digits (2q, 2q+1) of query q >> 1 for key rows g and g + 8.
+// ---------------------------------------------------------------------------
+
+__host__ __device__ constexpr int qmax_dig(int m) { return (int)((2147483647u / (unsigned)m)); }
+
+// digit `dg` (0..3) of the balanced base-256 representation of B (mod 2^32), as a byte
+__device__ __forceinline__ uint32_t dig_byte(uint32_t B, int dg) {
+  for (int c = 0; c < dg; ++c) {
+    const int d = (int)(int8_t)(B & 0xFFu);
+    B = (B - (uint32_t)d) >> 8;
+  }
+  return B & 0xFFu;
+}
+
+__device__ __forceinline__ int quant_dig(float v, float inv, int Qm) {
+  const float q = rintf(v * inv);
+  return (int)fminf(fmaxf(q, (float)-Qm), (float)Qm);
+}
+
+// Quantises the J query rows of group `sqg` to the digit grid (s_inv, s_mul,
+// s_qsum) and fills the B fragments:
+// Btab[(nt * W + mu) * 32 + lane] for column tile nt and MMA mu = 8 p + s.
+// With dup, J must be 1 and the one query's digits fill both column halves.
+template <int W>
+__device__ void build_tables_dig(const float* __restrict__ sqg, int J, int NT, bool dup, float est_scale,
+                                 float* s_inv, float* s_mul, int* s_qsum, uint2* Btab, int nwarps, int bar_id) {
+  constexpr int m = 32 * W;
+  constexpr int Qm = qmax_dig(m);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nthreads = 32 * nwarps;
+  for (int j = warp; j < J; j += nwarps) {
+    const float* row = sqg + (int64_t)j * m;
+    float mx = 0.f;
+    for (int i = lane; i < m; i += 32) mx = fmaxf(mx, fabsf(row[i]));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float inv = mx > 0.f ? (float)Qm / mx : 0.f;
+    int qs = 0;
+    for (int i = lane; i < m; i += 32) qs += quant_dig(row[i], inv, Qm);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+    if (lane == 0) {
+      s_inv[j] = inv;
+      s_mul[j] = est_scale * (mx > 0.f ? mx / (float)Qm : 0.f);
+      s_qsum[j] = qs;
+    }
+  }
+  named_barrier_or_sync(bar_id, nthreads);
+  const int entries = NT * W * 32;
+  for (int idx = threadIdx.x; idx < entries; idx += nthreads) {
+    const int ln = idx & 31;
+    const int mu = (idx >> 5) % W;
+    const int nt = (idx >> 5) / W;
+    const int n = ln >> 2, qq = ln & 3;
+    const int jq = dup ? 0 : nt * 2 + (n >> 2);
+    const int dg = n & 3;
+    const int p = mu >> 3, s = mu & 7;
+    uint32_t b[2] = {0u, 0u};
+    if (jq < J) {
+      const float inv = s_inv[jq];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const float* Sw = sqg + (int64_t)jq * m + 32 * (qq * (W / 4) + 2 * p + r);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 8 * e + s;
+          uint32_t B = 0u;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int t = i - 8 * k;
+            if (t < 0) break;
+            const int v = quant_dig(Sw[t], inv, Qm) - (t > 0 ? 2 * quant_dig(Sw[t - 1], inv, Qm) : 0);
+            B += (uint32_t)v << (8 * k);
+          }
+          b[r] |= dig_byte(B, dg) << (8 * e);
+        }
+      }
+    }
+    Btab[idx] = make_uint2(b[0], b[1]);
+  }
+  named_barrier_or_sync(bar_id, nthreads);
 }
 
 }  // namespace qjl_sign

@@ -55,7 +55,13 @@ def test_scores_and_projection_kernels(cuda_ok):
     norms = torch.ones((4, 1000), device="cuda")
     q = wl.normal((4, 128), 3, "cuda")
     names = _kernels(lambda: qjl.scores(P, bits, norms, qjl.project_queries(P, q).view(4, 1, 256)))
-    assert _has(names, "scores_decode_kernel") and _has(names, "project_dense_kernel"), names
+    # one or two queries per group: the shift-window digit kernel
+    assert _has(names, "scores_digit_kernel") and _has(names, "project_dense_kernel"), names
+    sq2 = torch.ones((4, 2, 256), device="cuda")
+    assert _has(_kernels(lambda: qjl.scores(P, bits, norms, sq2)), "scores_digit_kernel")
+    # three or four: the weight-class kernel
+    sq4 = torch.ones((4, 4, 256), device="cuda")
+    assert _has(_kernels(lambda: qjl.scores(P, bits, norms, sq4)), "scores_decode_kernel")
     # more than 4 queries per group take the streaming mma.sync kernel
     sq8 = torch.ones((4, 8, 256), device="cuda")
     assert _has(_kernels(lambda: qjl.scores(P, bits, norms, sq8)), "scores_stream_kernel")

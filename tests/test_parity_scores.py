@@ -1,4 +1,4 @@
-"""Estimator kernel vs the oracle, fed the oracle's bits and norms.
+"""Estimator kernels vs the oracle, fed the oracle's bits and norms.
 
 Tolerance: |gpu - oracle| <= 1e-3 * c * alpha * ||k|| * ||Sq||_1 per score.
 Covers the tensor-core kernel (m = 256, 512, 1024) and the SIMT kernel for
@@ -40,7 +40,11 @@ def _case(kind, d, m, G, J, N, seed=0):
 @pytest.mark.parametrize("m,G,J,N", [(256, 3, 1, 1000), (256, 1, 4, 4096), (256, 2, 16, 333), (512, 2, 4, 2049),
                                      (512, 1, 5, 100), (1024, 1, 64, 300), (1024, 2, 1, 1), (256, 4, 3, 17),
                                      (256, 1, 64, 200), (256, 50, 1, 100), (256, 37, 2, 300), (512, 20, 4, 129),
-                                     (512, 9, 3, 1000), (256, 300, 1, 7)])
+                                     (512, 9, 3, 1000), (256, 300, 1, 7),
+                                     # shift-window kernel: whole 1024-key stages, ragged tails, unaligned
+                                     # norm rows (N % 4 != 0), N = 1, m = 512 with one and two queries
+                                     (256, 2, 1, 3072), (256, 5, 2, 1025), (256, 3, 1, 1), (512, 3, 1, 2500),
+                                     (512, 2, 2, 1030), (256, 7, 1, 2051)])
 def test_scores_tensor_core(cuda_ok, m, G, J, N):
     _case("dense", 128, m, G, J, N)
 
