@@ -294,7 +294,7 @@ def build_workload(name, dev, qjl, wl, torch):
                   2 * D + M // 8 + 4, 2 * D * M, "dense_tc_kernel", "dense_tc.cu"),
             Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * M),
             Stage("scores", lambda: qjl.scores(P, bits.view(G, N, M // 32), norms.view(G, N), sq.view(G, 1, M), out=out),
-                  G * N, M // 8 + 4 + 4, 0, "scores_decode_kernel", "scores.cu"),
+                  G * N, M // 8 + 4 + 4, 0, "scores_digit_kernel", "scores.cu"),
         ]
         W.update(units=G * N, unit="keys/s", inputs=[keys, q], outputs=[out], dtype="bf16",
                  desc="%s: B=%d, heads=%d, N=%d, d=%d, m=%d dense bf16 S; quantize all keys, project 1 query/head, "

@@ -527,7 +527,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
 
   if (warp == kDecConsumers) {
     if (lane == 0) {
-      int64_t g = i0 / cpg, c = i0 - (i0 / cpg) * cpg;
+      // items newest first (see the consumer loop)
+      int64_t g = (i1 - 1) / cpg, c = (i1 - 1) - ((i1 - 1) / cpg) * cpg;
       int s = 0;
       uint32_t ph = 0;
       int64_t issued = 0;
@@ -541,7 +542,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
         mbar_expect_tx(&full[s], bbytes + (nbulk ? (uint32_t)cnt * 4 : 0u));
         bulk_g2s(sbits + (size_t)s * SK * W, bits + (g * N + n0) * W, bbytes, &full[s]);
         if (nbulk) bulk_g2s(snorm + (size_t)s * SK, nsrc, (uint32_t)cnt * 4, &full[s]);
-        if (++c == cpg) { c = 0; ++g; }
+        if (c == 0) { c = cpg - 1; --g; } else { --c; }
         if (++s == NS) { s = 0; ph ^= 1u; }
       }
       const int used = issued < NS ? (int)issued : NS;
@@ -556,10 +557,13 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
   }
 
   const int gq = lane >> 2, q = lane & 3, par = q & 1, half = q >> 1;
-  // stage bookkeeping kept incremental and 32-bit where it can be: chunk c of
-  // group g, with the norms and output pointers advanced by SK per stage
-  int64_t g = i0 / cpg;
-  int c = (int)(i0 - g * cpg);
+  // Each CTA walks its items newest first. When the keys were sketched just
+  // before (a whole-cache quantize, then scores), the tail of the bits array
+  // is still in L2, and reading it first takes it before the next reads
+  // evict it. Stage bookkeeping is incremental and 32-bit where it can be:
+  // chunk c of group g, with the norms and output pointers stepped per stage.
+  int64_t g = (i1 - 1) / cpg;
+  int c = (int)((i1 - 1) - g * cpg);
   const int cpg32 = (int)cpg;
   const int last_cnt = (int)(N - (cpg - 1) * SK);
   const bool groups_aligned = ((((uintptr_t)norms) & 15u) == 0) && (N % 4 == 0);
@@ -649,14 +653,15 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-    if (++c == cpg32) {
-      c = 0;
-      ++g;
-      nsrc = norms + g * N;
-      gout = scores + g * (int64_t)J * N;
+    if (c == 0) {
+      c = cpg32 - 1;
+      --g;
+      nsrc = norms + g * N + (int64_t)c * SK;
+      gout = scores + g * (int64_t)J * N + (int64_t)c * SK;
     } else {
-      nsrc += SK;
-      gout += SK;
+      --c;
+      nsrc -= SK;
+      gout -= SK;
     }
     if (++s == NS) { s = 0; ph ^= 1u; }
   }
