@@ -22,7 +22,9 @@ import torch
 from ._lib import Options, lib
 
 __all__ = ["Projection", "QJLError", "quantize_keys", "project_queries", "scores",
-           "quantize_values_2bit", "decode_attention", "decode_workspace_bytes", "lib", "KINDS"]
+           "quantize_values_2bit", "decode_attention", "decode_workspace_bytes", "PagedCache", "append_keys",
+           "append_values_2bit", "scores_paged", "decode_attention_paged", "decode_paged_workspace_bytes", "lib",
+           "KINDS"]
 
 KINDS = {"dense": 0, "dfqjl": 1, "pfqjl": 2}
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
@@ -175,4 +177,75 @@ def decode_attention(proj, bits, norms, codes, scale, zero, sq, softmax_scale, o
                                       G, N, _ptr(sq), J, float(softmax_scale), _ptr(out), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(stream)),
            "qjl_decode_attention")
+    return out
+
+
+class PagedCache:
+    """Caller-side description of a paged cache (pools, block table, lengths), all CUDA tensors.
+
+    bits [P*T, m/32] int32, norms [P*T] fp32, codes [P*T, d/16] int32, scale/zero [P*T, d/32] fp16,
+    block_table [G, max_pages] int32, seq_lens [G] int32; T = page_tokens, P = num_pages.
+    """
+
+    def __init__(self, page_tokens, block_table, seq_lens, bits, norms, codes=None, scale=None, zero=None):
+        self.page_tokens = int(page_tokens)
+        self.block_table, self.seq_lens = block_table, seq_lens
+        self.bits, self.norms, self.codes, self.scale, self.zero = bits, norms, codes, scale, zero
+        self.num_pages = norms.shape[0] // self.page_tokens
+        self.groups, self.max_pages = block_table.shape
+
+    def _table(self):
+        return (_ptr(self.block_table), int(self.max_pages), self.page_tokens, int(self.num_pages))
+
+
+def append_keys(proj, cache, keys, positions, stream=None):
+    """Sketch keys [G, d] into the cache at positions [G] (int32) of each group."""
+    _cuda(keys, "keys")
+    G = keys.shape[0]
+    _check(lib().qjl_append_keys(proj.handle, _ptr(keys), _DTYPES[keys.dtype], G, keys.stride(0), _ptr(positions),
+                                 *cache._table(), _ptr(cache.bits), _ptr(cache.norms), _stream(stream)),
+           "qjl_append_keys")
+
+
+def append_values_2bit(cache, v, positions, stream=None):
+    """2-bit values v [G, d] into the cache at positions [G] (int32) of each group."""
+    _cuda(v, "v")
+    G, d = v.shape
+    _check(lib().qjl_append_values_2bit(_ptr(v), _DTYPES[v.dtype], G, d, _ptr(positions), *cache._table(),
+                                        _ptr(cache.codes), _ptr(cache.scale), _ptr(cache.zero), _stream(stream)),
+           "qjl_append_values_2bit")
+
+
+def scores_paged(proj, cache, sq, max_len, out=None, stream=None):
+    """sq [G, J, m] -> estimates [G, J, max_len] over each group's seq_lens[g] tokens (the rest untouched)."""
+    _cuda(sq, "sq")
+    G, J = sq.shape[0], sq.shape[1]
+    if out is None:
+        out = torch.zeros((G, J, max_len), dtype=torch.float32, device=sq.device)
+    _check(lib().qjl_scores_paged(proj.handle, _ptr(cache.bits), _ptr(cache.norms), *cache._table(),
+                                  _ptr(cache.seq_lens), G, int(max_len), _ptr(sq), J, _ptr(out), _stream(stream)),
+           "qjl_scores_paged")
+    return out
+
+
+def decode_paged_workspace_bytes(groups, max_len, d):
+    return int(lib().qjl_decode_paged_workspace_bytes(groups, max_len, d))
+
+
+def decode_attention_paged(proj, cache, sq, max_len, softmax_scale, out=None, workspace=None, stream=None):
+    """sq [G, m] (one query per group) -> softmax(est * softmax_scale) . V_hat [G, d] over the paged cache."""
+    _cuda(sq, "sq")
+    G = sq.shape[0]
+    d = proj.d
+    if out is None:
+        out = torch.empty((G, d), dtype=torch.float32, device=sq.device)
+    need = decode_paged_workspace_bytes(G, max_len, d)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=sq.device)
+    _check(lib().qjl_decode_attention_paged(proj.handle, _ptr(cache.bits), _ptr(cache.norms), _ptr(cache.codes),
+                                            _ptr(cache.scale), _ptr(cache.zero), *cache._table(),
+                                            _ptr(cache.seq_lens), G, int(max_len), _ptr(sq), float(softmax_scale),
+                                            _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                            _stream(stream)),
+           "qjl_decode_attention_paged")
     return out

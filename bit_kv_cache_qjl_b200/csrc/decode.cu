@@ -337,11 +337,16 @@ __device__ __forceinline__ bool bulk_ok(const void* src, uint32_t bytes) {
   return (((uintptr_t)src & 15u) == 0) && (bytes % 16u == 0);
 }
 
-template <int W, int CPL>
+// PAGED reads group g's tokens t < seq_lens[g] through the block table
+// (PagedRead); N is then the bound max_len. Every array is bulk-copied per page
+// segment, rounded up to 4 tokens (never past the page: pages hold a multiple
+// of 16 tokens, and segments start 16-token aligned).
+template <int W, int CPL, bool PAGED>
 __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
     const uint32_t* __restrict__ bits, const float* __restrict__ norms, const uint32_t* __restrict__ codes,
     const uint16_t* __restrict__ scale, const uint16_t* __restrict__ zero, const float* __restrict__ sq, int64_t G,
-    int64_t N, int NS, float est_scale, float logit_scale, float* __restrict__ ws, int* __restrict__ err) {
+    int64_t N, int NS, float est_scale, float logit_scale, float* __restrict__ ws, int* __restrict__ err,
+    PagedRead pr) {
   using namespace qjl_sync;
   constexpr int d = 32 * CPL;
   constexpr int CW = d / 16;  // code words per token
@@ -381,23 +386,52 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
       bool stop = false;
       for (int64_t gi = g_first; gi <= g_last && !stop; ++gi) {
         const int64_t t0 = 16 * (max(tb, gi * plan.ntg) - gi * plan.ntg);
-        const int64_t t1 = min(N, 16 * (min(te, (gi + 1) * plan.ntg) - gi * plan.ntg));
-        const int64_t nst = (t1 - t0 + kDsStage - 1) / kDsStage;
+        int64_t t1 = min(N, 16 * (min(te, (gi + 1) * plan.ntg) - gi * plan.ntg));
+        if (PAGED) t1 = min(t1, min(max((int64_t)__ldg(pr.seq_lens + gi), (int64_t)0), N));
+        const int64_t nst = t1 > t0 ? (t1 - t0 + kDsStage - 1) / kDsStage : 0;
         for (int64_t k = 0; k < nst; ++k, ++issued) {
           if (!mbar_wait(&empty[s], ph ^ 1u)) { atomicOr(err, 1); stop = true; break; }
           const int64_t n0 = t0 + k * kDsStage;
           const uint32_t cnt = (uint32_t)(t1 - n0 < kDsStage ? t1 - n0 : kDsStage);
-          const int64_t row = gi * N + n0;
           unsigned char* st = ring + (size_t)s * L.bytes;
-          const void* src[5] = {bits + row * W, norms + row, codes + row * CW, scale + row * GW, zero + row * GW};
-          const uint32_t nb[5] = {cnt * W * 4, cnt * 4, cnt * CW * 4, cnt * GW * 2, cnt * GW * 2};
           const uint32_t off[5] = {L.bits, L.norms, L.codes, L.scale, L.zero};
-          uint32_t tx = 0;
-          for (int a = 0; a < 5; ++a)
-            if (bulk_ok(src[a], nb[a])) tx += nb[a];
-          mbar_expect_tx(&full[s], tx);
-          for (int a = 0; a < 5; ++a)
-            if (bulk_ok(src[a], nb[a])) bulk_g2s(st + off[a], src[a], nb[a], &full[s]);
+          const uint32_t per_tok[5] = {W * 4, 4, CW * 4, GW * 2, GW * 2};
+          if constexpr (PAGED) {
+            const int T = pr.page_tokens;
+            uint32_t tx = 0;
+            for (int pass = 0; pass < 2; ++pass) {
+              if (pass == 1) mbar_expect_tx(&full[s], tx);
+              for (int64_t lo = n0; lo < n0 + cnt;) {
+                const int64_t pi = lo / T;
+                const int64_t hi = min(n0 + (int64_t)cnt, (pi + 1) * T);
+                const uint32_t len4 = (uint32_t)((hi - lo + 3) & ~3);
+                const int pg = pi < pr.max_pages ? __ldg(pr.table + gi * (int64_t)pr.max_pages + pi) : -1;
+                if (pg >= 0 && (int64_t)pg < pr.num_pages) {
+                  const int64_t prow = (int64_t)pg * T + (lo - pi * T);
+                  const void* src[5] = {bits + prow * W, norms + prow, codes + prow * CW, scale + prow * GW,
+                                        zero + prow * GW};
+                  for (int a = 0; a < 5; ++a) {
+                    if (pass == 0) tx += len4 * per_tok[a];
+                    else bulk_g2s(st + off[a] + (lo - n0) * per_tok[a], src[a], len4 * per_tok[a], &full[s]);
+                  }
+                } else if (pass == 0) {
+                  atomicOr(err, 8);  // a bad page id: its tokens keep stale stage data
+                }
+                lo = hi;
+              }
+            }
+          } else {
+            const int64_t row = gi * N + n0;
+            const void* src[5] = {bits + row * W, norms + row, codes + row * CW, scale + row * GW, zero + row * GW};
+            uint32_t nb[5];
+            for (int a = 0; a < 5; ++a) nb[a] = cnt * per_tok[a];
+            uint32_t tx = 0;
+            for (int a = 0; a < 5; ++a)
+              if (bulk_ok(src[a], nb[a])) tx += nb[a];
+            mbar_expect_tx(&full[s], tx);
+            for (int a = 0; a < 5; ++a)
+              if (bulk_ok(src[a], nb[a])) bulk_g2s(st + off[a], src[a], nb[a], &full[s]);
+          }
           if (++s == NS) { s = 0; ph ^= 1u; }
         }
       }
@@ -419,8 +453,9 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
   bool dead = false;  // a timed-out wait: keep the loop's barriers, skip the work
   for (int64_t gi = g_first; gi <= g_last; ++gi) {
   const int64_t t0 = 16 * (max(tb, gi * plan.ntg) - gi * plan.ntg);
-  const int64_t t1 = min(N, 16 * (min(te, (gi + 1) * plan.ntg) - gi * plan.ntg));
-  const int64_t nst = (t1 - t0 + kDsStage - 1) / kDsStage;
+  int64_t t1 = min(N, 16 * (min(te, (gi + 1) * plan.ntg) - gi * plan.ntg));
+  if (PAGED) t1 = min(t1, min(max((int64_t)__ldg(pr.seq_lens + gi), (int64_t)0), N));
+  const int64_t nst = t1 > t0 ? (t1 - t0 + kDsStage - 1) / kDsStage : 0;
   build_tables_cls<W>(sq + gi * (int64_t)(32 * W), est_scale, s_inv, s_mul, s_qsum, Btab, kDsConsumers, 1);
   uint2 breg[W];
 #pragma unroll
@@ -448,10 +483,10 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
     if (!dead) {
     const unsigned char* st = ring + (size_t)s * L.bytes;
     const uint32_t* sb = reinterpret_cast<const uint32_t*>(st + L.bits);
-    const bool nb_norm = bulk_ok(norms + row0, (uint32_t)cnt * 4);
-    const bool nb_codes = bulk_ok(codes + row0 * CW, (uint32_t)cnt * CW * 4);
-    const bool nb_scale = bulk_ok(scale + row0 * GW, (uint32_t)cnt * GW * 2);
-    const bool nb_zero = bulk_ok(zero + row0 * GW, (uint32_t)cnt * GW * 2);
+    const bool nb_norm = PAGED || bulk_ok(norms + row0, (uint32_t)cnt * 4);
+    const bool nb_codes = PAGED || bulk_ok(codes + row0 * CW, (uint32_t)cnt * CW * 4);
+    const bool nb_scale = PAGED || bulk_ok(scale + row0 * GW, (uint32_t)cnt * GW * 2);
+    const bool nb_zero = PAGED || bulk_ok(zero + row0 * GW, (uint32_t)cnt * GW * 2);
     const float* snorm = reinterpret_cast<const float*>(st + L.norms);
     const uint32_t* scodes = reinterpret_cast<const uint32_t*>(st + L.codes);
     const uint16_t* sscale = reinterpret_cast<const uint16_t*>(st + L.scale);
@@ -618,7 +653,7 @@ __global__ void __launch_bounds__(128) decode_combine_stream_kernel(const float*
     const float* e = entry(c);
     Lsum += (e[0] == -INFINITY) ? 0.f : e[1] * exp2f(e[0] - M);
   }
-  const float invL = 1.f / Lsum;
+  const float invL = Lsum > 0.f ? 1.f / Lsum : 0.f;  // a group with no tokens (paged, seq_lens 0) gives 0
   for (int ch = threadIdx.x; ch < d; ch += blockDim.x) {
     float v = 0.f;
     for (int64_t c = c_lo; c <= c_hi; ++c) {
@@ -679,10 +714,11 @@ qjl_status launch_wc(const qjl_projection* P, const uint32_t* bits, const float*
   return qjl_check_launch("decode_combine_kernel");
 }
 
-template <int W, int CPL>
+template <int W, int CPL, bool PAGED = false>
 qjl_status launch_stream(const qjl_projection* P, const uint32_t* bits, const float* norms, const uint32_t* codes,
                          const uint16_t* scale, const uint16_t* zero, int64_t G, int64_t N, const float* sq,
-                         float softmax_scale, float* out, float* ws, cudaStream_t st) {
+                         float softmax_scale, float* out, float* ws, cudaStream_t st,
+                         const PagedRead& pr = PagedRead()) {
   constexpr int d = 32 * CPL;
   const DsLayout L = ds_layout(W, d);
   int NS = 4;  // one CTA per SM: about 168 KB in flight at d = 128, m = 256
@@ -691,7 +727,7 @@ qjl_status launch_stream(const qjl_projection* P, const uint32_t* bits, const fl
     --NS;
   const size_t smem = 3 * 64 * 4 + (size_t)W * 32 * sizeof(uint2) + (size_t)kDsConsumers * (d + 2) * 4 +
                       (size_t)NS * L.bytes + (size_t)2 * NS * 8;
-  auto kern = decode_stream_kernel<W, CPL>;
+  auto kern = decode_stream_kernel<W, CPL, PAGED>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return qjl_check_launch("decode_stream_kernel smem attribute");
@@ -700,7 +736,7 @@ qjl_status launch_stream(const qjl_projection* P, const uint32_t* bits, const fl
   const StreamPlan plan = stream_plan(G, N);
   qjl_log_launch("decode_stream_kernel", plan.ncta, kDsThreads, smem, 1);
   kern<<<(unsigned)plan.ncta, kDsThreads, smem, st>>>(bits, norms, codes, scale, zero, sq, G, N, NS, P->est_scale,
-                                                      softmax_scale, ws, err);
+                                                      softmax_scale, ws, err, pr);
   qjl_status s = qjl_check_launch("decode_stream_kernel");
   if (s != QJL_OK) return s;
   decode_combine_stream_kernel<<<(unsigned)G, 128, 0, st>>>(ws, G, N, d, out);
@@ -754,4 +790,18 @@ qjl_status launch_decode(const qjl_projection* P, const uint32_t* bits, const fl
     case 1024: return launch_w<32>(P, bits, norms, codes, scale, zero, G, N, sq, J, softmax_scale, out, w, st);
   }
   return qjl_set_error(QJL_ERR_UNSUPPORTED, "decode attention supports m in {256, 512, 1024}");
+}
+
+size_t decode_paged_workspace_bytes(int64_t groups, int64_t max_len, int d) {
+  return decode_workspace_bytes(groups, 1, max_len, d);
+}
+
+qjl_status launch_decode_paged(const qjl_projection* P, const uint32_t* bits_pool, const float* norms_pool,
+                               const uint32_t* codes_pool, const uint16_t* scale_pool, const uint16_t* zero_pool,
+                               const PagedRead& pr, int64_t G, int64_t max_len, const float* sq,
+                               float softmax_scale, float* out, void* ws, cudaStream_t st) {
+  if (P->m != 256 || P->d != 128)
+    return qjl_set_error(QJL_ERR_UNSUPPORTED, "paged decode attention supports d = 128 and m = 256");
+  return launch_stream<8, 4, true>(P, bits_pool, norms_pool, codes_pool, scale_pool, zero_pool, G, max_len, sq,
+                                   softmax_scale, out, reinterpret_cast<float*>(ws), st, pr);
 }

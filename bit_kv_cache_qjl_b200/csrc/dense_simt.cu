@@ -32,13 +32,20 @@ __global__ void __launch_bounds__(256) dense_simt_kernel(const void* __restrict_
                                                          const float* __restrict__ St,
                                                          uint32_t* __restrict__ bits,
                                                          float* __restrict__ norms,
-                                                         float* __restrict__ proj_out) {
+                                                         float* __restrict__ proj_out, PageMap pm,
+                                                         int* __restrict__ err) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int W = m >> 5;
   for (int64_t row = warp; row < rows; row += nwarps) {
     const int64_t xoff = row * ld;
+    // output row: the same row, or the key's page slot when appending to a paged cache
+    const int64_t orow = pm.slot(row);
+    if (orow < 0) {
+      if (lane == 0 && err) atomicOr(err, 8);
+      continue;
+    }
     float sumsq = 0.f;
     for (int c0 = 0; c0 < m; c0 += 32 * kRowsPerPass) {
       float acc[kRowsPerPass];
@@ -63,15 +70,15 @@ __global__ void __launch_bounds__(256) dense_simt_kernel(const void* __restrict_
         if (c >= m) break;
         if (bits) {
           const uint32_t word = __ballot_sync(0xffffffffu, acc[r] >= 0.f);
-          if (lane == 0) bits[row * W + (c >> 5)] = word;
+          if (lane == 0) bits[orow * W + (c >> 5)] = word;
         }
-        if (proj_out) proj_out[row * (int64_t)m + c + lane] = acc[r];
+        if (proj_out) proj_out[orow * (int64_t)m + c + lane] = acc[r];
       }
     }
     if (norms) {
 #pragma unroll
       for (int o = 16; o; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
-      if (lane == 0) norms[row] = sqrtf(sumsq);
+      if (lane == 0) norms[orow] = sqrtf(sumsq);
     }
   }
 }
@@ -116,15 +123,17 @@ qjl_status launch_project_dense(const qjl_projection* P, const float* q, int64_t
 }
 
 qjl_status launch_dense_simt(const qjl_projection* P, const void* x, int dtype, int64_t n, int64_t ld,
-                             uint32_t* bits, float* norms, float* proj_out, cudaStream_t st) {
+                             uint32_t* bits, float* norms, float* proj_out, cudaStream_t st, const PageMap& pm) {
+  if (n <= 0) return QJL_OK;
+  int* err = pm.pos ? qjl_error_flag(P->device) : nullptr;
   const int threads = 256;
   const int64_t want = (n + 7) / 8;
   const int blocks = (int)std::min<int64_t>(want, (int64_t)qjl_num_sms(P->device) * 16);
   if (dtype == QJL_F32)
     dense_simt_kernel<QJL_F32><<<blocks, threads, 0, st>>>(x, n, ld, P->d, P->m, P->St_f32, bits,
-                                                           norms, proj_out);
+                                                           norms, proj_out, pm, err);
   else
     dense_simt_kernel<QJL_BF16><<<blocks, threads, 0, st>>>(x, n, ld, P->d, P->m, P->St_f32, bits,
-                                                            norms, proj_out);
+                                                            norms, proj_out, pm, err);
   return qjl_check_launch("dense_simt_kernel");
 }

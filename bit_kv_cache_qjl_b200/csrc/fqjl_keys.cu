@@ -196,6 +196,7 @@ struct KeysArgs {
   float* norms;
   int W;                      // words per key row of bits
   int* err;
+  PageMap pm;                 // appends to a paged cache: row -> pool row, which also seeds the dither
 };
 
 template <int E, int L, int ES>
@@ -300,7 +301,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
 
   for (uint32_t phase = 0; q < nbatch; q += stride, phase ^= 1u) {
     const int64_t row = q * K + kp;
-    const bool valid = row < a.n;
+    // the output row (a page slot when appending to a paged cache) and the dither's token index
+    const int64_t orow = row < a.n ? a.pm.slot(row) : -1;
+    if (row < a.n && orow < 0) atomicOr(a.err, 8);
+    const bool valid = orow >= 0;
     if (!__all_sync(0xffffffffu, mbar_wait(bar, phase))) {
       // the batch never landed (the whole warp agrees): flag it, give the copy one more
       // bounded wait, and stop
@@ -308,7 +312,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
       mbar_wait(bar, phase);
       return;
     }
-    const uint64_t tok = a.first_token + (uint64_t)row;
+    const uint64_t tok = a.pm.pos ? (uint64_t)orow : a.first_token + (uint64_t)row;
     float norm = 0.f;
 
     for (int bl = 0; bl < nbl; ++bl) {
@@ -408,7 +412,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
       }
       // sign bits: element s*E + r is bit r % 32 of word (b*d + s*E + r) / 32 of the key's row
       if (valid) {
-        uint32_t* out = a.bits + row * (int64_t)a.W + ((b * d + s * E) >> 5);
+        uint32_t* out = a.bits + orow * (int64_t)a.W + ((b * d + s * E) >> 5);
 #pragma unroll
         for (int w = 0; w < E / 32; ++w) {
           uint32_t acc = 0;
@@ -422,7 +426,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
         }
       }
     }
-    if (valid && s == 0 && a.norms) a.norms[row] = norm;
+    if (valid && s == 0 && a.norms) a.norms[orow] = norm;
     // fetch the next batch into the same buffer (issuing it at the end of the batch measured
     // faster than right after the last read of the staged rows)
     __syncwarp();
@@ -528,7 +532,7 @@ std::vector<float> fqjl_key_tables(int d, int m, const float* D_r, const int32_t
 bool fqjl_keys_supported(const qjl_projection* P) { return P->d >= 32 && P->d <= 1024 && P->ktab; }
 
 qjl_status launch_fqjl_keys(const qjl_projection* P, const void* x, int dtype, int64_t n, int64_t ld,
-                            uint64_t first_token, uint32_t* bits, float* norms, cudaStream_t st) {
+                            uint64_t first_token, uint32_t* bits, float* norms, cudaStream_t st, const PageMap& pm) {
   if (n <= 0) return QJL_OK;
   KeysArgs a{};
   a.x = x;
@@ -546,6 +550,7 @@ qjl_status launch_fqjl_keys(const qjl_projection* P, const void* x, int dtype, i
   a.norms = norms;
   a.W = P->m / 32;
   a.err = qjl_error_flag(P->device);
+  a.pm = pm;
   if (!a.err) return qjl_set_error(QJL_ERR_CUDA, "cannot allocate the device error flag");
   switch (P->d) {
     case 32: return launch_el<32, 1>(P, a, dtype, n, st);

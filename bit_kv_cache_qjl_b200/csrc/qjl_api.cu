@@ -76,22 +76,6 @@ int* qjl_error_flag(int device) {
 
 namespace {
 
-// Switch to the projection's device for the duration of a call.
-struct DeviceGuard {
-  int prev = -1;
-  bool ok = true;
-  explicit DeviceGuard(int dev) {
-    if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
-    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
-  }
-  ~DeviceGuard() {
-    int cur = -1;
-    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
-  }
-};
-
-bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
-
 // fp64 standard normal from Philox words 0 and 1 (Box-Muller), rounded to fp32.
 float gaussian_f32(uint64_t seed, uint32_t c0, uint32_t c1, uint32_t c2, uint32_t stream) {
   qjl::U32x4 r = qjl::philox({c0, c1, c2, stream}, (uint32_t)seed, (uint32_t)(seed >> 32));

@@ -30,6 +30,55 @@ struct qjl_projection {
   float* h_D_g = nullptr;
 };
 
+// Row -> slot map of a paged cache (qjl_append_*): row r of an append batch is
+// group r's new token at position pos[r]; it lives in page
+// table[r * max_pages + pos[r] / page_tokens], slot pos[r] % page_tokens, i.e.
+// pool row page * page_tokens + slot. With pos == nullptr rows map to
+// themselves (the contiguous calls).
+struct PageMap {
+  const int32_t* pos = nullptr;
+  const int32_t* table = nullptr;
+  int max_pages = 0, page_tokens = 0;
+  int64_t num_pages = 0;
+#if defined(__CUDACC__)
+  // pool row of append row r, or -1 when the position or the page id is out of range
+  __device__ __forceinline__ int64_t slot(int64_t r) const {
+    if (!pos) return r;
+    const int p = __ldg(pos + r);
+    if (p < 0 || p >= max_pages * page_tokens) return -1;
+    const int pg = __ldg(table + r * (int64_t)max_pages + p / page_tokens);
+    if (pg < 0 || (int64_t)pg >= num_pages) return -1;
+    return (int64_t)pg * page_tokens + p % page_tokens;
+  }
+#endif
+};
+
+// Paged reads (qjl_scores_paged, qjl_decode_attention_paged): group g's token
+// t is pool row table[g * max_pages + t / page_tokens] * page_tokens +
+// t % page_tokens, for t < seq_lens[g] (clamped to [0, max_len]).
+struct PagedRead {
+  const int32_t* table = nullptr;
+  const int32_t* seq_lens = nullptr;
+  int max_pages = 0, page_tokens = 0;
+  int64_t num_pages = 0;
+};
+
+// Switch to the projection's device for the duration of a call.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
 // Error helpers (qjl_api.cu). set_error stores a thread-local message and returns s.
 qjl_status qjl_set_error(qjl_status s, const std::string& msg);
 qjl_status qjl_check_launch(const char* what);
@@ -37,7 +86,7 @@ qjl_status qjl_check_launch(const char* what);
 // Launchers. They assume validated arguments and return QJL_OK or QJL_ERR_CUDA.
 qjl_status launch_dense_simt(const qjl_projection* P, const void* keys, int dtype, int64_t n,
                              int64_t ld, uint32_t* bits, float* norms, float* proj_out,
-                             cudaStream_t st);
+                             cudaStream_t st, const PageMap& pm = PageMap());
 qjl_status launch_project_dense(const qjl_projection* P, const float* q, int64_t nq, int64_t ld,
                                 float* out, cudaStream_t st);
 bool dense_tc_supported(const qjl_projection* P, int dtype, const void* keys, int64_t ld);
@@ -47,7 +96,8 @@ qjl_status launch_fqjl_queries(const qjl_projection* P, const float* q, int64_t 
                                float* out, cudaStream_t st);
 std::vector<float> fqjl_key_tables(int d, int m, const float* D_r, const int32_t* perm, const float* D_g);
 qjl_status launch_fqjl_keys(const qjl_projection* P, const void* keys, int dtype, int64_t n, int64_t ld,
-                            uint64_t first_token, uint32_t* bits, float* norms, cudaStream_t st);
+                            uint64_t first_token, uint32_t* bits, float* norms, cudaStream_t st,
+                            const PageMap& pm = PageMap());
 bool scores_mma_supported(int m);
 bool scores_tc_supported(int m, int J);
 qjl_status launch_scores_tc(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t groups,
@@ -56,7 +106,15 @@ qjl_status launch_scores(const qjl_projection* P, const uint32_t* bits, const fl
                          int64_t groups, int64_t N, const float* sq, int J, float* scores,
                          cudaStream_t st);
 qjl_status launch_values_2bit(const void* v, int dtype, int64_t n, int d, uint32_t* codes,
-                              uint16_t* scale, uint16_t* zero, cudaStream_t st);
+                              uint16_t* scale, uint16_t* zero, cudaStream_t st, const PageMap& pm = PageMap());
+qjl_status launch_scores_paged(const qjl_projection* P, const uint32_t* bits_pool, const float* norms_pool,
+                               const PagedRead& pr, int64_t groups, int64_t max_len, const float* sq, int J,
+                               float* scores, cudaStream_t st);
+qjl_status launch_decode_paged(const qjl_projection* P, const uint32_t* bits_pool, const float* norms_pool,
+                               const uint32_t* codes_pool, const uint16_t* scale_pool, const uint16_t* zero_pool,
+                               const PagedRead& pr, int64_t groups, int64_t max_len, const float* sq,
+                               float softmax_scale, float* out, void* ws, cudaStream_t st);
+size_t decode_paged_workspace_bytes(int64_t groups, int64_t max_len, int d);
 size_t decode_workspace_bytes(int64_t groups, int J, int64_t N, int d);
 qjl_status launch_decode(const qjl_projection* P, const uint32_t* bits, const float* norms,
                          const uint32_t* codes, const uint16_t* scale, const uint16_t* zero,

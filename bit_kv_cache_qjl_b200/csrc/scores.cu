@@ -43,6 +43,9 @@
 namespace {
 
 using namespace qjl_sign;
+
+__device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kStageKeys = 256;
@@ -490,11 +493,13 @@ __device__ __forceinline__ void digit_epilogue(const int (&acc)[KT][NT][4], int 
   }
 }
 
-template <int W, int NT, bool DUP, int KT, int SKT>
+// PAGED reads group g's tokens t < seq_lens[g] through the block table
+// (PagedRead); N is then the bound max_len, and the row stride of scores.
+template <int W, int NT, bool DUP, int KT, int SKT, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
     const uint32_t* __restrict__ bits, const float* __restrict__ norms, const float* __restrict__ sq,
     int64_t G, int64_t N, int J, int NS, float est_scale, int64_t items_per_cta, float* __restrict__ scores,
-    int* __restrict__ err) {
+    int* __restrict__ err, PagedRead pr) {
   using namespace qjl_sync;
   constexpr int SK = SKT;
   constexpr int TPW = SK / 16 / kDecConsumers;  // tiles per consumer warp per stage
@@ -535,13 +540,44 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
       for (int64_t it = i0; it < i1; ++it, ++issued) {
         if (!mbar_wait(&empty[s], ph ^ 1u)) { atomicOr(err, 1); break; }
         const int64_t n0 = c * SK;
-        const int cnt = (int)(N - n0 < SK ? N - n0 : SK);
-        const float* nsrc = norms + g * N + n0;
-        const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
-        const uint32_t bbytes = (uint32_t)cnt * W * 4;
-        mbar_expect_tx(&full[s], bbytes + (nbulk ? (uint32_t)cnt * 4 : 0u));
-        bulk_g2s(sbits + (size_t)s * SK * W, bits + (g * N + n0) * W, bbytes, &full[s]);
-        if (nbulk) bulk_g2s(snorm + (size_t)s * SK, nsrc, (uint32_t)cnt * 4, &full[s]);
+        if constexpr (PAGED) {
+          // the stage's tokens [n0, n0 + cnt) of group g, one copy per page segment, each
+          // rounded up to 4 tokens (16 bytes of norms; never past the page, which holds a
+          // multiple of 16 tokens). An empty stage only arrives.
+          const int64_t Lg = min64(max64(__ldg(pr.seq_lens + g), 0), N);
+          const int cnt = (int)max64(0, min64(SK, Lg - n0));
+          const int T = pr.page_tokens;
+          uint32_t tx = 0;
+          for (int pass = 0; pass < 2; ++pass) {
+            if (pass == 1) mbar_expect_tx(&full[s], tx);
+            for (int64_t lo = n0; lo < n0 + cnt;) {
+              const int64_t pi = lo / T;
+              const int64_t hi = min64(n0 + cnt, (pi + 1) * T);
+              const uint32_t len4 = (uint32_t)((hi - lo + 3) & ~3);
+              const int pg = pi < pr.max_pages ? __ldg(pr.table + g * (int64_t)pr.max_pages + pi) : -1;
+              if (pg >= 0 && (int64_t)pg < pr.num_pages) {
+                const int64_t prow = (int64_t)pg * T + (lo - pi * T);
+                if (pass == 0) {
+                  tx += len4 * (W * 4 + 4);
+                } else {
+                  bulk_g2s(sbits + (size_t)s * SK * W + (lo - n0) * W, bits + prow * W, len4 * W * 4, &full[s]);
+                  bulk_g2s(snorm + (size_t)s * SK + (lo - n0), norms + prow, len4 * 4, &full[s]);
+                }
+              } else if (pass == 0) {
+                atomicOr(err, 8);  // a bad page id: its tokens keep stale stage data
+              }
+              lo = hi;
+            }
+          }
+        } else {
+          const int cnt = (int)(N - n0 < SK ? N - n0 : SK);
+          const float* nsrc = norms + g * N + n0;
+          const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
+          const uint32_t bbytes = (uint32_t)cnt * W * 4;
+          mbar_expect_tx(&full[s], bbytes + (nbulk ? (uint32_t)cnt * 4 : 0u));
+          bulk_g2s(sbits + (size_t)s * SK * W, bits + (g * N + n0) * W, bbytes, &full[s]);
+          if (nbulk) bulk_g2s(snorm + (size_t)s * SK, nsrc, (uint32_t)cnt * 4, &full[s]);
+        }
         if (c == 0) { c = cpg - 1; --g; } else { --c; }
         if (++s == NS) { s = 0; ph ^= 1u; }
       }
@@ -570,6 +606,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
   const float* nsrc = norms + g * N + (int64_t)c * SK;
   float* gout = scores + g * (int64_t)J * N + (int64_t)c * SK;
   int64_t cur_g = -1;
+  int64_t Lg = N;  // valid tokens of the current group (PAGED)
   int s = 0;
   uint32_t ph = 0;
   uint2 breg[NT == 1 ? W : 1];
@@ -578,7 +615,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
   bool dead = false;  // a timed-out wait: keep the loop's barriers, skip the work
   const int nitems = (int)(i1 - i0);
   for (int item = 0; item < nitems; ++item) {
-    const int cnt = c == cpg32 - 1 ? last_cnt : SK;
+    if (PAGED && g != cur_g) Lg = min64(max64(__ldg(pr.seq_lens + g), 0), N);
+    const int cnt = PAGED ? (int)max64(0, min64(SK, Lg - (int64_t)c * SK))
+                          : (c == cpg32 - 1 ? last_cnt : SK);
     if (g != cur_g) {
       named_sync(1, kDecConsumers * 32);
       build_tables_dig<W>(sq + g * (int64_t)J * (32 * W), J, NT, DUP, est_scale, s_inv, s_mul, s_qsum, Btab,
@@ -599,8 +638,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
     if (!dead) {
       // the producer bulk-copied the norms exactly when they were 16-byte aligned
       // and a multiple of 4; otherwise they are read from global memory
-      const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
-      const bool whole = groups_aligned && cnt == SK;
+      const bool nbulk = PAGED || ((((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0));
+      const bool whole = (PAGED || groups_aligned) && cnt == SK;
       const uint32_t* sb = sbits + (size_t)s * SK * W;
       const float* sn = snorm + (size_t)s * SK;
 #pragma unroll 1
@@ -752,14 +791,14 @@ qjl_status launch_decode_fast(const qjl_projection* P, const uint32_t* bits, con
   return qjl_check_launch("scores_decode_kernel");
 }
 
-template <int W, int NT, bool DUP, int KT, int SKT>
+template <int W, int NT, bool DUP, int KT, int SKT, bool PAGED = false>
 qjl_status launch_digit(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t G, int64_t N,
-                        const float* sq, int J, float* scores, cudaStream_t st) {
+                        const float* sq, int J, float* scores, cudaStream_t st, const PagedRead& pr = PagedRead()) {
   // ring depth: as many stages as keep two CTAs per SM within shared memory
   const int NS = SKT * (W + 1) * 4 * 4 <= 80 * 1024 ? 4 : (SKT * (W + 1) * 4 * 3 <= 110 * 1024 ? 3 : 2);
   const size_t smem = 3 * 64 * 4 + 256 + (size_t)NT * W * 32 * sizeof(uint2) + (size_t)NS * SKT * (W + 1) * 4 +
                       (size_t)2 * NS * 8;
-  auto kern = scores_digit_kernel<W, NT, DUP, KT, SKT>;
+  auto kern = scores_digit_kernel<W, NT, DUP, KT, SKT, PAGED>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return qjl_check_launch("scores_digit_kernel smem attribute");
@@ -774,18 +813,18 @@ qjl_status launch_digit(const qjl_projection* P, const uint32_t* bits, const flo
   const int64_t ipc = (total + grid - 1) / grid;
   const int64_t nblk = (total + ipc - 1) / ipc;
   qjl_log_launch("scores_digit_kernel", nblk, kDecThreads, smem, per_sm);
-  kern<<<(unsigned)nblk, kDecThreads, smem, st>>>(bits, norms, sq, G, N, J, NS, P->est_scale, ipc, scores, err);
+  kern<<<(unsigned)nblk, kDecThreads, smem, st>>>(bits, norms, sq, G, N, J, NS, P->est_scale, ipc, scores, err, pr);
   return qjl_check_launch("scores_digit_kernel");
 }
 
 // One or two queries per group: 1024-key stages; four tiles per batch at
 // m = 256, two at m = 512 (registers).
-template <int W>
+template <int W, bool PAGED = false>
 qjl_status launch_digit_w(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t G, int64_t N,
-                          const float* sq, int J, float* scores, cudaStream_t st) {
+                          const float* sq, int J, float* scores, cudaStream_t st, const PagedRead& pr = PagedRead()) {
   constexpr int KT = W == 8 ? 4 : 2;
-  return J == 1 ? launch_digit<W, 1, true, KT, 1024>(P, bits, norms, G, N, sq, J, scores, st)
-                : launch_digit<W, 1, false, KT, 1024>(P, bits, norms, G, N, sq, J, scores, st);
+  return J == 1 ? launch_digit<W, 1, true, KT, 1024, PAGED>(P, bits, norms, G, N, sq, J, scores, st, pr)
+                : launch_digit<W, 1, false, KT, 1024, PAGED>(P, bits, norms, G, N, sq, J, scores, st, pr);
 }
 
 }  // namespace
@@ -828,4 +867,13 @@ qjl_status launch_scores(const qjl_projection* P, const uint32_t* bits, const fl
   const int blocks = (int)std::min<int64_t>(want, (int64_t)qjl_num_sms(P->device) * 16);
   scores_simt_kernel<<<blocks, 256, 0, st>>>(bits, norms, sq, G, N, J, P->m / 32, P->est_scale, scores);
   return qjl_check_launch("scores_simt_kernel");
+}
+
+qjl_status launch_scores_paged(const qjl_projection* P, const uint32_t* bits_pool, const float* norms_pool,
+                               const PagedRead& pr, int64_t G, int64_t max_len, const float* sq, int J,
+                               float* scores, cudaStream_t st) {
+  if (J > 2 || (P->m != 256 && P->m != 512))
+    return qjl_set_error(QJL_ERR_UNSUPPORTED, "paged scores support q_per_group <= 2 and m in {256, 512}");
+  return P->m == 256 ? launch_digit_w<8, true>(P, bits_pool, norms_pool, G, max_len, sq, J, scores, st, pr)
+                     : launch_digit_w<16, true>(P, bits_pool, norms_pool, G, max_len, sq, J, scores, st, pr);
 }

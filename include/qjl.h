@@ -155,9 +155,10 @@ qjl_status qjl_project_queries(const qjl_projection* proj, const float* q, int64
  *   scores  out [groups][q_per_group][N] fp32.
  *   1 <= q_per_group <= 64. Grouped-query attention puts q_per_group query
  *   heads on one key head's bits.
- * Sq is rounded per (group, query) to 16-bit fixed point (scale max|Sq|/32639).
- * The sign sums are exact integers. The added error is at most
- * c*alpha*||k|| * m * max|Sq| / 65278.
+ * Sq is rounded per (group, query) to fixed point: with 1 or 2 queries per
+ * group at m = 256 or 512 to 31 - log2(m) bits (scale max|Sq| / (2^31/m - 1)),
+ * otherwise to 16 bits (scale max|Sq|/32639). The sign sums are exact
+ * integers, so the added error is at most c*alpha*||k|| * m * max|Sq| / 65278.
  */
 qjl_status qjl_scores(const qjl_projection* proj, const uint32_t* bits, const float* norms,
                       int64_t groups, int64_t N, const float* sq, int q_per_group,
@@ -234,6 +235,97 @@ qjl_status qjl_decode_attention_noalloc(const qjl_projection* proj, const uint32
                                         int64_t groups, int64_t N, const float* sq,
                                         int q_per_group, float softmax_scale, float* out,
                                         void* stream);
+
+/*
+ * Paged cache. A decode step appends one token per group (sequence x key head)
+ * and then reads the whole cache (KIVI abstract: the decode step loads the
+ * whole KV cache per generated token). A serving engine keeps such a cache in
+ * fixed-size pages. The pages name no layout; this one is ours:
+ *   - A pool holds num_pages pages of page_tokens token slots each.
+ *     page_tokens is a multiple of 16.
+ *   - Group g's logical token t lives in page block_table[g*max_pages +
+ *     t/page_tokens], slot t % page_tokens, i.e. pool row
+ *     page * page_tokens + slot.
+ *   - Pools are arrays over pool rows:
+ *       bits  [num_pages*page_tokens][m/32] uint32
+ *       norms [num_pages*page_tokens] fp32
+ *       codes [num_pages*page_tokens][d/16] uint32
+ *       scale, zero [num_pages*page_tokens][d/32] binary16
+ *     Their layout per row is that of the contiguous calls. Every pool is
+ *     16-byte aligned.
+ *   - block_table is int32 device [groups][max_pages]. positions and seq_lens
+ *     are int32 device [groups]. The caller owns pools, tables and lengths,
+ *     and assigns pages.
+ * The host checks everything it can see. The kernels check, before every
+ * access, the positions and the block-table entries they read: a position
+ * outside [0, max_pages*page_tokens) or a page id outside [0, num_pages) is
+ * skipped, so it is never read or written, and the call's results for it
+ * are undefined.
+ */
+
+/*
+ * Sketch one key per group (as qjl_quantize_keys) into the paged pools, at
+ * logical position positions[g] of group g.
+ *   keys  [groups][ld] of `dtype`, 16-byte aligned, ld*elsize % 16 == 0.
+ * The D-FQJL dither of a key is seeded by its pool row, page*page_tokens +
+ * slot (the first_token of the contiguous call). Dense keys take the fp32
+ * SIMT projection: one key per group and step is latency work.
+ */
+qjl_status qjl_append_keys(const qjl_projection* proj, const void* keys, qjl_dtype dtype,
+                           int64_t groups, int64_t ld, const int32_t* positions,
+                           const int32_t* block_table, int max_pages, int page_tokens,
+                           int64_t num_pages, uint32_t* bits_pool, float* norms_pool,
+                           void* stream);
+
+/*
+ * 2-bit per-token values (as qjl_quantize_values_2bit, bit for bit) of one
+ * token per group, written at positions[g] of group g.
+ *   v  [groups][d] of `dtype`, 16-byte aligned, d a multiple of 32.
+ */
+qjl_status qjl_append_values_2bit(const void* v, qjl_dtype dtype, int64_t groups, int d,
+                                  const int32_t* positions, const int32_t* block_table,
+                                  int max_pages, int page_tokens, int64_t num_pages,
+                                  uint32_t* codes_pool, uint16_t* scale_pool,
+                                  uint16_t* zero_pool, void* stream);
+
+/*
+ * The estimator of qjl_scores over each group's first seq_lens[g] tokens of
+ * a paged cache (seq_lens clamped to [0, max_len]).
+ *   max_len  host bound on seq_lens, <= max_pages*page_tokens. It is also the
+ *            row stride of scores.
+ *   sq       [groups][q_per_group][m] fp32, 16-byte aligned.
+ *   scores   out [groups][q_per_group][max_len] fp32. Entries at t >=
+ *            seq_lens[g] are not written.
+ * Supports 1 <= q_per_group <= 2 and m in {256, 512}: it is the shift-window
+ * kernel of qjl_scores, with bulk copies gathered per page segment.
+ */
+qjl_status qjl_scores_paged(const qjl_projection* proj, const uint32_t* bits_pool,
+                            const float* norms_pool, const int32_t* block_table, int max_pages,
+                            int page_tokens, int64_t num_pages, const int32_t* seq_lens,
+                            int64_t groups, int64_t max_len, const float* sq, int q_per_group,
+                            float* scores, void* stream);
+
+/* Workspace bytes qjl_decode_attention_paged needs for these sizes. */
+size_t qjl_decode_paged_workspace_bytes(int64_t groups, int64_t max_len, int d);
+
+/*
+ * Fused decode attention (as qjl_decode_attention, one query per group) over
+ * each group's first seq_lens[g] tokens of a paged cache.
+ *   max_len  host bound on seq_lens, <= max_pages*page_tokens.
+ *   sq       [groups][m] fp32.   out [groups][d] fp32.
+ *   ws       device workspace of >= qjl_decode_paged_workspace_bytes(...)
+ *            bytes, 16-byte aligned. Calls that overlap on the GPU must not
+ *            share it.
+ * A group with seq_lens[g] <= 0 gets an all-zero output row. Supports d = 128
+ * and m = 256.
+ */
+qjl_status qjl_decode_attention_paged(const qjl_projection* proj, const uint32_t* bits_pool,
+                                      const float* norms_pool, const uint32_t* codes_pool,
+                                      const uint16_t* scale_pool, const uint16_t* zero_pool,
+                                      const int32_t* block_table, int max_pages, int page_tokens,
+                                      int64_t num_pages, const int32_t* seq_lens, int64_t groups,
+                                      int64_t max_len, const float* sq, float softmax_scale,
+                                      float* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Static text for a status code. */
 const char* qjl_status_string(qjl_status s);

@@ -30,6 +30,7 @@ Modules:
     qjl        key sketch, query projection, asymmetric estimator
     kivi       2-bit per-token value quantisation
     attention  softmax(scores) . V over dequantised values
+    paged      append one token per group into pages; reads through a block table
 
 Parity status (each function's pins are in tests/test_oracle_*.py):
     The absolute bit stream of the generator is parity unpinned on CPU. It is
@@ -37,4 +38,4 @@ Parity status (each function's pins are in tests/test_oracle_*.py):
     library generator; see ``philox``.
 """
 
-from . import philox, params, hadamard, qjl, kivi, attention  # noqa: F401
+from . import philox, params, hadamard, qjl, kivi, attention, paged  # noqa: F401
