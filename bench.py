@@ -388,6 +388,55 @@ def build_workload(name, dev, qjl, wl, torch):
         W.update(units=G * Nd, unit="tokens/s", inputs=[keys, vals, q], outputs=[out], dtype="bf16",
                  desc="%s: D-FQJL sigma_rel 0.5, B=32, 32 heads, N=16384, d=128, m=256; quantize keys and 2-bit "
                       "values, project queries, fused softmax(QK)V decode" % name)
+    elif name == "paged_decode":
+        # the dfqjl_decode cache in 256-token pages under a shuffled block table; a step appends one
+        # key and one value per group (at the last position, so the length stays N) and attends over
+        # all N tokens through the table
+        Bd, Hd, Nd, m, T = 32, 32, 16384, 256, 256
+        G, pages = Bd * Hd, Nd // T
+        P = qjl.Projection(5, D, m, "dfqjl", dither_sigma_rel=0.5)
+        keys, vals = wl.decode_kv(dev, B=Bd, H=Hd, N=Nd, d=D)
+        keys, vals = keys.reshape(-1, D), vals.reshape(-1, D)
+        num_pages = G * pages + 64
+        perm = torch.randperm(num_pages, generator=torch.Generator().manual_seed(509))[:G * pages]
+        table = perm.view(G, pages).to(torch.int32).to(dev)
+        t = torch.arange(Nd, device=dev)
+        rows = (table.long()[:, t // T] * T + (t % T)[None, :]).reshape(-1)
+        R = num_pages * T
+        pool = dict(bits=torch.zeros((R, m // 32), dtype=torch.int32, device=dev),
+                    norms=torch.zeros((R,), dtype=torch.float32, device=dev),
+                    codes=torch.zeros((R, D // 16), dtype=torch.int32, device=dev),
+                    scale=torch.zeros((R, D // 32), dtype=torch.float16, device=dev),
+                    zero=torch.zeros((R, D // 32), dtype=torch.float16, device=dev))
+        b0, n0 = qjl.quantize_keys(P, keys)
+        c0, s0, z0 = qjl.quantize_values_2bit(vals)
+        for k, v in (("bits", b0), ("norms", n0), ("codes", c0), ("scale", s0), ("zero", z0)):
+            pool[k][rows] = v
+        del b0, n0, c0, s0, z0, rows
+        seq = torch.full((G,), Nd, dtype=torch.int32, device=dev)
+        cache = qjl.PagedCache(T, table, seq, pool["bits"], pool["norms"], pool["codes"], pool["scale"],
+                               pool["zero"])
+        pos = torch.full((G,), Nd - 1, dtype=torch.int32, device=dev)
+        newk = wl.normal((G, D), 511, dev, torch.bfloat16)
+        newv = wl.normal((G, D), 512, dev, torch.bfloat16)
+        q = wl.decode_queries(dev, B=Bd, H=Hd, d=D).reshape(-1, D)
+        sq = torch.empty((G, m), dtype=torch.float32, device=dev)
+        out = torch.empty((G, D), dtype=torch.float32, device=dev)
+        ws = torch.empty((qjl.decode_paged_workspace_bytes(G, Nd, D),), dtype=torch.uint8, device=dev)
+        smx = 1.0 / math.sqrt(D)
+        stages = [
+            Stage("append_keys", lambda: qjl.append_keys(P, cache, newk, pos), G, 2 * D + m // 8 + 4,
+                  fqjl_flops_per_key(D, m)),
+            Stage("append_values", lambda: qjl.append_values_2bit(cache, newv, pos), G, 2 * D + D // 4 + D // 8),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * m),
+            Stage("decode_attention_paged", lambda: qjl.decode_attention_paged(P, cache, sq, Nd, smx, out=out,
+                                                                               workspace=ws), G * Nd,
+                  m // 8 + 4 + D // 4 + D // 8, 0, "decode_stream_kernel", "decode.cu", launches=2),
+        ]
+        W.update(units=G * Nd, unit="tokens/s", inputs=[newk, newv, q], outputs=[out], dtype="bf16",
+                 desc="%s: D-FQJL sigma_rel 0.5, B=32, 32 heads, N=16384 in 256-token pages (shuffled block "
+                      "table), d=128, m=256; append 1 key + 2-bit value per head, project queries, fused paged "
+                      "decode" % name)
     else:
         raise SystemExit("unknown workload %s" % name)
     W["stages"] = stages
@@ -402,7 +451,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=["decode_llama7b", "gqa_decode", "dense_1head", "pfqjl_bulk_m256", "pfqjl_bulk_m1024",
-                             "dfqjl_decode"])
+                             "dfqjl_decode", "paged_decode"])
     ap.add_argument("--ref-sample", type=int, default=4096)
     ap.add_argument("--cpu-sample", type=int, default=1 << 21)
     ap.add_argument("--profile-case", default=None,
