@@ -34,6 +34,7 @@
 #include <stdlib.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <string.h>
 
 #include "qjl_internal.h"
@@ -642,10 +643,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
       const bool whole = (PAGED || groups_aligned) && cnt == SK;
       const uint32_t* sb = sbits + (size_t)s * SK * W;
       const float* sn = snorm + (size_t)s * SK;
-#pragma unroll 1
-      for (int i = 0; i < TPW; i += KT) {
-        const int tile0 = warp + i * kDecConsumers;
-        if (tile0 * 16 >= cnt) break;
+      // one batch of KT tiles from tile0: loads, shift-window MMAs, epilogue (CHECK: bounds and
+      // norm source checks for a partial or unaligned stage)
+      auto batch = [&](int tile0, auto check) {
+        constexpr bool CHECK = decltype(check)::value;
         uint32_t w0[KT][W / 4], w1[KT][W / 4];
 #pragma unroll
         for (int t = 0; t < KT; ++t) {
@@ -684,10 +685,26 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
             }
           }
         }
-        if (whole)
-          digit_epilogue<NT, DUP, KT, false>(acc, tile0, gq, par, half, cnt, nbulk, sn, nsrc, mul, qs, J, N, gout);
-        else
-          digit_epilogue<NT, DUP, KT, true>(acc, tile0, gq, par, half, cnt, nbulk, sn, nsrc, mul, qs, J, N, gout);
+        digit_epilogue<NT, DUP, KT, CHECK>(acc, tile0, gq, par, half, cnt, nbulk, sn, nsrc, mul, qs, J, N, gout);
+      };
+      if (whole) {
+        // a whole stage: at m = 256 the batches are unrolled, so one batch's epilogue can overlap the
+        // next one's MMAs (-3 % time for one query per group, -10 % for two); at m = 512 the
+        // registers would spill
+        if constexpr (W == 8) {
+#pragma unroll
+          for (int i = 0; i < TPW; i += KT) batch(warp + i * kDecConsumers, std::false_type());
+        } else {
+#pragma unroll 1
+          for (int i = 0; i < TPW; i += KT) batch(warp + i * kDecConsumers, std::false_type());
+        }
+      } else {
+#pragma unroll 1
+        for (int i = 0; i < TPW; i += KT) {
+          const int tile0 = warp + i * kDecConsumers;
+          if (tile0 * 16 >= cnt) break;
+          batch(tile0, std::true_type());
+        }
       }
     }
     __syncwarp();
