@@ -263,7 +263,8 @@ __device__ __forceinline__ void philox_x4(qjl::U32x4 (&c)[4], uint32_t k0, uint3
 
 // ---- kernel -------------------------------------------------------------------------------------
 
-template <int E, int L, int ES, int MODE>
+// PAGED: appends to a paged cache (a.pm maps rows to pool rows); otherwise rows map to themselves
+template <int E, int L, int ES, int MODE, bool PAGED>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const KeysArgs a) {
   using G = Geo<E, L, ES>;
   constexpr int K = G::K;
@@ -302,8 +303,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
   for (uint32_t phase = 0; q < nbatch; q += stride, phase ^= 1u) {
     const int64_t row = q * K + kp;
     // the output row (a page slot when appending to a paged cache) and the dither's token index
-    const int64_t orow = row < a.n ? a.pm.slot(row) : -1;
-    if (row < a.n && orow < 0) atomicOr(a.err, 8);
+    const int64_t orow = row < a.n ? (PAGED ? a.pm.slot(row) : row) : -1;
+    if (PAGED && row < a.n && orow < 0) atomicOr(a.err, 8);
     const bool valid = orow >= 0;
     if (!__all_sync(0xffffffffu, mbar_wait(bar, phase))) {
       // the batch never landed (the whole warp agrees): flag it, give the copy one more
@@ -312,7 +313,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
       mbar_wait(bar, phase);
       return;
     }
-    const uint64_t tok = a.pm.pos ? (uint64_t)orow : a.first_token + (uint64_t)row;
+    const uint64_t tok = PAGED ? (uint64_t)orow : a.first_token + (uint64_t)row;
     float norm = 0.f;
 
     for (int bl = 0; bl < nbl; ++bl) {
@@ -449,11 +450,11 @@ Layout layout_for(int d) {
   return g;
 }
 
-template <int E, int L, int ES, int MODE>
+template <int E, int L, int ES, int MODE, bool PAGED>
 qjl_status launch_t(const qjl_projection* P, KeysArgs a, int64_t n, cudaStream_t st) {
   using G = Geo<E, L, ES>;
   constexpr bool BUF = (MODE == MODE_P);
-  auto kern = fqjl_keys_kernel<E, L, ES, MODE>;
+  auto kern = fqjl_keys_kernel<E, L, ES, MODE, PAGED>;
   const int d = P->d, nb = P->m / d;
   const int per_launch = std::max(1, (int)std::min<size_t>(nb, kTableBudget / ((size_t)G::TBLK * 4)));
   const size_t per_warp = G::XBUF + 8 + (BUF ? G::GBUF : 0);
@@ -489,9 +490,14 @@ qjl_status launch_t(const qjl_projection* P, KeysArgs a, int64_t n, cudaStream_t
 template <int E, int L>
 qjl_status launch_el(const qjl_projection* P, const KeysArgs& a, int dtype, int64_t n, cudaStream_t st) {
   const bool dmode = P->kind == QJL_DFQJL;
+  if (a.pm.pos) {
+    if (dtype == QJL_F32)
+      return dmode ? launch_t<E, L, 4, MODE_D, true>(P, a, n, st) : launch_t<E, L, 4, MODE_P, true>(P, a, n, st);
+    return dmode ? launch_t<E, L, 2, MODE_D, true>(P, a, n, st) : launch_t<E, L, 2, MODE_P, true>(P, a, n, st);
+  }
   if (dtype == QJL_F32)
-    return dmode ? launch_t<E, L, 4, MODE_D>(P, a, n, st) : launch_t<E, L, 4, MODE_P>(P, a, n, st);
-  return dmode ? launch_t<E, L, 2, MODE_D>(P, a, n, st) : launch_t<E, L, 2, MODE_P>(P, a, n, st);
+    return dmode ? launch_t<E, L, 4, MODE_D, false>(P, a, n, st) : launch_t<E, L, 4, MODE_P, false>(P, a, n, st);
+  return dmode ? launch_t<E, L, 2, MODE_D, false>(P, a, n, st) : launch_t<E, L, 2, MODE_P, false>(P, a, n, st);
 }
 
 }  // namespace
