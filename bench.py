@@ -437,6 +437,51 @@ def build_workload(name, dev, qjl, wl, torch):
                  desc="%s: D-FQJL sigma_rel 0.5, B=32, 32 heads, N=16384 in 256-token pages (shuffled block "
                       "table), d=128, m=256; append 1 key + 2-bit value per head, project queries, fused paged "
                       "decode" % name)
+    elif name == "kivi_keys_decode":
+        # the KIVI per-channel 2-bit key baseline on the decode_llama7b keys: quantize every key per
+        # channel (32-token blocks) and score one query per head; "accuracy" compares its scores and the
+        # QJL sketch's (dense, m=256) with the exact inner products on sampled heads
+        G = B * H
+        keys = wl.llama_keys(dev, B=B, H=H, N=N, d=D).reshape(G, N, D)
+        q = wl.llama_queries(dev, B=B, H=H, d=D).reshape(G, 1, D)
+        nb = (N + 31) // 32
+        codes = torch.empty((G, N, D // 16), dtype=torch.int32, device=dev)
+        sc = torch.empty((G, nb, D), dtype=torch.float16, device=dev)
+        zr = torch.empty((G, nb, D), dtype=torch.float16, device=dev)
+        out = torch.empty((G, 1, N), dtype=torch.float32, device=dev)
+        stages = [
+            Stage("kivi_quantize_keys", lambda: qjl.kivi_quantize_keys_2bit(keys, codes, sc, zr), G * N,
+                  2 * D + D // 4 + 4 * D // 32, 0, "kivi_keys_quantize_kernel", "kivi_keys.cu"),
+            Stage("kivi_key_scores", lambda: qjl.kivi_key_scores(codes, sc, zr, q, out=out), G * N,
+                  D // 4 + 4 * D // 32 + 4, 0, "kivi_key_scores_kernel", "kivi_keys.cu"),
+        ]
+        W.update(units=G * N, unit="keys/s", inputs=[keys, q], outputs=[out], dtype="bf16",
+                 desc="%s: KIVI per-channel 2-bit keys (32-token blocks, fp16 scale/zero, 48 B/key) on B=8, "
+                      "heads=32, N=32768, d=128; quantize all keys, score 1 query/head" % name)
+
+        def accuracy(heads=(0, 37, 101, 255)):
+            import numpy as np
+            Pq = qjl.Projection(2, D, M, "dense", s_bf16=True)
+            res = {"sampled_heads": len(heads), "keys_per_head": N}
+            errs = {"kivi_2bit_per_channel": [], "qjl_dense_m256": []}
+            exact_all = []
+            for g in heads:
+                kh = keys[g].double().cpu().numpy()
+                qh = q[g, 0].double().cpu().numpy()
+                exact = kh @ qh
+                bits, nrm = qjl.quantize_keys(Pq, keys[g])
+                sqh = qjl.project_queries(Pq, q[g])
+                est = qjl.scores(Pq, bits.view(1, N, M // 32), nrm.view(1, N), sqh.view(1, 1, M))
+                errs["qjl_dense_m256"].append(est[0, 0].double().cpu().numpy() - exact)
+                errs["kivi_2bit_per_channel"].append(out[g, 0].double().cpu().numpy() - exact)
+                exact_all.append(exact)
+            ex = np.concatenate(exact_all)
+            for k, e in errs.items():
+                e = np.concatenate(e)
+                res[k] = {"rel_rms_error": float(np.sqrt((e * e).mean() / (ex * ex).mean())),
+                          "bytes_per_key": 48 if k.startswith("kivi") else M // 8 + 4}
+            return res
+        W["accuracy"] = accuracy
     else:
         raise SystemExit("unknown workload %s" % name)
     W["stages"] = stages
@@ -451,7 +496,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=["decode_llama7b", "gqa_decode", "dense_1head", "pfqjl_bulk_m256", "pfqjl_bulk_m1024",
-                             "dfqjl_decode", "paged_decode"])
+                             "dfqjl_decode", "paged_decode", "kivi_keys_decode"])
     ap.add_argument("--ref-sample", type=int, default=4096)
     ap.add_argument("--cpu-sample", type=int, default=1 << 21)
     ap.add_argument("--profile-case", default=None,
@@ -593,6 +638,8 @@ def main():
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
+    if "accuracy" in Wk and rank == 0:
+        line["accuracy"] = Wk["accuracy"]()
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

@@ -23,8 +23,8 @@ from ._lib import Options, lib
 
 __all__ = ["Projection", "QJLError", "quantize_keys", "project_queries", "scores",
            "quantize_values_2bit", "decode_attention", "decode_workspace_bytes", "PagedCache", "append_keys",
-           "append_values_2bit", "scores_paged", "decode_attention_paged", "decode_paged_workspace_bytes", "lib",
-           "KINDS"]
+           "append_values_2bit", "scores_paged", "decode_attention_paged", "decode_paged_workspace_bytes",
+           "kivi_quantize_keys_2bit", "kivi_key_scores", "lib", "KINDS"]
 
 KINDS = {"dense": 0, "dfqjl": 1, "pfqjl": 2}
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
@@ -248,4 +248,33 @@ def decode_attention_paged(proj, cache, sq, max_len, softmax_scale, out=None, wo
                                             _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                             _stream(stream)),
            "qjl_decode_attention_paged")
+    return out
+
+
+def kivi_quantize_keys_2bit(keys, codes=None, scale=None, zero=None, stream=None):
+    """KIVI per-channel 2-bit keys: keys [G, N, d] -> (codes [G, N, d/16] int32, scale, zero [G, ceil(N/32), d] fp16)."""
+    _cuda(keys, "keys")
+    G, N, d = keys.shape
+    nb = (N + 31) // 32
+    if codes is None:
+        codes = torch.empty((G, N, d // 16), dtype=torch.int32, device=keys.device)
+    if scale is None:
+        scale = torch.empty((G, nb, d), dtype=torch.float16, device=keys.device)
+    if zero is None:
+        zero = torch.empty((G, nb, d), dtype=torch.float16, device=keys.device)
+    _check(lib().qjl_kivi_quantize_keys_2bit(_ptr(keys), _DTYPES[keys.dtype], G, N, d, _ptr(codes), _ptr(scale),
+                                             _ptr(zero), _stream(stream)), "qjl_kivi_quantize_keys_2bit")
+    return codes, scale, zero
+
+
+def kivi_key_scores(codes, scale, zero, q, out=None, stream=None):
+    """<q, k_hat> over KIVI keys: q [G, J, d] fp32 -> [G, J, N] fp32."""
+    for t, nm in ((codes, "codes"), (scale, "scale"), (zero, "zero"), (q, "q")):
+        _cuda(t, nm)
+    G, N = codes.shape[0], codes.shape[1]
+    J, d = q.shape[1], q.shape[2]
+    if out is None:
+        out = torch.empty((G, J, N), dtype=torch.float32, device=q.device)
+    _check(lib().qjl_kivi_key_scores(_ptr(codes), _ptr(scale), _ptr(zero), G, N, d, _ptr(q), J, _ptr(out),
+                                     _stream(stream)), "qjl_kivi_key_scores")
     return out

@@ -44,6 +44,10 @@ SIGNATURES = {
     "qjl_decode_attention_paged": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                            c_int, c_int64, c_void_p, c_int64, c_int64, c_void_p, c_float, c_void_p,
                                            c_void_p, c_size_t, c_void_p]),
+    "qjl_kivi_quantize_keys_2bit": (c_int, [c_void_p, c_int, c_int64, c_int64, c_int, c_void_p, c_void_p, c_void_p,
+                                            c_void_p]),
+    "qjl_kivi_key_scores": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int, c_void_p, c_int, c_void_p,
+                                    c_void_p]),
     "qjl_status_string": (ctypes.c_char_p, [c_int]),
     "qjl_last_error_message": (ctypes.c_char_p, []),
     "qjl_version": (ctypes.c_char_p, []),

@@ -327,6 +327,36 @@ qjl_status qjl_decode_attention_paged(const qjl_projection* proj, const uint32_t
                                       int64_t max_len, const float* sq, float softmax_scale,
                                       float* out, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * KIVI per-channel 2-bit keys: the like-for-like baseline of the QJL sketch on
+ * the same shapes. The KIVI abstract ("KIVI: A Tuning-Free Asymmetric 2bit
+ * Quantization for KV Cache", "Vladimir Braverman" page) quantises keys per
+ * channel and values per token. A channel's group is a block of 32
+ * consecutive tokens of one key head; the last block of a ragged N is shorter.
+ * Per (block, channel): zero = fp16(min), scale = fp16(fp32(max - min) / 3),
+ * code = clamp(rint_even(fp32(fp32(k - zero) / scale)), 0, 3), or 0 when
+ * scale == 0. At d = 128 that is 48 bytes per key, against 36 for the QJL
+ * sketch at m = 256.
+ *   keys   [groups][N][d] of `dtype` (rows contiguous), d in {64, 128, 256}.
+ *   codes  out [groups][N][d/16] uint32: channel c at bits 2*(c%16) of word c/16.
+ *   scale, zero  out [groups][ceil(N/32)][d] binary16.
+ * All four buffers are 16-byte aligned.
+ */
+qjl_status qjl_kivi_quantize_keys_2bit(const void* keys, qjl_dtype dtype, int64_t groups, int64_t N,
+                                       int d, uint32_t* codes, uint16_t* scale, uint16_t* zero,
+                                       void* stream);
+
+/*
+ * Scores over KIVI keys:
+ *   scores[g][j][n] = sum_c q[g][j][c] * (code[g][n][c] * scale + zero)
+ * with the scale and zero of token n's block, accumulated in fp32.
+ *   q       [groups][q_per_group][d] fp32, 1 <= q_per_group <= 64.
+ *   scores  out [groups][q_per_group][N] fp32.
+ */
+qjl_status qjl_kivi_key_scores(const uint32_t* codes, const uint16_t* scale, const uint16_t* zero,
+                               int64_t groups, int64_t N, int d, const float* q, int q_per_group,
+                               float* scores, void* stream);
+
 /* Static text for a status code. */
 const char* qjl_status_string(qjl_status s);
 
