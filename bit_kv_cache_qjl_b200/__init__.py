@@ -24,7 +24,7 @@ from ._lib import Options, lib
 __all__ = ["Projection", "QJLError", "quantize_keys", "project_queries", "scores",
            "quantize_values_2bit", "decode_attention", "decode_workspace_bytes", "PagedCache", "append_keys",
            "append_values_2bit", "scores_paged", "decode_attention_paged", "decode_paged_workspace_bytes",
-           "kivi_quantize_keys_2bit", "kivi_key_scores", "lib", "KINDS"]
+           "kivi_quantize_keys_2bit", "kivi_key_scores", "device_errors", "lib", "KINDS"]
 
 KINDS = {"dense": 0, "dfqjl": 1, "pfqjl": 2}
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
@@ -278,3 +278,10 @@ def kivi_key_scores(codes, scale, zero, q, out=None, stream=None):
     _check(lib().qjl_kivi_key_scores(_ptr(codes), _ptr(scale), _ptr(zero), G, N, d, _ptr(q), J, _ptr(out),
                                      _stream(stream)), "qjl_kivi_key_scores")
     return out
+
+
+def device_errors(device=0, clear=True):
+    """The per-device error bits the kernels set (synchronises the device); see include/qjl.h."""
+    flags = ctypes.c_int(0)
+    lib().qjl_device_errors(int(device), int(bool(clear)), ctypes.byref(flags))
+    return flags.value

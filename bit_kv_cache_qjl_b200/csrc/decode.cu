@@ -415,7 +415,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
                     else bulk_g2s(st + off[a] + (lo - n0) * per_tok[a], src[a], len4 * per_tok[a], &full[s]);
                   }
                 } else if (pass == 0) {
-                  atomicOr(err, 8);  // a bad page id: its tokens keep stale stage data
+                  atomicOr(err, QJL_DEVERR_PAGE);  // a bad page id: its tokens keep stale stage data
                 }
                 lo = hi;
               }

@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(256) dense_simt_kernel(const void* __restrict_
     // output row: the same row, or the key's page slot when appending to a paged cache
     const int64_t orow = pm.slot(row);
     if (orow < 0) {
-      if (lane == 0 && err) atomicOr(err, 8);
+      if (lane == 0 && err) atomicOr(err, QJL_DEVERR_PAGE);
       continue;
     }
     float sumsq = 0.f;

@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
     const int64_t row = q * K + kp;
     // the output row (a page slot when appending to a paged cache) and the dither's token index
     const int64_t orow = row < a.n ? (PAGED ? a.pm.slot(row) : row) : -1;
-    if (PAGED && row < a.n && orow < 0) atomicOr(a.err, 8);
+    if (PAGED && row < a.n && orow < 0) atomicOr(a.err, QJL_DEVERR_PAGE);
     const bool valid = orow >= 0;
     if (!__all_sync(0xffffffffu, mbar_wait(bar, phase))) {
       // the batch never landed (the whole warp agrees): flag it, give the copy one more

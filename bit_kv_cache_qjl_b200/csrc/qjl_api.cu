@@ -99,8 +99,28 @@ float bf16_to_float(uint16_t b) {
   return f;
 }
 
+// Fault injection on the host: with QJL_FAIL_ALLOC_AFTER=k in the environment,
+// the projection's device allocations after the first k (process-wide) report
+// failure without calling cudaMalloc, so tests can drive the out-of-memory path
+// of qjl_make_projection without exhausting a GPU.
+bool injected_alloc_failure() {
+  static const long limit = [] {
+    const char* v = getenv("QJL_FAIL_ALLOC_AFTER");
+    return v ? atol(v) : -1L;
+  }();
+  static std::mutex mu;
+  static long count = 0;
+  if (limit < 0) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  return count++ >= limit;
+}
+
 template <class T>
 qjl_status dev_upload(T** dst, const T* src, size_t count) {
+  if (injected_alloc_failure()) {
+    *dst = nullptr;
+    return qjl_set_error(QJL_ERR_OOM, "cudaMalloc failed for projection parameters (injected by QJL_FAIL_ALLOC_AFTER)");
+  }
   if (cudaMalloc((void**)dst, count * sizeof(T)) != cudaSuccess) {
     cudaGetLastError();
     *dst = nullptr;

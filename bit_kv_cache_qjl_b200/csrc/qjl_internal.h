@@ -121,6 +121,15 @@ qjl_status launch_decode(const qjl_projection* P, const uint32_t* bits, const fl
                          int64_t groups, int64_t N, const float* sq, int J, float softmax_scale,
                          float* out, void* ws, size_t ws_bytes, cudaStream_t st);
 
+// Bits of the per-device error int (read by qjl_device_errors). Bits 1..32 mark
+// bounded waits that expired (each kernel's producer, drain, consumer and, in
+// the tcgen05 kernels, MMA, TMEM and norm-warp waits).
+enum : int {
+  QJL_DEVERR_WAITS = 63,   // bits 1, 2, 4, 8, 16, 32: a bounded wait expired
+  QJL_DEVERR_PAGE = 64,    // a paged-cache position or block-table entry was out of range and skipped
+  QJL_DEVERR_SELFTEST = 128  // qjl_selftest_bounded_wait's wait expired, as it should
+};
+
 // Per-device int the kernels set when a bounded wait expires (qjl_api.cu).
 // It is allocated on first use and never freed.
 int* qjl_error_flag(int device);

@@ -565,7 +565,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
                   bulk_g2s(snorm + (size_t)s * SK + (lo - n0), norms + prow, len4 * 4, &full[s]);
                 }
               } else if (pass == 0) {
-                atomicOr(err, 8);  // a bad page id: its tokens keep stale stage data
+                atomicOr(err, QJL_DEVERR_PAGE);  // a bad page id: its tokens keep stale stage data
               }
               lo = hi;
             }

@@ -357,6 +357,28 @@ qjl_status qjl_kivi_key_scores(const uint32_t* codes, const uint16_t* scale, con
                                int64_t groups, int64_t N, int d, const float* q, int q_per_group,
                                float* scores, void* stream);
 
+/*
+ * Device-side errors. Kernels never trap. A bounded wait that expires (4 s of
+ * wall time), or a paged-cache entry that is out of range, sets a bit in a
+ * per-device int and the kernel winds down. The bits are:
+ *   1, 2, 4, 8, 16, 32  a bounded wait expired (1: a producer's wait for a
+ *        free stage; 2: a final wait for a CTA's own copies; 4: a consumer's
+ *        wait for a full stage; 8, 16, 32: the tcgen05 kernels' MMA-completion,
+ *        TMEM and norm-warp waits)
+ *   64   a paged-cache position or block-table entry was out of range (skipped)
+ *   128  qjl_selftest_bounded_wait's wait expired (as it should)
+ * qjl_device_errors synchronises `device`, stores the int in *flags and, if
+ * `clear` is nonzero, zeroes it. It returns QJL_ERR_DEVICE when any bit was
+ * set, else QJL_OK.
+ */
+qjl_status qjl_device_errors(int device, int clear, int* flags);
+
+/* Launch (asynchronously, on the legacy default stream) one thread that
+ * waits on a barrier nothing completes, bounded by limit_ns (1..1e9). When
+ * the limit passes it sets bit 128 and returns. Tests use it to check the
+ * expiry path without hanging the GPU. */
+qjl_status qjl_selftest_bounded_wait(int device, uint64_t limit_ns);
+
 /* Static text for a status code. */
 const char* qjl_status_string(qjl_status s);
 
