@@ -456,12 +456,13 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
   int64_t t1 = min(N, 16 * (min(te, (gi + 1) * plan.ntg) - gi * plan.ntg));
   if (PAGED) t1 = min(t1, min(max((int64_t)__ldg(pr.seq_lens + gi), (int64_t)0), N));
   const int64_t nst = t1 > t0 ? (t1 - t0 + kDsStage - 1) / kDsStage : 0;
-  build_tables_cls<W>(sq + gi * (int64_t)(32 * W), est_scale, s_inv, s_mul, s_qsum, Btab, kDsConsumers, 1);
+  build_tables_dig<W>(sq + gi * (int64_t)(32 * W), 1, 1, true, est_scale, s_inv, s_mul, s_qsum, Btab, kDsConsumers,
+                      1);
   uint2 breg[W];
 #pragma unroll
   for (int mu = 0; mu < W; ++mu) breg[mu] = Btab[mu * 32 + lane];
-  const float xmul = s_mul[0] * 0.03125f * logit_scale * 1.4426950408889634f;  // to log2-domain logits
-  const int qs32 = 32 * s_qsum[0];
+  const float xmul = s_mul[0] * logit_scale * 1.4426950408889634f;  // to log2-domain logits
+  const uint32_t qsum = (uint32_t)s_qsum[0];
   const int gq = lane >> 2, q = lane & 3;
   // value accumulation: lane = 8 tg + cs takes channels c0 = cs PL .. c0 + PL - 1 of the tokens
   // of group tg. At step j a warp covers four consecutive rows 4 (j & 3) + tg of its tile j / 4,
@@ -505,46 +506,43 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
         w1[t2][2 * kk] = b.x; w1[t2][2 * kk + 1] = b.y;
       }
     }
+    // shift-window sign sums (build_tables_dig): the A fragments are the words shifted right by
+    // s = 0..7, unmasked; both B column halves carry the query's four digits
     int accm[KT][4];
 #pragma unroll
     for (int p = 0; p < W / 8; ++p) {
 #pragma unroll
-      for (int sh = 0; sh < 2; ++sh) {
+      for (int sh = 0; sh < 8; ++sh) {
+        const uint2 bb = breg[8 * p + sh];
 #pragma unroll
-        for (int Ji = 0; Ji < 4; ++Ji) {
-          const uint32_t M = 0x01010101u << (2 * Ji);
-          const uint2 bb = breg[8 * p + 2 * Ji + sh];
-#pragma unroll
-          for (int t2 = 0; t2 < KT; ++t2) {
-            // the odd bit of each pair straight from the word (weight 2 * 4^Ji; B holds Q / 2)
-            const uint32_t Ms = M << sh;
-            const uint32_t a0 = w0[t2][2 * p] & Ms, a1 = w1[t2][2 * p] & Ms;
-            const uint32_t a2 = w0[t2][2 * p + 1] & Ms, a3 = w1[t2][2 * p + 1] & Ms;
-            if (p == 0 && sh == 0 && Ji == 0) mma_u8s8_zero(accm[t2], a0, a1, a2, a3, bb.x, bb.y);
-            else mma_u8s8_acc(accm[t2], a0, a1, a2, a3, bb.x, bb.y);
-          }
+        for (int t2 = 0; t2 < KT; ++t2) {
+          const uint32_t a0 = w0[t2][2 * p] >> sh, a1 = w1[t2][2 * p] >> sh;
+          const uint32_t a2 = w0[t2][2 * p + 1] >> sh, a3 = w1[t2][2 * p + 1] >> sh;
+          if (p == 0 && sh == 0) mma_u8s8_zero(accm[t2], a0, a1, a2, a3, bb.x, bb.y);
+          else mma_u8s8_acc(accm[t2], a0, a1, a2, a3, bb.x, bb.y);
         }
       }
     }
-    // lane q of quad gq ends with tile t2 = q, rows gq (r = 0) and gq + 8 (r = 1)
-    const int sft = 2 * (3 - q);
+    // lane (gq, q = 2 half + par) holds digits (2 par, 2 par + 1) of rows gq and gq + 8. The pair
+    // (q, q ^ 1) completes row gq + 8 par of tile 2k + half: x[k], k = 0, 1.
+    const int par = q & 1, half = q >> 1;
+    const uint32_t hm = par ? 65536u : 1u;
     float x[2];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      int mine = 0;
+    for (int k = 0; k < 2; ++k) {
+      int cc[4];
 #pragma unroll
-      for (int t2 = 0; t2 < KT; ++t2) {
-        int v = (accm[t2][2 * r] * 256 + accm[t2][2 * r + 1]) << sft;
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        if (t2 == q) mine = v;
-      }
-      const int row = (warp + q * kDsConsumers) * 16 + gq + 8 * r;
+      for (int j = 0; j < 4; ++j) cc[j] = half ? accm[2 * k + 1][j] : accm[2 * k][j];
+      const uint32_t P0 = (uint32_t)cc[0] * hm + (uint32_t)cc[1] * (hm << 8);
+      const uint32_t P1 = (uint32_t)cc[2] * hm + (uint32_t)cc[3] * (hm << 8);
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, par ? P0 : P1, 1);
+      const uint32_t tot = (par ? P1 : P0) + recv;
+      const int row = (warp + (2 * k + half) * kDsConsumers) * 16 + gq + 8 * par;
       if (row < cnt) {
         const float nrm = nb_norm ? snorm[row] : __ldg(norms + row0 + row);
-        x[r] = xmul * nrm * (float)(mine - qs32);
+        x[k] = xmul * nrm * (float)(int)(2u * tot - qsum);
       } else {
-        x[r] = -INFINITY;
+        x[k] = -INFINITY;
       }
     }
     // ---- online softmax over the warp's 64 tokens
@@ -561,14 +559,15 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
       for (int c = 0; c < PL; ++c) acc[c] *= corr;
       const float p0 = exp2f(x[0] - mn), p1 = exp2f(x[1] - mn);
       l_lane += p0 + p1;
-      // ---- p * v_hat: the token at (tile t2, row) has its p in lane 4 (row % 8) + t2, register row / 8
+      // ---- p * v_hat: the token at (tile t2, row) has its p in lane 4 (row % 8) + 2 (t2 % 2) + row / 8,
+      // register t2 / 2
       if (cnt == kDsStage && nb_codes && nb_scale && nb_zero) {
         // whole stage in shared memory: no per-token bounds or source selection
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int t2 = j >> 2, row = 4 * (j & 3) + tg;
           const int tok = (warp + t2 * kDsConsumers) * 16 + row;
-          const float pt = __shfl_sync(0xffffffffu, (j & 3) < 2 ? p0 : p1, 4 * (row & 7) + t2);
+          const float pt = __shfl_sync(0xffffffffu, (t2 >> 1) ? p1 : p0, 4 * (row & 7) + 2 * (t2 & 1) + (row >> 3));
           pv_accum<PL>(scodes + tok * CW + cwi, c0, sscale[tok * GW + grp], szero[tok * GW + grp], pt, acc, accz);
         }
       } else {
@@ -576,7 +575,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
         for (int j = 0; j < 16; ++j) {
           const int t2 = j >> 2, row = 4 * (j & 3) + tg;
           const int tok = (warp + t2 * kDsConsumers) * 16 + row;
-          const float pt = __shfl_sync(0xffffffffu, (j & 3) < 2 ? p0 : p1, 4 * (row & 7) + t2);
+          const float pt = __shfl_sync(0xffffffffu, (t2 >> 1) ? p1 : p0, 4 * (row & 7) + 2 * (t2 & 1) + (row >> 3));
           if (tok >= cnt) continue;
           uint32_t cwd[PL < 16 ? 1 : PL / 16];
 #pragma unroll
