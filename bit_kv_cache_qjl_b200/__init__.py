@@ -24,7 +24,8 @@ from ._lib import Options, lib
 __all__ = ["Projection", "QJLError", "quantize_keys", "project_queries", "scores",
            "quantize_values_2bit", "decode_attention", "decode_workspace_bytes", "PagedCache", "append_keys",
            "append_values_2bit", "scores_paged", "decode_attention_paged", "decode_paged_workspace_bytes",
-           "kivi_quantize_keys_2bit", "kivi_key_scores", "device_errors", "lib", "KINDS"]
+           "kivi_quantize_keys_2bit", "kivi_key_scores", "device_errors", "prefill_attention", "lib",
+           "KINDS"]
 
 KINDS = {"dense": 0, "dfqjl": 1, "pfqjl": 2}
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
@@ -285,3 +286,16 @@ def device_errors(device=0, clear=True):
     flags = ctypes.c_int(0)
     lib().qjl_device_errors(int(device), int(bool(clear)), ctypes.byref(flags))
     return flags.value
+
+
+def prefill_attention(proj, bits, norms, codes, scale, zero, sq, softmax_scale, out=None, stream=None):
+    """Causal prefill: bits [G, L, m/32], norms [G, L], codes/scale/zero per token, sq [G, L, m] -> out [G, L, d]."""
+    for t, nm in ((bits, "bits"), (norms, "norms"), (codes, "codes"), (scale, "scale"), (zero, "zero"), (sq, "sq")):
+        _cuda(t, nm)
+    G, L = norms.shape
+    if out is None:
+        out = torch.empty((G, L, proj.d), dtype=torch.float32, device=norms.device)
+    _check(lib().qjl_prefill_attention(proj.handle, _ptr(bits), _ptr(norms), _ptr(codes), _ptr(scale), _ptr(zero), G, L,
+                                       _ptr(sq), float(softmax_scale), _ptr(out), _stream(stream)),
+           "qjl_prefill_attention")
+    return out

@@ -50,6 +50,8 @@ SIGNATURES = {
                                     c_void_p]),
     "qjl_device_errors": (c_int, [c_int, c_int, ctypes.POINTER(c_int)]),
     "qjl_selftest_bounded_wait": (c_int, [c_int, c_uint64]),
+    "qjl_prefill_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64,
+                                      c_void_p, c_float, c_void_p, c_void_p]),
     "qjl_status_string": (ctypes.c_char_p, [c_int]),
     "qjl_last_error_message": (ctypes.c_char_p, []),
     "qjl_version": (ctypes.c_char_p, []),

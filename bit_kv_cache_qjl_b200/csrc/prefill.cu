@@ -1,0 +1,285 @@
+// Causal prefill attention over sketched keys and 2-bit values.
+//
+// At prefill every position is a query that attends to the keys at or before
+// it. The scores are the QJL estimator (QJL abstract, "Majid Daliri" page)
+// over the packed sign bits, the values the KIVI per-token 2-bit codes (KIVI
+// abstract, "Vladimir Braverman" page):
+//   out[g][i] = sum_{j <= i} softmax_j(scale * est(q_i, k_j)) * v_hat[g][j].
+//
+// One warp (one CTA) per 16 consecutive queries of a key head. The warp walks
+// the key axis in 16-key steps up to its diagonal:
+//   * scores: shift-window sign sums (build_tables_dig) on the u8 x s8
+//     mma.sync, two queries per n8 column tile, so 8 column tiles cover the
+//     warp's 16 queries; then the causal and length masks;
+//   * an online base-2 softmax, with each query's running max and sum kept
+//     identical in every lane;
+//   * P . V on the fp16 tensor-core path (mma.sync m16n8k16, fp32
+//     accumulate). P goes through shared memory to ldmatrix as the A
+//     fragment; the step's 16 values are dequantised to fp16
+//     (code * scale + zero) into shared memory and read with ldmatrix.trans
+//     as the B fragments of 16 channel tiles.
+// P and v_hat are rounded to binary16 (relative 2^-11 each); the sums run in
+// fp32. Key data is re-read by every later query tile of the head, so it is
+// read straight from global memory and served by L2.
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "qjl_internal.h"
+#include "sign_mma.cuh"
+
+namespace {
+
+using namespace qjl_sign;
+
+constexpr int kQ = 16;          // queries per warp (CTA)
+constexpr int kWs = 8;          // sign words per key (m = 256)
+constexpr int kD = 128;         // head dim
+constexpr int kNT = kQ / 2;     // digit column tiles
+constexpr int kPS = 24;         // P tile row stride (halves): 48 bytes, 16-byte aligned rows
+constexpr int kVS = kD + 8;     // V tile row stride (halves): 272 bytes
+
+struct PrefillSmem {
+  uint2 btab[kNT * kWs * 32];
+  float s_inv[64], s_mul[64];
+  int s_qsum[64];
+  __align__(16) __half P[kQ * kPS];
+  __align__(16) __half V[16 * kVS];
+};
+
+__device__ __forceinline__ void ldm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+
+__device__ __forceinline__ void ldm_x2_trans(uint32_t (&r)[2], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__global__ void __launch_bounds__(32) prefill_kernel(const uint32_t* __restrict__ bits, const float* __restrict__ norms,
+                                                     const uint32_t* __restrict__ codes,
+                                                     const uint16_t* __restrict__ scale,
+                                                     const uint16_t* __restrict__ zero, const float* __restrict__ sq,
+                                                     int64_t G, int64_t L, float est_scale, float logit2,
+                                                     float* __restrict__ out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(smem_raw);
+  const int lane = threadIdx.x;
+  const int64_t nqt = (L + kQ - 1) / kQ;
+  // the heaviest query tiles (late in the sequence) first
+  const int64_t tile = (nqt - 1) - (int64_t)(blockIdx.x / G);
+  const int64_t g = (int64_t)(blockIdx.x % G);
+  const int64_t q0 = tile * kQ;
+  const int nq = (int)min((int64_t)kQ, L - q0);
+
+  build_tables_dig<kWs>(sq + (g * L + q0) * (32 * kWs), nq, kNT, false, est_scale, S.s_inv, S.s_mul, S.s_qsum,
+                        S.btab, 1, 0);
+
+  const int gq = lane >> 2, q = lane & 3, par = q & 1, half = q >> 1;
+  const uint32_t hm = par ? 65536u : 1u;
+  float o[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[n][j] = 0.f;
+  float m_run[kQ], l_run[kQ];
+#pragma unroll
+  for (int j = 0; j < kQ; ++j) {
+    m_run[j] = -INFINITY;
+    l_run[j] = 0.f;
+  }
+  const int64_t ktiles = q0 / 16 + 1;  // keys 0 .. q0 + 15 (the diagonal tile is the last)
+  for (int64_t kt = 0; kt < ktiles; ++kt) {
+    const int64_t k0 = kt * 16;
+    // ---- scores: rows g and g + 8 of the key tile, words 2q and 2q + 1
+    uint32_t w0[2] = {0u, 0u}, w1[2] = {0u, 0u};
+    if (k0 + gq < L) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(bits + (g * L + k0 + gq) * kWs + 2 * q));
+      w0[0] = v.x; w0[1] = v.y;
+    }
+    if (k0 + gq + 8 < L) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(bits + (g * L + k0 + gq + 8) * kWs + 2 * q));
+      w1[0] = v.x; w1[1] = v.y;
+    }
+    int acc[kNT][4];
+#pragma unroll
+    for (int sh = 0; sh < 8; ++sh) {
+      const uint32_t a0 = w0[0] >> sh, a1 = w1[0] >> sh, a2 = w0[1] >> sh, a3 = w1[1] >> sh;
+#pragma unroll
+      for (int ct = 0; ct < kNT; ++ct) {
+        const uint2 bb = S.btab[(ct * kWs + sh) * 32 + lane];
+        if (sh == 0) {
+          asm volatile(
+              "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+              "{%10,%10,%10,%10};\n"
+              : "=r"(acc[ct][0]), "=r"(acc[ct][1]), "=r"(acc[ct][2]), "=r"(acc[ct][3])
+              : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(bb.x), "r"(bb.y), "r"(0));
+        } else {
+          mma_u8s8(acc[ct], a0, a1, a2, a3, bb.x, bb.y);
+        }
+      }
+    }
+    // lane (gq, q) completes key kr = gq + 8 par for query 2 ct + half of each column tile
+    const int kr = gq + 8 * par;
+    const int64_t kg = k0 + kr;
+    const float nrm = kg < L ? __ldg(norms + g * L + kg) : 0.f;
+    float xv[kNT];
+#pragma unroll
+    for (int ct = 0; ct < kNT; ++ct) {
+      const uint32_t P0 = (uint32_t)acc[ct][0] * hm + (uint32_t)acc[ct][1] * (hm << 8);
+      const uint32_t P1 = (uint32_t)acc[ct][2] * hm + (uint32_t)acc[ct][3] * (hm << 8);
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, par ? P0 : P1, 1);
+      const uint32_t tot = (par ? P1 : P0) + recv;
+      const int jq = 2 * ct + half;
+      const bool ok = jq < nq && kg < L && kg <= q0 + jq;
+      xv[ct] = ok ? logit2 * S.s_mul[jq] * nrm * (float)(int)(2u * tot - (uint32_t)S.s_qsum[jq]) : -INFINITY;
+    }
+    // ---- online softmax: the step's max and sum per query, over the 16 lanes of the query's half
+    float tmax[kQ], corr[kQ], mnew[kQ];
+#pragma unroll
+    for (int ct = 0; ct < kNT; ++ct) {
+      float v = xv[ct];
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+      const float other = __shfl_xor_sync(0xffffffffu, v, 2);
+      // static register indices: query 2 ct is this lane's when half == 0
+      tmax[2 * ct] = half ? other : v;
+      tmax[2 * ct + 1] = half ? v : other;
+    }
+#pragma unroll
+    for (int j = 0; j < kQ; ++j) {
+      mnew[j] = fmaxf(m_run[j], tmax[j]);
+      corr[j] = mnew[j] == -INFINITY ? 1.f : exp2f(m_run[j] - mnew[j]);
+      m_run[j] = mnew[j];
+    }
+    float pv[kNT];
+#pragma unroll
+    for (int ct = 0; ct < kNT; ++ct) {
+      const float mj = half ? mnew[2 * ct + 1] : mnew[2 * ct];
+      pv[ct] = (xv[ct] == -INFINITY) ? 0.f : exp2f(xv[ct] - mj);
+      float sv = pv[ct];
+      sv += __shfl_xor_sync(0xffffffffu, sv, 1);
+      sv += __shfl_xor_sync(0xffffffffu, sv, 4);
+      sv += __shfl_xor_sync(0xffffffffu, sv, 8);
+      sv += __shfl_xor_sync(0xffffffffu, sv, 16);
+      const float so = __shfl_xor_sync(0xffffffffu, sv, 2);
+      l_run[2 * ct] = l_run[2 * ct] * corr[2 * ct] + (half ? so : sv);
+      l_run[2 * ct + 1] = l_run[2 * ct + 1] * corr[2 * ct + 1] + (half ? sv : so);
+    }
+    // rescale the accumulator rows (queries gq and gq + 8)
+    {
+      float c0 = corr[0], c1 = corr[8];
+#pragma unroll
+      for (int j = 1; j < 8; ++j) if (j == gq) { c0 = corr[j]; c1 = corr[j + 8]; }
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        o[n][0] *= c0; o[n][1] *= c0;
+        o[n][2] *= c1; o[n][3] *= c1;
+      }
+    }
+    // ---- P (fp16) into shared memory as [query][key]
+    __syncwarp();
+#pragma unroll
+    for (int ct = 0; ct < kNT; ++ct) S.P[(2 * ct + half) * kPS + kr] = __float2half_rn(pv[ct]);
+    // ---- v_hat (fp16) into shared memory as [key][channel]: lane takes key lane / 2, channels 64 (lane % 2) ..
+    {
+      const int kk = lane >> 1, cb = 64 * (lane & 1);
+      const int64_t kgv = k0 + kk;
+      __half2* vrow = reinterpret_cast<__half2*>(S.V + kk * kVS + cb);
+      if (kgv < L) {
+        const uint4 cw = __ldg(reinterpret_cast<const uint4*>(codes + (g * L + kgv) * (kD / 16) + cb / 16));
+        const uint32_t ws[4] = {cw.x, cw.y, cw.z, cw.w};
+        const float s0 = __half2float(__ushort_as_half(__ldg(scale + (g * L + kgv) * (kD / 32) + cb / 32)));
+        const float z0 = __half2float(__ushort_as_half(__ldg(zero + (g * L + kgv) * (kD / 32) + cb / 32)));
+        const float s1 = __half2float(__ushort_as_half(__ldg(scale + (g * L + kgv) * (kD / 32) + cb / 32 + 1)));
+        const float z1 = __half2float(__ushort_as_half(__ldg(zero + (g * L + kgv) * (kD / 32) + cb / 32 + 1)));
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float s = w < 2 ? s0 : s1, z = w < 2 ? z0 : z1;
+#pragma unroll
+          for (int c = 0; c < 16; c += 2) {
+            const float v0 = fmaf((float)((ws[w] >> (2 * c)) & 3u), s, z);
+            const float v1 = fmaf((float)((ws[w] >> (2 * c + 2)) & 3u), s, z);
+            vrow[(16 * w + c) / 2] = __floats2half2_rn(v0, v1);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) vrow[c] = __floats2half2_rn(0.f, 0.f);
+      }
+    }
+    __syncwarp();
+    // ---- o += P . v_hat
+    uint32_t afr[4];
+    ldm_x4(afr, S.P + (lane & 15) * kPS + 8 * (lane >> 4));
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      uint32_t bfr[2];
+      ldm_x2_trans(bfr, S.V + (lane & 15) * kVS + 8 * n);
+      mma_f16(o[n], afr, bfr);
+    }
+    __syncwarp();
+  }
+  // ---- normalise and store rows gq and gq + 8
+  float l0 = l_run[0], l1 = l_run[8];
+#pragma unroll
+  for (int j = 1; j < 8; ++j) if (j == gq) { l0 = l_run[j]; l1 = l_run[j + 8]; }
+  const float i0 = 1.f / l0, i1 = 1.f / l1;
+#pragma unroll
+  for (int n = 0; n < 16; ++n) {
+    const int ch = 8 * n + 2 * q;
+    if (gq < nq) {
+      float2* p = reinterpret_cast<float2*>(out + (g * L + q0 + gq) * kD + ch);
+      *p = make_float2(o[n][0] * i0, o[n][1] * i0);
+    }
+    if (gq + 8 < nq) {
+      float2* p = reinterpret_cast<float2*>(out + (g * L + q0 + gq + 8) * kD + ch);
+      *p = make_float2(o[n][2] * i1, o[n][3] * i1);
+    }
+  }
+}
+
+}  // namespace
+
+extern "C" qjl_status qjl_prefill_attention(const qjl_projection* P, const uint32_t* bits, const float* norms,
+                                            const uint32_t* codes, const uint16_t* scale, const uint16_t* zero,
+                                            int64_t groups, int64_t L, const float* sq, float softmax_scale,
+                                            float* out, void* stream) {
+  qjl_set_error(QJL_OK, "");
+  if (!P) return qjl_set_error(QJL_ERR_INVALID_ARG, "projection is NULL");
+  if (groups < 0 || L < 0 || groups > (1 << 20) || L > (1 << 24))
+    return qjl_set_error(QJL_ERR_INVALID_ARG, "groups/L out of range");
+  if (!isfinite(softmax_scale)) return qjl_set_error(QJL_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (P->d != kD || P->m != 32 * kWs)
+    return qjl_set_error(QJL_ERR_UNSUPPORTED, "prefill attention supports d = 128 and m = 256");
+  if (groups == 0 || L == 0) return QJL_OK;
+  if (!bits || !norms || !codes || !scale || !zero || !sq || !out) return qjl_set_error(QJL_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(bits) || !aligned16(codes) || !aligned16(sq) || !aligned16(out) || ((uintptr_t)norms & 3u) ||
+      ((uintptr_t)scale & 1u) || ((uintptr_t)zero & 1u))
+    return qjl_set_error(QJL_ERR_INVALID_ARG, "bits, codes, sq and out must be 16-byte aligned; norms, scale, zero naturally");
+  const int64_t nqt = (L + kQ - 1) / kQ;
+  if (groups * nqt > ((int64_t)1 << 31) - 1) return qjl_set_error(QJL_ERR_UNSUPPORTED, "too many query tiles");
+  DeviceGuard gd(P->device);
+  if (!gd.ok) return qjl_set_error(QJL_ERR_CUDA, "cannot select the projection's device");
+  const size_t smem = sizeof(PrefillSmem);
+  if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return qjl_check_launch("prefill_kernel smem attribute");
+  prefill_kernel<<<(unsigned)(groups * nqt), 32, smem, (cudaStream_t)stream>>>(
+      bits, norms, codes, scale, zero, sq, groups, L, P->est_scale, softmax_scale * 1.4426950408889634f, out);
+  return qjl_check_launch("prefill_kernel");
+}

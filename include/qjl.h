@@ -328,6 +328,25 @@ qjl_status qjl_decode_attention_paged(const qjl_projection* proj, const uint32_t
                                       float* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Causal prefill attention over a sketched key cache and 2-bit values (QJL
+ * abstract for the scores; KIVI abstract for the values). Every position is a
+ * query that attends to the keys at or before it:
+ *   out[g][i][:] = sum_{j <= i} softmax_j(softmax_scale * est[g][i][j]) * v_hat[g][j][:]
+ * with est as in qjl_scores (sq[g][i] against key j) and v_hat = code * scale
+ * + zero. P and v_hat enter the tensor cores as binary16, and the sums run in
+ * fp32.
+ *   bits/norms/codes/scale/zero  the cache of L tokens per group, as in
+ *                                qjl_decode_attention.
+ *   sq    [groups][L][m] fp32: the projected query of every position.
+ *   out   [groups][L][d] fp32.
+ * Supports d = 128 and m = 256. bits, codes, sq and out must be 16-byte aligned.
+ */
+qjl_status qjl_prefill_attention(const qjl_projection* proj, const uint32_t* bits,
+                                 const float* norms, const uint32_t* codes, const uint16_t* scale,
+                                 const uint16_t* zero, int64_t groups, int64_t L, const float* sq,
+                                 float softmax_scale, float* out, void* stream);
+
+/*
  * KIVI per-channel 2-bit keys: the like-for-like baseline of the QJL sketch on
  * the same shapes. The KIVI abstract ("KIVI: A Tuning-Free Asymmetric 2bit
  * Quantization for KV Cache", "Vladimir Braverman" page) quantises keys per

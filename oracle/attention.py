@@ -24,3 +24,17 @@ def decode_attention(est, vhat, softmax_scale):
     """est [G][J][N] estimated scores, vhat [G][N][d] -> out [G][J][d] (fp64)."""
     p = softmax(np.asarray(est, dtype=np.float64) * softmax_scale, axis=-1)
     return np.einsum("gjn,gnd->gjd", p, np.asarray(vhat, dtype=np.float64))
+
+
+def prefill_attention(est, vhat, softmax_scale):
+    """Causal prefill: est [G][L][L] (query i, key j) and vhat [G][L][d] -> out [G][L][d] (fp64).
+
+    Query i attends to keys 0..i: the scores of later keys are masked out before
+    the softmax. This is the many-query form of decode_attention.
+    """
+    est = np.asarray(est, dtype=np.float64)
+    G, L, _ = est.shape
+    mask = np.tril(np.ones((L, L), dtype=bool))
+    x = np.where(mask[None], est * softmax_scale, -np.inf)
+    p = softmax(x, axis=-1)
+    return np.einsum("gij,gjd->gid", p, np.asarray(vhat, dtype=np.float64)), p
