@@ -249,6 +249,17 @@ def profile_case(case, n):
     elif case == "values":
         v = wl.normal((n, D), 506, dev, torch.bfloat16)
         run = lambda: qjl.quantize_values_2bit(v)
+    elif case == "prefill":
+        # 8 heads x 4096 tokens of the prefill workload (n is ignored)
+        Gp, Lp = 8, 4096
+        P = qjl.Projection(2, D, M, "dense")
+        keys, vals = wl.decode_kv(dev, B=1, H=Gp, N=Lp, d=D)
+        bits, norms = qjl.quantize_keys(P, keys.reshape(-1, D))
+        codes, sc, zr = qjl.quantize_values_2bit(vals.reshape(-1, D))
+        sq = qjl.project_queries(P, wl.normal((Gp * Lp, D), 407, dev))
+        run = lambda: qjl.prefill_attention(P, bits.view(Gp, Lp, -1), norms.view(Gp, Lp), codes.view(Gp, Lp, -1),
+                                            sc.view(Gp, Lp, -1), zr.view(Gp, Lp, -1), sq.view(Gp, Lp, M),
+                                            1 / math.sqrt(D))
     else:
         P = qjl.Projection(5, D, M, "dfqjl")
         G = max(1, n // 16384)
@@ -437,6 +448,37 @@ def build_workload(name, dev, qjl, wl, torch):
                  desc="%s: D-FQJL sigma_rel 0.5, B=32, 32 heads, N=16384 in 256-token pages (shuffled block "
                       "table), d=128, m=256; append 1 key + 2-bit value per head, project queries, fused paged "
                       "decode" % name)
+    elif name == "prefill_causal":
+        # causal prefill of 32 heads x 4096 tokens (d=128, m=256 dense): sketch the keys, quantize the values,
+        # project every position's query, then the fused causal attention; units are query-key pairs
+        Gp, Lp, m = 32, 4096, 256
+        P = qjl.Projection(2, D, m, "dense", s_bf16=True)
+        keys, vals = wl.decode_kv(dev, B=1, H=Gp, N=Lp, d=D)
+        keys, vals = keys.reshape(-1, D), vals.reshape(-1, D)
+        q = wl.normal((Gp * Lp, D), 407, dev)
+        bits = torch.empty((Gp * Lp, m // 32), dtype=torch.int32, device=dev)
+        norms = torch.empty((Gp * Lp,), dtype=torch.float32, device=dev)
+        codes = torch.empty((Gp * Lp, D // 16), dtype=torch.int32, device=dev)
+        sc = torch.empty((Gp * Lp, D // 32), dtype=torch.float16, device=dev)
+        zr = torch.empty((Gp * Lp, D // 32), dtype=torch.float16, device=dev)
+        sq = torch.empty((Gp * Lp, m), dtype=torch.float32, device=dev)
+        out = torch.empty((Gp, Lp, D), dtype=torch.float32, device=dev)
+        pairs = Gp * Lp * (Lp + 1) // 2
+        stages = [
+            Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), Gp * Lp,
+                  2 * D + m // 8 + 4, 2 * D * m, "dense_tc_kernel", "dense_tc.cu"),
+            Stage("quantize_values", lambda: qjl.quantize_values_2bit(vals, codes=codes, scale=sc, zero=zr), Gp * Lp,
+                  2 * D + D // 4 + D // 8),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), Gp * Lp, 4 * D + 4 * m),
+            # work per (query, key) pair: 2 d flops of P.V plus 2 m of sign-dot multiply-adds
+            Stage("prefill_attention", lambda: qjl.prefill_attention(
+                P, bits.view(Gp, Lp, -1), norms.view(Gp, Lp), codes.view(Gp, Lp, -1), sc.view(Gp, Lp, -1),
+                zr.view(Gp, Lp, -1), sq.view(Gp, Lp, m), 1.0 / math.sqrt(D), out=out), pairs, 0, 2 * D + 2 * m,
+                "prefill_kernel", "prefill.cu", "tensor"),
+        ]
+        W.update(units=pairs, unit="query-key pairs/s", inputs=[keys, vals, q], outputs=[out], dtype="bf16",
+                 desc="%s: 32 heads x 4096 tokens, d=128, m=256 dense bf16 S; quantize keys and 2-bit values, project "
+                      "all queries, fused causal attention" % name)
     elif name == "kivi_keys_decode":
         # the KIVI per-channel 2-bit key baseline on the decode_llama7b keys: quantize every key per
         # channel (32-token blocks) and score one query per head; "accuracy" compares its scores and the
@@ -496,11 +538,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=["decode_llama7b", "gqa_decode", "dense_1head", "pfqjl_bulk_m256", "pfqjl_bulk_m1024",
-                             "dfqjl_decode", "paged_decode", "kivi_keys_decode"])
+                             "dfqjl_decode", "paged_decode", "kivi_keys_decode", "prefill_causal"])
     ap.add_argument("--ref-sample", type=int, default=4096)
     ap.add_argument("--cpu-sample", type=int, default=1 << 21)
     ap.add_argument("--profile-case", default=None,
-                    choices=["quantize", "scores", "fqjl", "fqjl1024", "dfqjl", "values", "decode"],
+                    choices=["quantize", "scores", "fqjl", "fqjl1024", "dfqjl", "values", "decode", "prefill"],
                     help="run one small case of a single kernel (3 launches after 2 warm-ups) for ncu")
     ap.add_argument("--profile-keys", type=int, default=1 << 20)
     ap.add_argument("--e2e-steps", type=int, default=5)

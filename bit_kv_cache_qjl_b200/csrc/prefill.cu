@@ -17,7 +17,10 @@
 //     accumulate). P goes through shared memory to ldmatrix as the A
 //     fragment; the step's 16 values are dequantised to fp16
 //     (code * scale + zero) into shared memory and read with ldmatrix.trans
-//     as the B fragments of 16 channel tiles.
+//     as the B fragments of 16 channel tiles. Each step's key data is loaded
+//     one step ahead. (Dequantising the values once into an fp16 workspace
+//     and streaming tiles of it with cp.async measured slower: 3.35 against
+//     3.01 ms for 32 heads x 4096 tokens.)
 // P and v_hat are rounded to binary16 (relative 2^-11 each); the sums run in
 // fp32. Key data is re-read by every later query tile of the head, so it is
 // read straight from global memory and served by L2.
@@ -95,25 +98,46 @@ __global__ void __launch_bounds__(32) prefill_kernel(const uint32_t* __restrict_
   for (int n = 0; n < 16; ++n)
 #pragma unroll
     for (int j = 0; j < 4; ++j) o[n][j] = 0.f;
-  float m_run[kQ], l_run[kQ];
+  float m_run[kQ], l_part[kNT];
 #pragma unroll
-  for (int j = 0; j < kQ; ++j) {
-    m_run[j] = -INFINITY;
-    l_run[j] = 0.f;
-  }
+  for (int j = 0; j < kQ; ++j) m_run[j] = -INFINITY;
+#pragma unroll
+  for (int ct = 0; ct < kNT; ++ct) l_part[ct] = 0.f;
   const int64_t ktiles = q0 / 16 + 1;  // keys 0 .. q0 + 15 (the diagonal tile is the last)
+  // the global data of a 16-key step, loaded one step ahead: this lane's sign words of key rows
+  // gq and gq + 8, the norm of its key row, and the codes, scales and zeros of its value slice
+  struct StepData {
+    uint2 wa, wb;
+    float nrm;
+    uint4 cw;
+    uint16_t s0, z0, s1, z1;
+  };
+  const int kr = gq + 8 * par;
+  const int kk = lane >> 1, cb = 64 * (lane & 1);
+  auto load_step = [&](int64_t k0, StepData& sd) {
+    sd.wa = k0 + gq < L ? __ldg(reinterpret_cast<const uint2*>(bits + (g * L + k0 + gq) * kWs + 2 * q)) : make_uint2(0, 0);
+    sd.wb = k0 + gq + 8 < L ? __ldg(reinterpret_cast<const uint2*>(bits + (g * L + k0 + gq + 8) * kWs + 2 * q))
+                            : make_uint2(0, 0);
+    sd.nrm = k0 + kr < L ? __ldg(norms + g * L + k0 + kr) : 0.f;
+    const int64_t kgv = k0 + kk;
+    if (kgv < L) {
+      sd.cw = __ldg(reinterpret_cast<const uint4*>(codes + (g * L + kgv) * (kD / 16) + cb / 16));
+      const int64_t gi = (g * L + kgv) * (kD / 32) + cb / 32;
+      sd.s0 = __ldg(scale + gi); sd.z0 = __ldg(zero + gi);
+      sd.s1 = __ldg(scale + gi + 1); sd.z1 = __ldg(zero + gi + 1);
+    } else {
+      // past the last token: zero values (P is 0 there)
+      sd.cw = make_uint4(0, 0, 0, 0);
+      sd.s0 = sd.z0 = sd.s1 = sd.z1 = 0;
+    }
+  };
+  StepData cur, nxt;
+  load_step(0, cur);
   for (int64_t kt = 0; kt < ktiles; ++kt) {
     const int64_t k0 = kt * 16;
+    if (kt + 1 < ktiles) load_step(k0 + 16, nxt);
     // ---- scores: rows g and g + 8 of the key tile, words 2q and 2q + 1
-    uint32_t w0[2] = {0u, 0u}, w1[2] = {0u, 0u};
-    if (k0 + gq < L) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(bits + (g * L + k0 + gq) * kWs + 2 * q));
-      w0[0] = v.x; w0[1] = v.y;
-    }
-    if (k0 + gq + 8 < L) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(bits + (g * L + k0 + gq + 8) * kWs + 2 * q));
-      w1[0] = v.x; w1[1] = v.y;
-    }
+    const uint32_t w0[2] = {cur.wa.x, cur.wa.y}, w1[2] = {cur.wb.x, cur.wb.y};
     int acc[kNT][4];
 #pragma unroll
     for (int sh = 0; sh < 8; ++sh) {
@@ -133,9 +157,8 @@ __global__ void __launch_bounds__(32) prefill_kernel(const uint32_t* __restrict_
       }
     }
     // lane (gq, q) completes key kr = gq + 8 par for query 2 ct + half of each column tile
-    const int kr = gq + 8 * par;
     const int64_t kg = k0 + kr;
-    const float nrm = kg < L ? __ldg(norms + g * L + kg) : 0.f;
+    const float nrm = cur.nrm;
     float xv[kNT];
 #pragma unroll
     for (int ct = 0; ct < kNT; ++ct) {
@@ -171,15 +194,9 @@ __global__ void __launch_bounds__(32) prefill_kernel(const uint32_t* __restrict_
 #pragma unroll
     for (int ct = 0; ct < kNT; ++ct) {
       const float mj = half ? mnew[2 * ct + 1] : mnew[2 * ct];
+      const float cj = half ? corr[2 * ct + 1] : corr[2 * ct];
       pv[ct] = (xv[ct] == -INFINITY) ? 0.f : exp2f(xv[ct] - mj);
-      float sv = pv[ct];
-      sv += __shfl_xor_sync(0xffffffffu, sv, 1);
-      sv += __shfl_xor_sync(0xffffffffu, sv, 4);
-      sv += __shfl_xor_sync(0xffffffffu, sv, 8);
-      sv += __shfl_xor_sync(0xffffffffu, sv, 16);
-      const float so = __shfl_xor_sync(0xffffffffu, sv, 2);
-      l_run[2 * ct] = l_run[2 * ct] * corr[2 * ct] + (half ? so : sv);
-      l_run[2 * ct + 1] = l_run[2 * ct + 1] * corr[2 * ct + 1] + (half ? sv : so);
+      l_part[ct] = l_part[ct] * cj + pv[ct];  // this lane's share of query 2 ct + half's sum
     }
     // rescale the accumulator rows (queries gq and gq + 8)
     {
@@ -197,30 +214,21 @@ __global__ void __launch_bounds__(32) prefill_kernel(const uint32_t* __restrict_
 #pragma unroll
     for (int ct = 0; ct < kNT; ++ct) S.P[(2 * ct + half) * kPS + kr] = __float2half_rn(pv[ct]);
     // ---- v_hat (fp16) into shared memory as [key][channel]: lane takes key lane / 2, channels 64 (lane % 2) ..
+    // The code comes out as float(2^23 | code) - 2^23, with no conversion instruction.
     {
-      const int kk = lane >> 1, cb = 64 * (lane & 1);
-      const int64_t kgv = k0 + kk;
       __half2* vrow = reinterpret_cast<__half2*>(S.V + kk * kVS + cb);
-      if (kgv < L) {
-        const uint4 cw = __ldg(reinterpret_cast<const uint4*>(codes + (g * L + kgv) * (kD / 16) + cb / 16));
-        const uint32_t ws[4] = {cw.x, cw.y, cw.z, cw.w};
-        const float s0 = __half2float(__ushort_as_half(__ldg(scale + (g * L + kgv) * (kD / 32) + cb / 32)));
-        const float z0 = __half2float(__ushort_as_half(__ldg(zero + (g * L + kgv) * (kD / 32) + cb / 32)));
-        const float s1 = __half2float(__ushort_as_half(__ldg(scale + (g * L + kgv) * (kD / 32) + cb / 32 + 1)));
-        const float z1 = __half2float(__ushort_as_half(__ldg(zero + (g * L + kgv) * (kD / 32) + cb / 32 + 1)));
+      const uint32_t ws[4] = {cur.cw.x, cur.cw.y, cur.cw.z, cur.cw.w};
+      const float s0 = __half2float(__ushort_as_half(cur.s0)), z0 = __half2float(__ushort_as_half(cur.z0));
+      const float s1 = __half2float(__ushort_as_half(cur.s1)), z1 = __half2float(__ushort_as_half(cur.z1));
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float s = w < 2 ? s0 : s1, z = w < 2 ? z0 : z1;
+      for (int w = 0; w < 4; ++w) {
+        const float sw = w < 2 ? s0 : s1, zw = w < 2 ? z0 : z1;
 #pragma unroll
-          for (int c = 0; c < 16; c += 2) {
-            const float v0 = fmaf((float)((ws[w] >> (2 * c)) & 3u), s, z);
-            const float v1 = fmaf((float)((ws[w] >> (2 * c + 2)) & 3u), s, z);
-            vrow[(16 * w + c) / 2] = __floats2half2_rn(v0, v1);
-          }
+        for (int c = 0; c < 16; c += 2) {
+          const float c0 = __uint_as_float(0x4B000000u | ((ws[w] >> (2 * c)) & 3u)) - 8388608.f;
+          const float c1 = __uint_as_float(0x4B000000u | ((ws[w] >> (2 * c + 2)) & 3u)) - 8388608.f;
+          vrow[(16 * w + c) / 2] = __floats2half2_rn(fmaf(c0, sw, zw), fmaf(c1, sw, zw));
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) vrow[c] = __floats2half2_rn(0.f, 0.f);
       }
     }
     __syncwarp();
@@ -234,6 +242,20 @@ __global__ void __launch_bounds__(32) prefill_kernel(const uint32_t* __restrict_
       mma_f16(o[n], afr, bfr);
     }
     __syncwarp();
+    cur = nxt;
+  }
+  // ---- each query's sum: its 16 key lanes (lane bits 0, 2, 3, 4), then the other half's queries
+  float l_run[kQ];
+#pragma unroll
+  for (int ct = 0; ct < kNT; ++ct) {
+    float v = l_part[ct];
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 16);
+    const float other = __shfl_xor_sync(0xffffffffu, v, 2);
+    l_run[2 * ct] = half ? other : v;
+    l_run[2 * ct + 1] = half ? v : other;
   }
   // ---- normalise and store rows gq and gq + 8
   float l0 = l_run[0], l1 = l_run[8];

@@ -16,7 +16,9 @@ pytestmark = pytest.mark.gpu
                                              ("dense", 128, 512, 37, dict(s_bf16=True)),
                                              ("pfqjl", 256, 1024, 64, {}),
                                              ("dfqjl", 128, 256, 33, {}),
-                                             ("pfqjl", 128, 256, 5, dict(dg_outer=True))])
+                                             ("pfqjl", 128, 256, 5, dict(dg_outer=True)),
+                                             # many queries (a prefill): the warp-per-row kernel
+                                             ("dense", 128, 256, 3000, dict(s_bf16=True))])
 def test_project_queries(cuda_ok, kind, d, m, nq, kw):
     P = Projection(21, d, m, kind, **kw)
     q = wl.normal((nq, d), 55, "cuda")
