@@ -6,8 +6,10 @@
 // abstract, "Vladimir Braverman" page):
 //   out[g][i] = sum_{j <= i} softmax_j(scale * est(q_i, k_j)) * v_hat[g][j].
 //
-// One warp (one CTA) per 16 consecutive queries of a key head. The warp walks
-// the key axis in 16-key steps up to its diagonal:
+// One warp per 16 consecutive queries of a key head, four warps (64 queries)
+// per CTA. The warps walk the key axis in 16-key steps, each up to its own
+// diagonal; the CTA dequantises each step's value tile once for all four.
+// Per warp and step:
 //   * scores: shift-window sign sums (build_tables_dig) on the u8 x s8
 //     mma.sync, two queries per n8 column tile, so 8 column tiles cover the
 //     warp's 16 queries; then the causal and length masks;
@@ -16,9 +18,10 @@
 //   * P . V on the fp16 tensor-core path (mma.sync m16n8k16, fp32
 //     accumulate). P goes through shared memory to ldmatrix as the A
 //     fragment; the step's 16 values are dequantised to fp16
-//     (code * scale + zero) into shared memory and read with ldmatrix.trans
-//     as the B fragments of 16 channel tiles. Each step's key data is loaded
-//     one step ahead. (Dequantising the values once into an fp16 workspace
+//     (code * scale + zero) into a double-buffered shared tile, one code word
+//     per thread of the CTA, and read with ldmatrix.trans as the B fragments of
+//     16 channel tiles. Each step's key and value data is loaded one step
+//     ahead. (Dequantising the values once into an fp16 workspace
 //     and streaming tiles of it with cp.async measured slower: 3.35 against
 //     3.01 ms for 32 heads x 4096 tokens.)
 // P and v_hat are rounded to binary16 (relative 2^-11 each); the sums run in
@@ -44,12 +47,18 @@ constexpr int kNT = kQ / 2;     // digit column tiles
 constexpr int kPS = 24;         // P tile row stride (halves): 48 bytes, 16-byte aligned rows
 constexpr int kVS = kD + 8;     // V tile row stride (halves): 272 bytes
 
-struct PrefillSmem {
+constexpr int kWarps = 4;       // warps per CTA: 64 consecutive queries share each value tile
+
+struct WarpSmem {
   uint2 btab[kNT * kWs * 32];
   float s_inv[64], s_mul[64];
   int s_qsum[64];
   __align__(16) __half P[kQ * kPS];
-  __align__(16) __half V[16 * kVS];
+};
+
+struct PrefillSmem {
+  WarpSmem w[kWarps];
+  __align__(16) __half V[2][16 * kVS];  // the step's value tile, double-buffered, shared by the warps
 };
 
 __device__ __forceinline__ void ldm_x4(uint32_t (&r)[4], const void* p) {
@@ -72,24 +81,37 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], c
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-__global__ void __launch_bounds__(32) prefill_kernel(const uint32_t* __restrict__ bits, const float* __restrict__ norms,
-                                                     const uint32_t* __restrict__ codes,
-                                                     const uint16_t* __restrict__ scale,
-                                                     const uint16_t* __restrict__ zero, const float* __restrict__ sq,
-                                                     int64_t G, int64_t L, float est_scale, float logit2,
-                                                     float* __restrict__ out) {
+__global__ void __launch_bounds__(kWarps * 32) prefill_kernel(const uint32_t* __restrict__ bits,
+                                                              const float* __restrict__ norms,
+                                                              const uint32_t* __restrict__ codes,
+                                                              const uint16_t* __restrict__ scale,
+                                                              const uint16_t* __restrict__ zero,
+                                                              const float* __restrict__ sq, int64_t G, int64_t L,
+                                                              float est_scale, float logit2, float* __restrict__ out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(smem_raw);
-  const int lane = threadIdx.x;
-  const int64_t nqt = (L + kQ - 1) / kQ;
+  PrefillSmem& SM = *reinterpret_cast<PrefillSmem*>(smem_raw);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  WarpSmem& S = SM.w[warp];
+  constexpr int kCQ = kWarps * kQ;
+  const int64_t nqt = (L + kCQ - 1) / kCQ;
   // the heaviest query tiles (late in the sequence) first
   const int64_t tile = (nqt - 1) - (int64_t)(blockIdx.x / G);
   const int64_t g = (int64_t)(blockIdx.x % G);
-  const int64_t q0 = tile * kQ;
-  const int nq = (int)min((int64_t)kQ, L - q0);
+  const int64_t q0c = tile * kCQ;
+  const int64_t q0 = q0c + kQ * warp;                        // this warp's first query
+  const int nq = (int)max((int64_t)0, min((int64_t)kQ, L - q0));
+  // the CTA's key steps run to its last warp with queries
+  const int64_t wl = min((int64_t)(kWarps - 1), (L - 1 - q0c) / kQ);
+  const int64_t ktiles_cta = (q0c + kQ * wl) / 16 + 1;
+  const int64_t ktiles = nq > 0 ? q0 / 16 + 1 : 0;         // this warp's steps: up to its diagonal
 
-  build_tables_dig<kWs>(sq + (g * L + q0) * (32 * kWs), nq, kNT, false, est_scale, S.s_inv, S.s_mul, S.s_qsum,
-                        S.btab, 1, 0);
+  // every warp's tables, each built by the whole CTA
+  for (int w = 0; w < kWarps; ++w) {
+    const int64_t qw = q0c + kQ * w;
+    const int nw = (int)max((int64_t)0, min((int64_t)kQ, L - qw));
+    build_tables_dig<kWs>(sq + (g * L + min(qw, L - 1)) * (32 * kWs), nw, kNT, false, est_scale, SM.w[w].s_inv,
+                          SM.w[w].s_mul, SM.w[w].s_qsum, SM.w[w].btab, kWarps, 0);
+  }
 
   const int gq = lane >> 2, q = lane & 3, par = q & 1, half = q >> 1;
   const uint32_t hm = par ? 65536u : 1u;
@@ -103,39 +125,64 @@ __global__ void __launch_bounds__(32) prefill_kernel(const uint32_t* __restrict_
   for (int j = 0; j < kQ; ++j) m_run[j] = -INFINITY;
 #pragma unroll
   for (int ct = 0; ct < kNT; ++ct) l_part[ct] = 0.f;
-  const int64_t ktiles = q0 / 16 + 1;  // keys 0 .. q0 + 15 (the diagonal tile is the last)
-  // the global data of a 16-key step, loaded one step ahead: this lane's sign words of key rows
-  // gq and gq + 8, the norm of its key row, and the codes, scales and zeros of its value slice
+  // the sign words and norm of a 16-key step, loaded one step ahead (this lane's words of key rows
+  // gq and gq + 8, and the norm of its key row kr), and this thread's share of the value tile: key
+  // t / 8, code word t % 8 (16 channels) with its scale and zero
   struct StepData {
     uint2 wa, wb;
     float nrm;
-    uint4 cw;
-    uint16_t s0, z0, s1, z1;
+  };
+  struct ValData {
+    uint32_t cw;
+    uint16_t s, z;
   };
   const int kr = gq + 8 * par;
-  const int kk = lane >> 1, cb = 64 * (lane & 1);
+  const int vk = threadIdx.x >> 3, vw = threadIdx.x & 7;
   auto load_step = [&](int64_t k0, StepData& sd) {
     sd.wa = k0 + gq < L ? __ldg(reinterpret_cast<const uint2*>(bits + (g * L + k0 + gq) * kWs + 2 * q)) : make_uint2(0, 0);
     sd.wb = k0 + gq + 8 < L ? __ldg(reinterpret_cast<const uint2*>(bits + (g * L + k0 + gq + 8) * kWs + 2 * q))
                             : make_uint2(0, 0);
     sd.nrm = k0 + kr < L ? __ldg(norms + g * L + k0 + kr) : 0.f;
-    const int64_t kgv = k0 + kk;
-    if (kgv < L) {
-      sd.cw = __ldg(reinterpret_cast<const uint4*>(codes + (g * L + kgv) * (kD / 16) + cb / 16));
-      const int64_t gi = (g * L + kgv) * (kD / 32) + cb / 32;
-      sd.s0 = __ldg(scale + gi); sd.z0 = __ldg(zero + gi);
-      sd.s1 = __ldg(scale + gi + 1); sd.z1 = __ldg(zero + gi + 1);
+  };
+  auto load_val = [&](int64_t k0, ValData& vd) {
+    if (k0 + vk < L) {
+      vd.cw = __ldg(codes + (g * L + k0 + vk) * (kD / 16) + vw);
+      vd.s = __ldg(scale + (g * L + k0 + vk) * (kD / 32) + (vw >> 1));
+      vd.z = __ldg(zero + (g * L + k0 + vk) * (kD / 32) + (vw >> 1));
     } else {
-      // past the last token: zero values (P is 0 there)
-      sd.cw = make_uint4(0, 0, 0, 0);
-      sd.s0 = sd.z0 = sd.s1 = sd.z1 = 0;
+      vd.cw = 0u;  // past the last token: zero values (P is 0 there)
+      vd.s = vd.z = 0;
     }
   };
   StepData cur, nxt;
-  load_step(0, cur);
-  for (int64_t kt = 0; kt < ktiles; ++kt) {
+  ValData vcur, vnxt;
+  if (ktiles > 0) load_step(0, cur);
+  load_val(0, vcur);
+  for (int64_t kt = 0; kt < ktiles_cta; ++kt) {
     const int64_t k0 = kt * 16;
+    __half* Vt = SM.V[kt & 1];
+    // ---- v_hat (fp16) of this thread's 16 channels into the shared tile [key][channel]; the code
+    // comes out as float(2^23 | code) - 2^23, with no conversion instruction
+    {
+      const float sw = __half2float(__ushort_as_half(vcur.s)), zw = __half2float(__ushort_as_half(vcur.z));
+      uint32_t h[8];
+#pragma unroll
+      for (int c = 0; c < 16; c += 2) {
+        const float c0 = __uint_as_float(0x4B000000u | ((vcur.cw >> (2 * c)) & 3u)) - 8388608.f;
+        const float c1 = __uint_as_float(0x4B000000u | ((vcur.cw >> (2 * c + 2)) & 3u)) - 8388608.f;
+        const __half2 v = __floats2half2_rn(fmaf(c0, sw, zw), fmaf(c1, sw, zw));
+        h[c / 2] = *reinterpret_cast<const uint32_t*>(&v);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(Vt + vk * kVS + 16 * vw);
+      dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
+      dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+    }
+    if (kt + 1 < ktiles_cta) load_val(k0 + 16, vnxt);
     if (kt + 1 < ktiles) load_step(k0 + 16, nxt);
+    // the tile is complete for every warp; the other buffer is free (every warp passed this barrier
+    // only after finishing the step that read it)
+    __syncthreads();
+    if (kt < ktiles) {
     // ---- scores: rows g and g + 8 of the key tile, words 2q and 2q + 1
     const uint32_t w0[2] = {cur.wa.x, cur.wa.y}, w1[2] = {cur.wb.x, cur.wb.y};
     int acc[kNT][4];
@@ -213,24 +260,6 @@ __global__ void __launch_bounds__(32) prefill_kernel(const uint32_t* __restrict_
     __syncwarp();
 #pragma unroll
     for (int ct = 0; ct < kNT; ++ct) S.P[(2 * ct + half) * kPS + kr] = __float2half_rn(pv[ct]);
-    // ---- v_hat (fp16) into shared memory as [key][channel]: lane takes key lane / 2, channels 64 (lane % 2) ..
-    // The code comes out as float(2^23 | code) - 2^23, with no conversion instruction.
-    {
-      __half2* vrow = reinterpret_cast<__half2*>(S.V + kk * kVS + cb);
-      const uint32_t ws[4] = {cur.cw.x, cur.cw.y, cur.cw.z, cur.cw.w};
-      const float s0 = __half2float(__ushort_as_half(cur.s0)), z0 = __half2float(__ushort_as_half(cur.z0));
-      const float s1 = __half2float(__ushort_as_half(cur.s1)), z1 = __half2float(__ushort_as_half(cur.z1));
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float sw = w < 2 ? s0 : s1, zw = w < 2 ? z0 : z1;
-#pragma unroll
-        for (int c = 0; c < 16; c += 2) {
-          const float c0 = __uint_as_float(0x4B000000u | ((ws[w] >> (2 * c)) & 3u)) - 8388608.f;
-          const float c1 = __uint_as_float(0x4B000000u | ((ws[w] >> (2 * c + 2)) & 3u)) - 8388608.f;
-          vrow[(16 * w + c) / 2] = __floats2half2_rn(fmaf(c0, sw, zw), fmaf(c1, sw, zw));
-        }
-      }
-    }
     __syncwarp();
     // ---- o += P . v_hat
     uint32_t afr[4];
@@ -238,11 +267,13 @@ __global__ void __launch_bounds__(32) prefill_kernel(const uint32_t* __restrict_
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
       uint32_t bfr[2];
-      ldm_x2_trans(bfr, S.V + (lane & 15) * kVS + 8 * n);
+      ldm_x2_trans(bfr, Vt + (lane & 15) * kVS + 8 * n);
       mma_f16(o[n], afr, bfr);
     }
     __syncwarp();
     cur = nxt;
+    }
+    vcur = vnxt;
   }
   // ---- each query's sum: its 16 key lanes (lane bits 0, 2, 3, 4), then the other half's queries
   float l_run[kQ];
@@ -294,14 +325,14 @@ extern "C" qjl_status qjl_prefill_attention(const qjl_projection* P, const uint3
   if (!aligned16(bits) || !aligned16(codes) || !aligned16(sq) || !aligned16(out) || ((uintptr_t)norms & 3u) ||
       ((uintptr_t)scale & 1u) || ((uintptr_t)zero & 1u))
     return qjl_set_error(QJL_ERR_INVALID_ARG, "bits, codes, sq and out must be 16-byte aligned; norms, scale, zero naturally");
-  const int64_t nqt = (L + kQ - 1) / kQ;
+  const int64_t nqt = (L + kWarps * kQ - 1) / (kWarps * kQ);
   if (groups * nqt > ((int64_t)1 << 31) - 1) return qjl_set_error(QJL_ERR_UNSUPPORTED, "too many query tiles");
   DeviceGuard gd(P->device);
   if (!gd.ok) return qjl_set_error(QJL_ERR_CUDA, "cannot select the projection's device");
   const size_t smem = sizeof(PrefillSmem);
   if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return qjl_check_launch("prefill_kernel smem attribute");
-  prefill_kernel<<<(unsigned)(groups * nqt), 32, smem, (cudaStream_t)stream>>>(
+  prefill_kernel<<<(unsigned)(groups * nqt), kWarps * 32, smem, (cudaStream_t)stream>>>(
       bits, norms, codes, scale, zero, sq, groups, L, P->est_scale, softmax_scale * 1.4426950408889634f, out);
   return qjl_check_launch("prefill_kernel");
 }
