@@ -9,6 +9,7 @@
 // One warp per 16 consecutive queries of a key head, four warps (64 queries)
 // per CTA. The warps walk the key axis in 16-key steps, each up to its own
 // diagonal; the CTA dequantises each step's value tile once for all four.
+// At 168 registers and 72 KB of shared memory three CTAs (12 warps) fit on an SM.
 // Per warp and step:
 //   * scores: shift-window sign sums (build_tables_dig) on the u8 x s8
 //     mma.sync, two queries per n8 column tile, so 8 column tiles cover the
@@ -18,7 +19,7 @@
 //   * P . V on the fp16 tensor-core path (mma.sync m16n8k16, fp32
 //     accumulate). P goes through shared memory to ldmatrix as the A
 //     fragment; the step's 16 values are dequantised to fp16
-//     (code * scale + zero) into a double-buffered shared tile, one code word
+//     (code * scale + zero) into a shared tile, one code word
 //     per thread of the CTA, and read with ldmatrix.trans as the B fragments of
 //     16 channel tiles. Each step's key and value data is loaded one step
 //     ahead. (Dequantising the values once into an fp16 workspace
@@ -51,14 +52,14 @@ constexpr int kWarps = 4;       // warps per CTA: 64 consecutive queries share e
 
 struct WarpSmem {
   uint2 btab[kNT * kWs * 32];
-  float s_inv[64], s_mul[64];
-  int s_qsum[64];
+  float s_inv[kQ], s_mul[kQ];
+  int s_qsum[kQ];
   __align__(16) __half P[kQ * kPS];
 };
 
 struct PrefillSmem {
   WarpSmem w[kWarps];
-  __align__(16) __half V[2][16 * kVS];  // the step's value tile, double-buffered, shared by the warps
+  __align__(16) __half V[16 * kVS];  // the step's value tile, shared by the warps
 };
 
 __device__ __forceinline__ void ldm_x4(uint32_t (&r)[4], const void* p) {
@@ -81,7 +82,7 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], c
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-__global__ void __launch_bounds__(kWarps * 32) prefill_kernel(const uint32_t* __restrict__ bits,
+__global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t* __restrict__ bits,
                                                               const float* __restrict__ norms,
                                                               const uint32_t* __restrict__ codes,
                                                               const uint16_t* __restrict__ scale,
@@ -160,7 +161,7 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_kernel(const uint32_t* __
   load_val(0, vcur);
   for (int64_t kt = 0; kt < ktiles_cta; ++kt) {
     const int64_t k0 = kt * 16;
-    __half* Vt = SM.V[kt & 1];
+    __half* Vt = SM.V;
     // ---- v_hat (fp16) of this thread's 16 channels into the shared tile [key][channel]; the code
     // comes out as float(2^23 | code) - 2^23, with no conversion instruction
     {
@@ -179,8 +180,7 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_kernel(const uint32_t* __
     }
     if (kt + 1 < ktiles_cta) load_val(k0 + 16, vnxt);
     if (kt + 1 < ktiles) load_step(k0 + 16, nxt);
-    // the tile is complete for every warp; the other buffer is free (every warp passed this barrier
-    // only after finishing the step that read it)
+    // the tile is complete for every warp
     __syncthreads();
     if (kt < ktiles) {
     // ---- scores: rows g and g + 8 of the key tile, words 2q and 2q + 1
@@ -274,6 +274,8 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_kernel(const uint32_t* __
     cur = nxt;
     }
     vcur = vnxt;
+    // every warp is done with the tile before the next step overwrites it
+    __syncthreads();
   }
   // ---- each query's sum: its 16 key lanes (lane bits 0, 2, 3, 4), then the other half's queries
   float l_run[kQ];
