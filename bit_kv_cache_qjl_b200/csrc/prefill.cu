@@ -9,13 +9,16 @@
 // One warp per 16 consecutive queries of a key head, four warps (64 queries)
 // per CTA. The warps walk the key axis in 16-key steps, each up to its own
 // diagonal; the CTA dequantises each step's value tile once for all four.
-// At 168 registers and 72 KB of shared memory three CTAs (12 warps) fit on an SM.
+// At under 170 registers and 73 KB of shared memory three CTAs (12 warps) fit
+// on an SM.
 // Per warp and step:
 //   * scores: shift-window sign sums (build_tables_dig) on the u8 x s8
 //     mma.sync, two queries per n8 column tile, so 8 column tiles cover the
 //     warp's 16 queries; then the causal and length masks;
-//   * an online base-2 softmax, with each query's running max and sum kept
-//     identical in every lane;
+//   * an online base-2 softmax: a lane keeps the running max of the eight
+//     queries whose scores it holds, and its share of their sums; the
+//     rescale factors reach the lanes holding the output rows through
+//     shared memory;
 //   * P . V on the fp16 tensor-core path (mma.sync m16n8k16, fp32
 //     accumulate). P goes through shared memory to ldmatrix as the A
 //     fragment; the step's 16 values are dequantised to fp16
@@ -51,9 +54,10 @@ constexpr int kVS = kD + 8;     // V tile row stride (halves): 272 bytes
 constexpr int kWarps = 4;       // warps per CTA: 64 consecutive queries share each value tile
 
 struct WarpSmem {
-  uint2 btab[kNT * kWs * 32];
-  float s_inv[kQ], s_mul[kQ];
+  uint4 btab[kNT * kWs * 16];  // two shifts' B fragments per lane and entry
+  float s_inv[kQ], s_mul[kQ];  // s_mul: then times log2(e) * softmax scale
   int s_qsum[kQ];
+  float xq[kQ];  // per-query exchange: the step's rescale factors, then the final sums
   __align__(16) __half P[kQ * kPS];
 };
 
@@ -72,6 +76,16 @@ __device__ __forceinline__ void ldm_x2_trans(uint32_t (&r)[2], const void* p) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
                : "=r"(r[0]), "=r"(r[1])
                : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+
+// d = a . b with a zero accumulator input
+__device__ __forceinline__ void mma_u8s8_first(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};\n"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
 __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
@@ -103,16 +117,19 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
   const int nq = (int)max((int64_t)0, min((int64_t)kQ, L - q0));
   // the CTA's key steps run to its last warp with queries
   const int64_t wl = min((int64_t)(kWarps - 1), (L - 1 - q0c) / kQ);
-  const int64_t ktiles_cta = (q0c + kQ * wl) / 16 + 1;
-  const int64_t ktiles = nq > 0 ? q0 / 16 + 1 : 0;         // this warp's steps: up to its diagonal
+  const int ktiles_cta = (int)((q0c + kQ * wl) / 16 + 1);
+  const int ktiles = nq > 0 ? (int)(q0 / 16 + 1) : 0;    // this warp's steps: up to its diagonal
 
   // every warp's tables, each built by the whole CTA
   for (int w = 0; w < kWarps; ++w) {
     const int64_t qw = q0c + kQ * w;
     const int nw = (int)max((int64_t)0, min((int64_t)kQ, L - qw));
-    build_tables_dig<kWs>(sq + (g * L + min(qw, L - 1)) * (32 * kWs), nw, kNT, false, est_scale, SM.w[w].s_inv,
-                          SM.w[w].s_mul, SM.w[w].s_qsum, SM.w[w].btab, kWarps, 0);
+    build_tables_dig<kWs, true>(sq + (g * L + min(qw, L - 1)) * (32 * kWs), nw, kNT, false, est_scale,
+                                SM.w[w].s_inv, SM.w[w].s_mul, SM.w[w].s_qsum,
+                                reinterpret_cast<uint2*>(SM.w[w].btab), kWarps, 0);
   }
+  if (lane < kQ) S.s_mul[lane] *= logit2;
+  __syncwarp();
 
   const int gq = lane >> 2, q = lane & 3, par = q & 1, half = q >> 1;
   const uint32_t hm = par ? 65536u : 1u;
@@ -121,11 +138,14 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
   for (int n = 0; n < 16; ++n)
 #pragma unroll
     for (int j = 0; j < 4; ++j) o[n][j] = 0.f;
-  float m_run[kQ], l_part[kNT];
+  // the lane's eight queries 2 ct + half: running max (the same in all 16 lanes of the query) and
+  // this lane's share of the running sum
+  float m_own[kNT], l_part[kNT];
 #pragma unroll
-  for (int j = 0; j < kQ; ++j) m_run[j] = -INFINITY;
-#pragma unroll
-  for (int ct = 0; ct < kNT; ++ct) l_part[ct] = 0.f;
+  for (int ct = 0; ct < kNT; ++ct) {
+    m_own[ct] = -INFINITY;
+    l_part[ct] = 0.f;
+  }
   // the sign words and norm of a 16-key step, loaded one step ahead (this lane's words of key rows
   // gq and gq + 8, and the norm of its key row kr), and this thread's share of the value tile: key
   // t / 8, code word t % 8 (16 channels) with its scale and zero
@@ -139,17 +159,23 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
   };
   const int kr = gq + 8 * par;
   const int vk = threadIdx.x >> 3, vw = threadIdx.x & 7;
-  auto load_step = [&](int64_t k0, StepData& sd) {
-    sd.wa = k0 + gq < L ? __ldg(reinterpret_cast<const uint2*>(bits + (g * L + k0 + gq) * kWs + 2 * q)) : make_uint2(0, 0);
-    sd.wb = k0 + gq + 8 < L ? __ldg(reinterpret_cast<const uint2*>(bits + (g * L + k0 + gq + 8) * kWs + 2 * q))
-                            : make_uint2(0, 0);
-    sd.nrm = k0 + kr < L ? __ldg(norms + g * L + k0 + kr) : 0.f;
+  // 32-bit offsets from this group's and lane's first element (L <= 2^24)
+  const int Li = (int)L;
+  const uint2* bits_l = reinterpret_cast<const uint2*>(bits + (g * L + gq) * kWs + 2 * q);
+  const float* norms_l = norms + g * L + kr;
+  const uint32_t* codes_l = codes + (g * L + vk) * (kD / 16) + vw;
+  const uint16_t* scale_l = scale + (g * L + vk) * (kD / 32) + (vw >> 1);
+  const uint16_t* zero_l = zero + (g * L + vk) * (kD / 32) + (vw >> 1);
+  auto load_step = [&](int k0, StepData& sd) {
+    sd.wa = k0 + gq < Li ? __ldg(bits_l + k0 * (kWs / 2)) : make_uint2(0, 0);
+    sd.wb = k0 + gq + 8 < Li ? __ldg(bits_l + (k0 + 8) * (kWs / 2)) : make_uint2(0, 0);
+    sd.nrm = k0 + kr < Li ? __ldg(norms_l + k0) : 0.f;
   };
-  auto load_val = [&](int64_t k0, ValData& vd) {
-    if (k0 + vk < L) {
-      vd.cw = __ldg(codes + (g * L + k0 + vk) * (kD / 16) + vw);
-      vd.s = __ldg(scale + (g * L + k0 + vk) * (kD / 32) + (vw >> 1));
-      vd.z = __ldg(zero + (g * L + k0 + vk) * (kD / 32) + (vw >> 1));
+  auto load_val = [&](int k0, ValData& vd) {
+    if (k0 + vk < Li) {
+      vd.cw = __ldg(codes_l + k0 * (kD / 16));
+      vd.s = __ldg(scale_l + k0 * (kD / 32));
+      vd.z = __ldg(zero_l + k0 * (kD / 32));
     } else {
       vd.cw = 0u;  // past the last token: zero values (P is 0 there)
       vd.s = vd.z = 0;
@@ -159,8 +185,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
   ValData vcur, vnxt;
   if (ktiles > 0) load_step(0, cur);
   load_val(0, vcur);
-  for (int64_t kt = 0; kt < ktiles_cta; ++kt) {
-    const int64_t k0 = kt * 16;
+  for (int kt = 0; kt < ktiles_cta; ++kt) {
+    const int k0 = kt * 16;
     __half* Vt = SM.V;
     // ---- v_hat (fp16) of this thread's 16 channels into the shared tile [key][channel]; the code
     // comes out as float(2^23 | code) - 2^23, with no conversion instruction
@@ -187,24 +213,31 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
     const uint32_t w0[2] = {cur.wa.x, cur.wa.y}, w1[2] = {cur.wb.x, cur.wb.y};
     int acc[kNT][4];
 #pragma unroll
-    for (int sh = 0; sh < 8; ++sh) {
-      const uint32_t a0 = w0[0] >> sh, a1 = w1[0] >> sh, a2 = w0[1] >> sh, a3 = w1[1] >> sh;
+    for (int sp = 0; sp < kWs / 2; ++sp) {
+      // shifts 2 sp and 2 sp + 1, two column tiles at a time: one 16-byte table load per tile
 #pragma unroll
-      for (int ct = 0; ct < kNT; ++ct) {
-        const uint2 bb = S.btab[(ct * kWs + sh) * 32 + lane];
-        if (sh == 0) {
-          asm volatile(
-              "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-              "{%10,%10,%10,%10};\n"
-              : "=r"(acc[ct][0]), "=r"(acc[ct][1]), "=r"(acc[ct][2]), "=r"(acc[ct][3])
-              : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(bb.x), "r"(bb.y), "r"(0));
-        } else {
-          mma_u8s8(acc[ct], a0, a1, a2, a3, bb.x, bb.y);
+      for (int cg = 0; cg < kNT; cg += 2) {
+        uint4 bb[2];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) bb[c] = S.btab[((cg + c) * (kWs / 2) + sp) * 32 + lane];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int sh = 2 * sp + h;
+          const uint32_t a0 = w0[0] >> sh, a1 = w1[0] >> sh, a2 = w0[1] >> sh, a3 = w1[1] >> sh;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            if (sp == 0 && h == 0)
+              mma_u8s8_first(acc[cg + c], a0, a1, a2, a3, bb[c].x, bb[c].y);
+            else
+              mma_u8s8(acc[cg + c], a0, a1, a2, a3, h ? bb[c].z : bb[c].x, h ? bb[c].w : bb[c].y);
+          }
         }
       }
     }
     // lane (gq, q) completes key kr = gq + 8 par for query 2 ct + half of each column tile
-    const int64_t kg = k0 + kr;
+    // key kr's offset from the warp's first query; query jq sees it when rel <= jq < nq (which also
+    // keeps it below L, since q0 + nq <= L)
+    const int rel = k0 - (int)q0 + kr;
     const float nrm = cur.nrm;
     float xv[kNT];
 #pragma unroll
@@ -214,11 +247,12 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
       const uint32_t recv = __shfl_xor_sync(0xffffffffu, par ? P0 : P1, 1);
       const uint32_t tot = (par ? P1 : P0) + recv;
       const int jq = 2 * ct + half;
-      const bool ok = jq < nq && kg < L && kg <= q0 + jq;
-      xv[ct] = ok ? logit2 * S.s_mul[jq] * nrm * (float)(int)(2u * tot - (uint32_t)S.s_qsum[jq]) : -INFINITY;
+      xv[ct] = (rel <= jq && jq < nq) ? S.s_mul[jq] * nrm * (float)(int)(2u * tot - (uint32_t)S.s_qsum[jq])
+                                      : -INFINITY;
     }
-    // ---- online softmax: the step's max and sum per query, over the 16 lanes of the query's half
-    float tmax[kQ], corr[kQ], mnew[kQ];
+    // ---- online softmax of the lane's queries: the step's max over the query's 16 key lanes
+    // (lane bits 0, 2, 3, 4)
+    float pv[kNT], corr[kNT];
 #pragma unroll
     for (int ct = 0; ct < kNT; ++ct) {
       float v = xv[ct];
@@ -226,41 +260,30 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-      const float other = __shfl_xor_sync(0xffffffffu, v, 2);
-      // static register indices: query 2 ct is this lane's when half == 0
-      tmax[2 * ct] = half ? other : v;
-      tmax[2 * ct + 1] = half ? v : other;
+      const float mnew = fmaxf(m_own[ct], v);
+      corr[ct] = mnew == -INFINITY ? 1.f : exp2f(m_own[ct] - mnew);
+      m_own[ct] = mnew;
+      pv[ct] = (xv[ct] == -INFINITY) ? 0.f : exp2f(xv[ct] - mnew);
+      l_part[ct] = l_part[ct] * corr[ct] + pv[ct];
     }
+    // ---- P (fp16) into shared memory as [query][key], and the queries' rescale factors
+    __syncwarp();
 #pragma unroll
-    for (int j = 0; j < kQ; ++j) {
-      mnew[j] = fmaxf(m_run[j], tmax[j]);
-      corr[j] = mnew[j] == -INFINITY ? 1.f : exp2f(m_run[j] - mnew[j]);
-      m_run[j] = mnew[j];
-    }
-    float pv[kNT];
+    for (int ct = 0; ct < kNT; ++ct) S.P[(2 * ct + half) * kPS + kr] = __float2half_rn(pv[ct]);
+    if ((lane & ~2) == 0) {
 #pragma unroll
-    for (int ct = 0; ct < kNT; ++ct) {
-      const float mj = half ? mnew[2 * ct + 1] : mnew[2 * ct];
-      const float cj = half ? corr[2 * ct + 1] : corr[2 * ct];
-      pv[ct] = (xv[ct] == -INFINITY) ? 0.f : exp2f(xv[ct] - mj);
-      l_part[ct] = l_part[ct] * cj + pv[ct];  // this lane's share of query 2 ct + half's sum
+      for (int ct = 0; ct < kNT; ++ct) S.xq[2 * ct + half] = corr[ct];
     }
+    __syncwarp();
     // rescale the accumulator rows (queries gq and gq + 8)
     {
-      float c0 = corr[0], c1 = corr[8];
-#pragma unroll
-      for (int j = 1; j < 8; ++j) if (j == gq) { c0 = corr[j]; c1 = corr[j + 8]; }
+      const float c0 = S.xq[gq], c1 = S.xq[gq + 8];
 #pragma unroll
       for (int n = 0; n < 16; ++n) {
         o[n][0] *= c0; o[n][1] *= c0;
         o[n][2] *= c1; o[n][3] *= c1;
       }
     }
-    // ---- P (fp16) into shared memory as [query][key]
-    __syncwarp();
-#pragma unroll
-    for (int ct = 0; ct < kNT; ++ct) S.P[(2 * ct + half) * kPS + kr] = __float2half_rn(pv[ct]);
-    __syncwarp();
     // ---- o += P . v_hat
     uint32_t afr[4];
     ldm_x4(afr, S.P + (lane & 15) * kPS + 8 * (lane >> 4));
@@ -277,8 +300,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
     // every warp is done with the tile before the next step overwrites it
     __syncthreads();
   }
-  // ---- each query's sum: its 16 key lanes (lane bits 0, 2, 3, 4), then the other half's queries
-  float l_run[kQ];
+  // ---- each query's sum over its 16 key lanes (lane bits 0, 2, 3, 4), through shared memory to the
+  // lanes that hold its output row
+  float l_q[kNT];
 #pragma unroll
   for (int ct = 0; ct < kNT; ++ct) {
     float v = l_part[ct];
@@ -286,15 +310,16 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
     v += __shfl_xor_sync(0xffffffffu, v, 4);
     v += __shfl_xor_sync(0xffffffffu, v, 8);
     v += __shfl_xor_sync(0xffffffffu, v, 16);
-    const float other = __shfl_xor_sync(0xffffffffu, v, 2);
-    l_run[2 * ct] = half ? other : v;
-    l_run[2 * ct + 1] = half ? v : other;
+    l_q[ct] = v;
   }
-  // ---- normalise and store rows gq and gq + 8
-  float l0 = l_run[0], l1 = l_run[8];
+  __syncwarp();
+  if ((lane & ~2) == 0) {
 #pragma unroll
-  for (int j = 1; j < 8; ++j) if (j == gq) { l0 = l_run[j]; l1 = l_run[j + 8]; }
-  const float i0 = 1.f / l0, i1 = 1.f / l1;
+    for (int ct = 0; ct < kNT; ++ct) S.xq[2 * ct + half] = l_q[ct];
+  }
+  __syncwarp();
+  // ---- normalise and store rows gq and gq + 8
+  const float i0 = 1.f / S.xq[gq], i1 = 1.f / S.xq[gq + 8];
 #pragma unroll
   for (int n = 0; n < 16; ++n) {
     const int ch = 8 * n + 2 * q;

@@ -261,8 +261,11 @@ __device__ __forceinline__ int quant_dig(float v, float inv, int Qm) {
 // Quantises the J query rows of group `sqg` to the digit grid (s_inv, s_mul,
 // s_qsum) and fills the B fragments:
 // Btab[(nt * W + mu) * 32 + lane] for column tile nt and MMA mu = 8 p + s.
+// With PAIR the fragments of MMAs 2a and 2a + 1 sit side by side for each
+// lane, so one 16-byte load fetches both: entry (nt, mu, lane) is at
+// (nt * W + (mu & ~1)) * 32 + 2 lane + (mu & 1).
 // With dup, J must be 1 and the one query's digits fill both column halves.
-template <int W>
+template <int W, bool PAIR = false>
 __device__ void build_tables_dig(const float* __restrict__ sqg, int J, int NT, bool dup, float est_scale,
                                  float* s_inv, float* s_mul, int* s_qsum, uint2* Btab, int nwarps, int bar_id) {
   constexpr int m = 32 * W;
@@ -317,7 +320,7 @@ __device__ void build_tables_dig(const float* __restrict__ sqg, int J, int NT, b
         }
       }
     }
-    Btab[idx] = make_uint2(b[0], b[1]);
+    Btab[PAIR ? (nt * W + (mu & ~1)) * 32 + 2 * ln + (mu & 1) : idx] = make_uint2(b[0], b[1]);
   }
   named_barrier_or_sync(bar_id, nthreads);
 }
