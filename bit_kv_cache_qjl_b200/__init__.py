@@ -61,6 +61,14 @@ def _cuda(t, name):
         raise ValueError("%s must be contiguous" % name)
 
 
+def _cuda_rows(t, name):
+    """A 2-D CUDA tensor whose rows are contiguous; the row stride is passed as ld."""
+    if not (isinstance(t, torch.Tensor) and t.is_cuda):
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dim() != 2 or t.stride(1) != 1 or t.stride(0) < t.shape[1]:
+        raise ValueError("%s must be 2-D with contiguous rows" % name)
+
+
 class Projection:
     """A drawn random map (dense S, D-FQJL or P-FQJL) resident on the current device."""
 
@@ -118,8 +126,10 @@ def quantize_keys(proj, keys, first_token=0, bits=None, norms=None, stream=None)
 
 
 def project_queries(proj, q, out=None, stream=None):
-    """q [nq, d] fp32 -> S_eff q [nq, m] fp32 (no quantisation)."""
-    _cuda(q, "q")
+    """q [nq, d] fp32 (rows contiguous, any row stride) -> S_eff q [nq, m] fp32 (no quantisation)."""
+    _cuda_rows(q, "q")
+    if q.dtype != torch.float32:
+        raise TypeError("q must be float32")
     nq = q.shape[0]
     if out is None:
         out = torch.empty((nq, proj.m), dtype=torch.float32, device=q.device)

@@ -111,8 +111,10 @@ __global__ void __launch_bounds__(256) project_dense_kernel(const float* __restr
 
 qjl_status launch_project_dense(const qjl_projection* P, const float* q, int64_t nq, int64_t ld, float* out,
                                 cudaStream_t st) {
-  // many queries (a prefill projects every position): one warp per query row, the same fp32
-  // sum over j as below, with far less launch overhead than one CTA per query
+  // many queries (a prefill projects every position): with a bf16 S_eff the tensor cores at fp32
+  // accuracy (three bf16 parts of each query), else one warp per query row, the same fp32 sum over
+  // j as below, with far less launch overhead than one CTA per query
+  if (nq >= 1024 && project_mma_supported(P, q, ld, out)) return launch_project_mma(P, q, nq, ld, out, st);
   if (nq >= 1024) return launch_dense_simt(P, q, QJL_F32, nq, ld, nullptr, nullptr, out, st);
   const size_t smem = (size_t)P->d * sizeof(float);
   for (int64_t r0 = 0; r0 < nq; r0 += 65535) {

@@ -89,6 +89,11 @@ qjl_status launch_dense_simt(const qjl_projection* P, const void* keys, int dtyp
                              cudaStream_t st, const PageMap& pm = PageMap());
 qjl_status launch_project_dense(const qjl_projection* P, const float* q, int64_t nq, int64_t ld,
                                 float* out, cudaStream_t st);
+// many-query dense projection on the bf16 tensor cores (S_eff exactly bf16; the
+// query split into three bf16 parts): fp32 accuracy
+bool project_mma_supported(const qjl_projection* P, const float* q, int64_t ld, const float* out);
+qjl_status launch_project_mma(const qjl_projection* P, const float* q, int64_t nq, int64_t ld, float* out,
+                              cudaStream_t st);
 bool dense_tc_supported(const qjl_projection* P, int dtype, const void* keys, int64_t ld);
 qjl_status launch_dense_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld,
                            uint32_t* bits, float* norms, cudaStream_t st);

@@ -83,3 +83,13 @@ def test_values_and_decode_kernels(cuda_ok):
     # several queries per group take the tile-per-warp kernel and the split combine
     names = _kernels(lambda: run(2))
     assert _has(names, "decode_partial_kernel") and _has(names, "decode_combine_kernel"), names
+
+
+def test_many_query_projection_kernels(cuda_ok):
+    # a prefill's projection of every position: the bf16 tensor-core kernel when S_eff is bf16,
+    # the warp-per-row SIMT kernel when S is fp32
+    q = wl.normal((2048, 128), 4, "cuda")
+    Pb = qjl.Projection(2, 128, 256, "dense", s_bf16=True)
+    assert _has(_kernels(lambda: qjl.project_queries(Pb, q)), "project_mma_kernel")
+    Pf = qjl.Projection(2, 128, 256, "dense", s_bf16=False)
+    assert _has(_kernels(lambda: qjl.project_queries(Pf, q)), "dense_simt_kernel")

@@ -17,8 +17,13 @@ pytestmark = pytest.mark.gpu
                                              ("pfqjl", 256, 1024, 64, {}),
                                              ("dfqjl", 128, 256, 33, {}),
                                              ("pfqjl", 128, 256, 5, dict(dg_outer=True)),
-                                             # many queries (a prefill): the warp-per-row kernel
-                                             ("dense", 128, 256, 3000, dict(s_bf16=True))])
+                                             # many queries (a prefill): the bf16 tensor-core kernel
+                                             # with three bf16 parts per query element (bf16 S), the
+                                             # warp-per-row kernel (fp32 S)
+                                             ("dense", 128, 256, 3000, dict(s_bf16=True)),
+                                             ("dense", 128, 512, 1037, dict(s_bf16=True)),
+                                             ("dense", 64, 128, 1024, dict(s_bf16=True)),
+                                             ("dense", 128, 256, 2000, dict(s_bf16=False))])
 def test_project_queries(cuda_ok, kind, d, m, nq, kw):
     P = Projection(21, d, m, kind, **kw)
     q = wl.normal((nq, d), 55, "cuda")
@@ -32,5 +37,24 @@ def test_project_queries(cuda_ok, kind, d, m, nq, kw):
     else:
         rown = np.sqrt(d) * np.abs(O.D_g).max()
     tol = 1e-5 * qn * rown + 1e-30
+    err = np.abs(host(sq) - want)
+    assert np.all(err <= tol), (err / tol).max()
+
+
+def test_project_queries_many_strided_and_scaled(cuda_ok):
+    """Tensor-core projection of many queries: a row stride above d, and rows whose magnitudes
+    span many binades (the three bf16 parts must keep fp32 accuracy at every scale)."""
+    d, m, nq, ld = 128, 256, 1500, 136
+    P = Projection(23, d, m, "dense", s_bf16=True)
+    base = wl.normal((nq, ld), 57, "cuda")
+    scale = torch.pow(2.0, torch.linspace(-30, 30, nq, device="cuda"))[:, None]
+    qfull = base * scale
+    q = qfull[:, :d]
+    sq = project_queries(P, q)
+    torch.cuda.synchronize()
+    O = oracle_projection(P)
+    qh = host(q)
+    want = oracle.qjl.project_queries(O, qh)
+    tol = 1e-5 * np.linalg.norm(qh, axis=1, keepdims=True) * np.linalg.norm(O.S, axis=1)[None, :]
     err = np.abs(host(sq) - want)
     assert np.all(err <= tol), (err / tol).max()
