@@ -88,6 +88,13 @@ __device__ __forceinline__ void mma_u8s8_first(int (&d)[4], uint32_t a0, uint32_
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
+// 2^x on the special-function unit (PTX ex2.approx.ftz: about 2^-22 relative error, 2^-inf = 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -261,9 +268,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
       const float mnew = fmaxf(m_own[ct], v);
-      corr[ct] = mnew == -INFINITY ? 1.f : exp2f(m_own[ct] - mnew);
+      corr[ct] = mnew == -INFINITY ? 1.f : ex2(m_own[ct] - mnew);
       m_own[ct] = mnew;
-      pv[ct] = (xv[ct] == -INFINITY) ? 0.f : exp2f(xv[ct] - mnew);
+      pv[ct] = (xv[ct] == -INFINITY) ? 0.f : ex2(xv[ct] - mnew);
       l_part[ct] = l_part[ct] * corr[ct] + pv[ct];
     }
     // ---- P (fp16) into shared memory as [query][key], and the queries' rescale factors
