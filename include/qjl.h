@@ -142,6 +142,11 @@ qjl_status qjl_quantize_keys(const qjl_projection* proj, const void* keys, qjl_d
  * QJL abstract. sq[i] = S_eff q_i (dense) or the FQJL map of q_i, without
  * dither and without sign.
  *   q   [nq][ld] fp32, ld >= d.   sq  out [nq][m] fp32.
+ * The sums are fp32-accurate on every path. A dense map with bf16 S_eff and
+ * nq >= 1024 runs on the bf16 tensor cores: each query element splits into
+ * three bf16 parts, and the products with the exactly-bf16 S_eff are exact in
+ * fp32. That path needs d % 16 == 0, m % 128 == 0, q and sq 8-byte aligned
+ * and ld even. Otherwise an fp32 SIMT kernel runs.
  */
 qjl_status qjl_project_queries(const qjl_projection* proj, const float* q, int64_t nq,
                                int64_t ld, float* sq, void* stream);
