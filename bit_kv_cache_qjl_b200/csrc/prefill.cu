@@ -22,7 +22,7 @@
 //   * P . V on the fp16 tensor-core path (mma.sync m16n8k16, fp32
 //     accumulate). P goes through shared memory to ldmatrix as the A
 //     fragment; the step's 16 values are dequantised to fp16
-//     (code * scale + zero) into a shared tile, one code word
+//     (code * scale + zero, packed half2 arithmetic) into a shared tile, one code word
 //     per thread of the CTA, and read with ldmatrix.trans as the B fragments of
 //     16 channel tiles. Each step's key and value data is loaded one step
 //     ahead. (Dequantising the values once into an fp16 workspace
@@ -195,17 +195,20 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
   for (int kt = 0; kt < ktiles_cta; ++kt) {
     const int k0 = kt * 16;
     __half* Vt = SM.V;
-    // ---- v_hat (fp16) of this thread's 16 channels into the shared tile [key][channel]; the code
-    // comes out as float(2^23 | code) - 2^23, with no conversion instruction
+    // ---- v_hat (fp16) of this thread's 16 channels 16 vw + i into the shared tile [key][position].
+    // Within each 16-channel group, channels i and i + 8 sit side by side (positions 2i, 2i + 1), so
+    // one shift and one mask put both codes in the halves of a word: 0x6400 | code is 1024 + code in
+    // fp16, and (h - 1024) s + z is one packed subtract (exact) and one packed fused multiply-add
+    // (one rounding to fp16)
     {
-      const float sw = __half2float(__ushort_as_half(vcur.s)), zw = __half2float(__ushort_as_half(vcur.z));
+      const __half2 s2 = __half2half2(__ushort_as_half(vcur.s)), z2 = __half2half2(__ushort_as_half(vcur.z));
+      const __half2 k1024 = __half2half2(__ushort_as_half((unsigned short)0x6400u));
       uint32_t h[8];
 #pragma unroll
-      for (int c = 0; c < 16; c += 2) {
-        const float c0 = __uint_as_float(0x4B000000u | ((vcur.cw >> (2 * c)) & 3u)) - 8388608.f;
-        const float c1 = __uint_as_float(0x4B000000u | ((vcur.cw >> (2 * c + 2)) & 3u)) - 8388608.f;
-        const __half2 v = __floats2half2_rn(fmaf(c0, sw, zw), fmaf(c1, sw, zw));
-        h[c / 2] = *reinterpret_cast<const uint32_t*>(&v);
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t x = ((vcur.cw >> (2 * i)) & 0x00030003u) | 0x64006400u;
+        const __half2 v = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), k1024), s2, z2);
+        h[i] = *reinterpret_cast<const uint32_t*>(&v);
       }
       uint4* dst = reinterpret_cast<uint4*>(Vt + vk * kVS + 16 * vw);
       dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
@@ -327,16 +330,19 @@ __global__ void __launch_bounds__(kWarps * 32, 3) prefill_kernel(const uint32_t*
   __syncwarp();
   // ---- normalise and store rows gq and gq + 8
   const float i0 = 1.f / S.xq[gq], i1 = 1.f / S.xq[gq + 8];
+  // accumulator positions 8n + 2q and 8n + 2q + 1 hold channels ch and ch + 8 (the value tile's order)
 #pragma unroll
   for (int n = 0; n < 16; ++n) {
-    const int ch = 8 * n + 2 * q;
+    const int ch = 16 * (n >> 1) + 4 * (n & 1) + q;
     if (gq < nq) {
-      float2* p = reinterpret_cast<float2*>(out + (g * L + q0 + gq) * kD + ch);
-      *p = make_float2(o[n][0] * i0, o[n][1] * i0);
+      float* p = out + (g * L + q0 + gq) * kD + ch;
+      p[0] = o[n][0] * i0;
+      p[8] = o[n][1] * i0;
     }
     if (gq + 8 < nq) {
-      float2* p = reinterpret_cast<float2*>(out + (g * L + q0 + gq + 8) * kD + ch);
-      *p = make_float2(o[n][2] * i1, o[n][3] * i1);
+      float* p = out + (g * L + q0 + gq + 8) * kD + ch;
+      p[0] = o[n][2] * i1;
+      p[8] = o[n][3] * i1;
     }
   }
 }
