@@ -33,9 +33,9 @@ Modules:
     paged      append one token per group into pages; reads through a block table
 
 Parity status (each function's pins are in tests/test_oracle_*.py):
-    The absolute bit stream of the generator is parity unpinned on CPU. It is
-    pinned only by its statistics and by agreement with the separately written
-    library generator; see ``philox``.
+    Every function is pinned. The generator's bit stream is pinned by the
+    published Philox4x32-10 known-answer vectors, and by its statistics; see
+    ``philox``.
 """
 
 from . import philox, params, hadamard, qjl, kivi, attention, paged  # noqa: F401

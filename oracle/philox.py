@@ -17,10 +17,10 @@ as 1, 2, 3" (SC'11):
 
 Everything is vectorised over numpy uint64 arrays that hold 32-bit values.
 
-Parity unpinned (bit stream): no CPU library here implements Philox4x32. The
-tests pin the statistics (uniformity, Gaussian moments, permutation
-uniformity). They also check that this generator and the library's own copy
-agree bit for bit.
+Pins: the known-answer vectors published with the definition (three
+(counter, key) inputs and their outputs) fix the bit stream. The tests also pin
+the statistics (uniformity, Gaussian moments, permutation uniformity), and
+they check that this generator and the library's own copy agree bit for bit.
 """
 
 import numpy as np

@@ -1,7 +1,8 @@
 """Pins for the oracle's generator and parameter draws.
 
-No CPU library here implements Philox4x32-10, so the bit stream itself is
-parity unpinned on CPU. These tests pin what the method relies on: uniform
+The bit stream is pinned by the known-answer vectors published with the
+Philox definition (Salmon et al., SC'11, Random123): three (counter, key)
+inputs whose ten-round outputs are fixed. These tests also pin what the method relies on: uniform
 words and bits, standard-normal Box-Muller output, uniform permutations,
 balanced Rademacher signs, independent streams, and the avalanche property
 of the block function (one flipped counter bit changes about half of the
@@ -168,3 +169,18 @@ def test_dither_prefix_and_block_structure():
     assert np.all(np.isfinite(b))
     # the radius draw is never 0 or 1: |xi| is bounded by sqrt(-2 ln 2^-24)
     assert np.max(np.abs(P.dither(24, 128, 1024, np.arange(500)))) < math.sqrt(2 * 24 * math.log(2)) + 1e-9
+
+
+@pytest.mark.parametrize("ctr,key,want", [
+    ((0x00000000, 0x00000000, 0x00000000, 0x00000000), (0x00000000, 0x00000000),
+     (0x6627e8d5, 0xe169c58d, 0xbc57ac4c, 0x9b00dbd8)),
+    ((0xffffffff, 0xffffffff, 0xffffffff, 0xffffffff), (0xffffffff, 0xffffffff),
+     (0x408f276d, 0x41c83b0e, 0xa20bc7c6, 0x6d5451fd)),
+    ((0x243f6a88, 0x85a308d3, 0x13198a2e, 0x03707344), (0xa4093822, 0x299f31d0),
+     (0xd16cfe09, 0x94fdcceb, 0x5001e420, 0x24126ea1)),
+])
+def test_known_answer_vectors(ctr, key, want):
+    """Philox4x32-10 known-answer vectors published with the generator's definition."""
+    args = [np.array([v], dtype=np.uint64) for v in ctr + key]
+    got = tuple(int(np.asarray(w).ravel()[0]) for w in ph.philox4x32_10(*args))
+    assert got == want
