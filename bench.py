@@ -192,6 +192,19 @@ def cpu_oracle_rate(sample_keys, seconds_hint=None):
     return heads * per / dt, dt, threads, heads * per
 
 
+def default_desc():
+    """The workload text of the default step (decode_llama7b), shared by both arms' config."""
+    return ("%s: B=%d, heads=%d, N=%d, d=%d, m=%d dense bf16 S; quantize all keys, project 1 query/head, "
+            "score all keys" % (WORKLOAD, B, H, N, D, M))
+
+
+def run_config(desc, units, world):
+    """The JSON line's config: the same dict for our arm and the reference arm."""
+    return {"workload": desc, "units_per_step": units * world,
+            "l2": "inputs larger than L2 (126 MB) in every step, no flush",
+            "parallelism": "replicas (weak)" if world > 1 else "single GPU"}
+
+
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -210,10 +223,10 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD + " (CPU oracle sample)", "sample_keys": sample,
-                                            "B": B, "H": H, "N": N, "d": D, "m": M},
+            "data": "synthetic", "config": run_config(default_desc(), B * H * N, world),
             "cpu_baseline": {"value": value, "unit": "keys/s", "cores": threads, "kind": "oracle",
-                             "sample": "%d keys (one head slice) per step: oracle quantize + project + score" % sample},
+                             "sample": "%d keys (one head slice of the workload) per step: oracle quantize + "
+                                       "project + score" % sample},
             "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
@@ -307,9 +320,7 @@ def build_workload(name, dev, qjl, wl, torch):
             Stage("scores", lambda: qjl.scores(P, bits.view(G, N, M // 32), norms.view(G, N), sq.view(G, 1, M), out=out),
                   G * N, M // 8 + 4 + 4, 0, "scores_digit_kernel", "scores.cu"),
         ]
-        W.update(units=G * N, unit="keys/s", inputs=[keys, q], outputs=[out], dtype="bf16",
-                 desc="%s: B=%d, heads=%d, N=%d, d=%d, m=%d dense bf16 S; quantize all keys, project 1 query/head, "
-                      "score all keys" % (name, B, H, N, D, M))
+        W.update(units=G * N, unit="keys/s", inputs=[keys, q], outputs=[out], dtype="bf16", desc=default_desc())
     elif name == "gqa_decode":
         Bq, Hq, Hkv, Nq, m = 16, 32, 8, 131072, 512
         G, J = Bq * Hkv, Hq // Hkv
@@ -669,9 +680,7 @@ def main():
         "metric": METRIC, "value": value, "unit": Wk["unit"], "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": Wk["dtype"], "data": "synthetic",
-        "config": {"workload": Wk["desc"], "units_per_step": units * world,
-                   "l2": "inputs larger than L2 (126 MB) in every step, no flush",
-                   "parallelism": "replicas (weak)" if world > 1 else "single GPU"},
+        "config": run_config(Wk["desc"], units, world),
         "roofline": roof,
         "kernels": kernels,
         "e2e": {"value": world * units / (e2e_ms * 1e-3), "unit": Wk["unit"], "h2d_bytes_per_step": h2d,
