@@ -7,6 +7,9 @@
   products with fp32 accumulation carry the fp32 dot product.
 * The prefill dequantises 2-bit codes in half2: the bit pattern 0x6400 | c is
   1024 + c in binary16, and (1024 + c) - 1024 = c exactly.
+* The score kernels' shift-window sign sums with four signed base-256 digit
+  columns reproduce sum_i b_i Q_i exactly, with no int32 overflow, up to the
+  digit grid's bound |Q_i| <= (2^31 - 1) / m.
 """
 
 import numpy as np
@@ -71,3 +74,61 @@ def test_half2_code_pattern():
         lo = np.array([x & 0xFFFF], dtype=np.uint16).view(np.float16)[0]
         hi = np.array([x >> 16], dtype=np.uint16).view(np.float16)[0]
         assert float(lo) - 1024 == codes[i] and float(hi) - 1024 == codes[i + 8]
+
+
+def _window_digits(Q):
+    """Per bit i of a 32-bit word: the weight B_i that makes the shift windows exact, as four signed
+    base-256 digits. Byte e of (w >> s) is sum_t 2^t b_(8e+s+t); B = K^-1 Q for the unit lower-
+    triangular window matrix K, i.e. B_i = sum_k 256^k (Q_(i-8k) - 2 Q_(i-8k-1)) mod 2^32."""
+    B = np.zeros(32, dtype=np.int64)
+    for i in range(32):
+        v = 0
+        for k in range(4):
+            j = i - 8 * k
+            if j < 0:
+                break
+            v += (int(Q[j]) - (2 * int(Q[j - 1]) if j > 0 else 0)) << (8 * k)
+        B[i] = v % (1 << 32)
+    dig = np.zeros((32, 4), dtype=np.int64)
+    for i in range(32):
+        u = int(B[i])
+        for c in range(4):
+            d = u & 0xFF
+            d = d - 256 if d >= 128 else d
+            dig[i, c] = d
+            u = ((u - d) % (1 << 32)) >> 8
+    return dig
+
+
+def test_shift_window_digits_give_the_exact_sign_sum():
+    """The decode-score and prefill kernels' sign sums: eight shifted copies of each sign word as
+    u8 operands against four signed digit columns, int32 accumulation, then D0 + 2^8 D1 + 2^16 D2
+    + 2^24 D3 in wrapping 32-bit arithmetic. It must equal sum_i b_i Q_i exactly for |Q_i| up to
+    (2^31 - 1) / m, and no int32 accumulator may overflow."""
+    rng = np.random.default_rng(9)
+    for m in (256, 512):
+        qmax = (2 ** 31 - 1) // m
+        for trial in range(12):
+            Q = rng.integers(-qmax, qmax + 1, size=m)
+            if trial == 0:
+                Q[:] = qmax
+            if trial == 1:
+                Q[:] = -qmax
+            words = rng.integers(0, 1 << 32, size=m // 32, dtype=np.uint64)
+            if trial in (0, 1):
+                words[:] = (1 << 32) - 1
+            D = np.zeros(4, dtype=np.int64)
+            for w_idx, w in enumerate(words.tolist()):
+                dig = _window_digits(Q[32 * w_idx:32 * (w_idx + 1)])
+                for s in range(8):
+                    r = w >> s
+                    for e in range(4):
+                        a = (r >> (8 * e)) & 0xFF
+                        D += a * dig[8 * e + s]
+                assert np.all(np.abs(D) < 2 ** 31)
+            tot = int(sum(int(D[c]) << (8 * c) for c in range(4)) % (1 << 32))
+            tot = tot - (1 << 32) if tot >= 1 << 31 else tot
+            bits = np.array([(int(words[i // 32]) >> (i % 32)) & 1 for i in range(m)])
+            assert tot == int((bits * Q).sum())
+            # the estimator's signed sum: 2 tot - sum Q = sum (2 b - 1) Q
+            assert 2 * tot - int(Q.sum()) == int(((2 * bits - 1) * Q).sum())
