@@ -78,3 +78,33 @@ def test_workspace_sizing(L):
     # 2-4 queries per group: groups x splits x queries slots of d + 2 floats
     assert b2 > 0 and b2 % (2 * 130 * 4) == 0
     assert L.qjl_decode_workspace_bytes(1024, 4, 16384, 128) == 2 * b2
+
+
+def test_kivi_key_argument_checks(L):
+    z = ctypes.c_void_p(0)
+    bad = ctypes.c_void_p(8)                                                  # misaligned
+    q = L.qjl_kivi_quantize_keys_2bit
+    assert q(z, 5, 2, 64, 128, z, z, z, None) == -1                           # unknown dtype
+    assert q(z, 1, -1, 64, 128, z, z, z, None) == -1                          # negative groups
+    assert q(z, 1, 2, 64, 96, z, z, z, None) == -2                            # d outside {64, 128, 256}
+    assert q(z, 1, 0, 64, 128, z, z, z, None) == 0                            # no groups: a no-op
+    assert q(z, 1, 2, 0, 128, z, z, z, None) == 0                             # no tokens: a no-op
+    assert q(z, 1, 2, 64, 128, z, z, z, None) == -1                           # NULL pointers
+    assert q(bad, 1, 2, 64, 128, bad, bad, bad, None) == -1
+    assert b"aligned" in L.qjl_last_error_message()
+    s = L.qjl_kivi_key_scores
+    assert s(z, z, z, 2, 64, 128, z, 0, z, None) == -1                        # q_per_group < 1
+    assert s(z, z, z, 2, 64, 128, z, 65, z, None) == -1                       # q_per_group > 64
+    assert s(z, z, z, 2, 64, 32, z, 1, z, None) == -2                         # unsupported d
+    assert s(z, z, z, 0, 64, 128, z, 1, z, None) == 0                         # no groups: a no-op
+    assert s(z, z, z, 2, 64, 128, z, 1, z, None) == -1                        # NULL pointers
+    assert s(bad, z, z, 2, 64, 128, z, 1, z, None) == -1
+
+
+def test_paged_and_prefill_calls_reject_a_null_projection(L):
+    z = ctypes.c_void_p(0)
+    assert L.qjl_append_keys(None, z, 1, 1, 128, z, z, 1, 16, 1, z, z, None) == -1
+    assert L.qjl_scores_paged(None, z, z, z, 1, 16, 1, z, 1, 16, z, 1, z, None) == -1
+    assert L.qjl_decode_attention_paged(None, z, z, z, z, z, z, 1, 16, 1, z, 1, 16, z, 1.0, z, z, 0, None) == -1
+    assert L.qjl_prefill_attention(None, z, z, z, z, z, 1, 16, z, 1.0, z, None) == -1
+    assert b"NULL" in L.qjl_last_error_message() or b"projection" in L.qjl_last_error_message()
