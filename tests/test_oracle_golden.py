@@ -5,7 +5,7 @@ import os
 
 import numpy as np
 
-from oracle import kivi, params as P, qjl
+from oracle import attention, kivi, params as P, qjl
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden", "oracle_small.json")
 
@@ -27,3 +27,18 @@ def test_oracle_matches_frozen_fixture():
     assert codes.tolist() == v["codes"]
     assert scale.astype(np.float64).tolist() == v["scale"]
     assert zero.astype(np.float64).tolist() == v["zero"]
+
+
+
+def test_kivi_keys_and_prefill_match_frozen_fixture():
+    data = json.load(open(GOLD))
+    k = data["kivi_keys"]
+    codes, scale, zero = kivi.quantize_keys_per_channel(np.array(k["k"], dtype=np.float32))
+    assert codes.astype(np.int64).tolist() == k["codes"]
+    assert scale.astype(np.float64).tolist() == k["scale"]
+    assert zero.astype(np.float64).tolist() == k["zero"]
+    sc = kivi.key_scores(codes, scale, zero, np.array(k["q"], dtype=np.float64))
+    assert np.allclose(sc, k["scores"], rtol=1e-13, atol=1e-13)
+    p = data["prefill"]
+    out, _ = attention.prefill_attention(np.array(p["est"]), np.array(p["vhat"]), p["scale"])
+    assert np.allclose(out, p["out"], rtol=1e-13, atol=1e-13)
