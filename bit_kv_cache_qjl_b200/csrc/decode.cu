@@ -731,7 +731,7 @@ qjl_status launch_stream(const qjl_projection* P, const uint32_t* bits, const fl
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
     return qjl_check_launch("decode_stream_kernel smem attribute");
   int* err = qjl_error_flag(P->device);
-  if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  if (!err) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   const StreamPlan plan = stream_plan(G, N);
   qjl_log_launch("decode_stream_kernel", plan.ncta, kDsThreads, smem, 1);
   kern<<<(unsigned)plan.ncta, kDsThreads, smem, st>>>(bits, norms, codes, scale, zero, sq, G, N, NS, P->est_scale,

@@ -10,10 +10,12 @@
 //
 // The array is a host-side symbol: its name in host code is not a device
 // address. The first call on each device resolves the address with
-// cudaGetSymbolAddress, with that device current, and caches it. That first
-// call should therefore come before any stream capture. Every call shares the
-// array, and overlapping calls on the GPU race. The kernels write every
-// workspace entry they later read, so stale contents need no clearing.
+// cudaGetSymbolAddress, with that device current, and caches it (as it does
+// for the kernels' error int, also static device storage). That first call
+// should therefore come before any stream capture, and the cached addresses
+// last as long as the device's primary context. Every call shares the array,
+// and overlapping calls on the GPU race. The kernels write every workspace
+// entry they later read, so stale contents need no clearing.
 
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -52,9 +54,15 @@ extern "C" qjl_status qjl_decode_attention_noalloc(const qjl_projection* P, cons
                                                    const uint32_t* codes, const uint16_t* scale, const uint16_t* zero,
                                                    int64_t groups, int64_t N, const float* sq, int J,
                                                    float softmax_scale, float* out, void* stream) {
+  qjl_set_error(QJL_OK, "");
   if (!P) return qjl_set_error(QJL_ERR_INVALID_ARG, "projection is NULL");
-  if (groups < 0 || N < 0 || J < 1 || J > 64) return qjl_set_error(QJL_ERR_INVALID_ARG, "groups/N/q_per_group out of range");
-  if (groups > 0 && N > 0 && P->d % 32 == 0) {
+  // the range checks of qjl_decode_attention, before the workspace size is computed from them
+  if (groups < 0 || N < 0 || groups > (1 << 24) || N > ((int64_t)1 << 36))
+    return qjl_set_error(QJL_ERR_INVALID_ARG, "groups/N out of range");
+  if (J < 1 || J > 64) return qjl_set_error(QJL_ERR_INVALID_ARG, "q_per_group must be in 1..64");
+  if (P->d % 32 || P->d > 1024)
+    return qjl_set_error(QJL_ERR_UNSUPPORTED, "decode attention needs d a multiple of 32, <= 1024");
+  if (groups > 0 && N > 0) {
     const size_t need = decode_workspace_bytes(groups, J, N, P->d);
     if (need > QJL_DECODE_NOALLOC_SCRATCH_BYTES)
       return qjl_set_error(QJL_ERR_WORKSPACE,
@@ -73,6 +81,8 @@ extern "C" qjl_status qjl_decode_attention_noalloc(const qjl_projection* P, cons
   }
   void* ws = nullptr;
   qjl_status st = scratch_address(P->device, &ws);
+  if (st == QJL_OK && !qjl_error_flag(P->device))
+    st = qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   if (st == QJL_OK)
     st = qjl_decode_attention(P, bits, norms, codes, scale, zero, groups, N, sq, J, softmax_scale, out, ws,
                               QJL_DECODE_NOALLOC_SCRATCH_BYTES, stream);

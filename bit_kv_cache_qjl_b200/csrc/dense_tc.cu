@@ -33,6 +33,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <string.h>
+
 #include <mutex>
 
 #include "qjl_internal.h"
@@ -473,14 +475,44 @@ bool dense_tc_supported(const qjl_projection* P, int dtype, const void* keys, in
   return pick_stages(P->d, P->m) >= 2 && get_encode() != nullptr;
 }
 
+static_assert(sizeof(CUtensorMap) == sizeof(qjl_projection::s_map), "CUtensorMap size");
+
+void dense_tc_prepare(qjl_projection* P) {
+  P->s_map_ok = P->S_bf16 && make_map(reinterpret_cast<CUtensorMap*>(P->s_map), P->S_bf16, (uint64_t)P->m,
+                                      (uint64_t)P->d, (uint64_t)P->d, (uint32_t)std::min(P->m, 256));
+}
+
 qjl_status launch_dense_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld, uint32_t* bits,
                            float* norms, cudaStream_t st) {
-  CUtensorMap tmK, tmS;
-  if (!make_map(&tmK, keys, (uint64_t)n, (uint64_t)P->d, (uint64_t)ld, BM) ||
-      !make_map(&tmS, P->S_bf16, (uint64_t)P->m, (uint64_t)P->d, (uint64_t)P->d, (uint32_t)std::min(P->m, 256)))
-    return qjl_set_error(QJL_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  // The keys' map is cached per thread for the last (pointer, rows, ld, d): a
+  // caller that quantises the same buffer every step encodes it once. S's map
+  // was encoded with the projection.
+  struct KeyMapCache {
+    const void* ptr = nullptr;
+    int64_t n = -1, ld = -1;
+    int d = -1;
+    CUtensorMap map;
+  };
+  static thread_local KeyMapCache kc;
+  if (kc.ptr != keys || kc.n != n || kc.ld != ld || kc.d != P->d) {
+    kc.ptr = nullptr;
+    if (!make_map(&kc.map, keys, (uint64_t)n, (uint64_t)P->d, (uint64_t)ld, BM))
+      return qjl_set_error(QJL_ERR_CUDA, "cuTensorMapEncodeTiled failed for the keys");
+    kc.ptr = keys;
+    kc.n = n;
+    kc.ld = ld;
+    kc.d = P->d;
+  }
+  const CUtensorMap tmK = kc.map;
+  CUtensorMap tmS;
+  if (P->s_map_ok) {
+    memcpy(&tmS, P->s_map, sizeof(tmS));
+  } else if (!make_map(&tmS, P->S_bf16, (uint64_t)P->m, (uint64_t)P->d, (uint64_t)P->d,
+                       (uint32_t)std::min(P->m, 256))) {
+    return qjl_set_error(QJL_ERR_CUDA, "cuTensorMapEncodeTiled failed for S");
+  }
   int* err = qjl_error_flag(P->device);
-  if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  if (!err) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   const int ns = pick_stages(P->d, P->m);
   const size_t smem = smem_bytes(P->d, P->m, ns);
   TcParams prm{n, P->m, ns, (P->m + 255) / 256, bits, norms, err};

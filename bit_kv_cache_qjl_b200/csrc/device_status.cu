@@ -52,7 +52,7 @@ qjl_status qjl_device_errors(int device, int clear, int* flags) {
   DeviceGuard g(device);
   if (!g.ok) return qjl_set_error(QJL_ERR_CUDA, "cannot select the device");
   int* err = qjl_error_flag(device);
-  if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  if (!err) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   if (cudaDeviceSynchronize() != cudaSuccess) return qjl_check_launch("qjl_device_errors: synchronize");
   if (cudaMemcpy(flags, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return qjl_check_launch("qjl_device_errors: read");
@@ -66,7 +66,7 @@ qjl_status qjl_selftest_bounded_wait(int device, uint64_t limit_ns) {
   DeviceGuard g(device);
   if (!g.ok) return qjl_set_error(QJL_ERR_CUDA, "cannot select the device");
   int* err = qjl_error_flag(device);
-  if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  if (!err) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   selftest_wait_kernel<<<1, 32>>>(limit_ns, err);
   return qjl_check_launch("selftest_wait_kernel");
 }

@@ -557,7 +557,7 @@ qjl_status launch_fqjl_keys(const qjl_projection* P, const void* x, int dtype, i
   a.W = P->m / 32;
   a.err = qjl_error_flag(P->device);
   a.pm = pm;
-  if (!a.err) return qjl_set_error(QJL_ERR_CUDA, "cannot allocate the device error flag");
+  if (!a.err) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   switch (P->d) {
     case 32: return launch_el<32, 1>(P, a, dtype, n, st);
     case 64: return launch_el<64, 1>(P, a, dtype, n, st);

@@ -60,7 +60,7 @@ qjl_status qjl_append_keys(const qjl_projection* P, const void* keys, qjl_dtype 
   if (((uintptr_t)positions & 3u)) return qjl_set_error(QJL_ERR_INVALID_ARG, "positions must be 4-byte aligned");
   DeviceGuard g(P->device);
   if (!g.ok) return qjl_set_error(QJL_ERR_CUDA, "cannot select the projection's device");
-  if (!qjl_error_flag(P->device)) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  if (!qjl_error_flag(P->device)) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   PageMap pm;
   pm.pos = positions;
   pm.table = block_table;
@@ -91,7 +91,7 @@ qjl_status qjl_append_values_2bit(const void* v, qjl_dtype dtype, int64_t groups
   if (((uintptr_t)positions & 3u)) return qjl_set_error(QJL_ERR_INVALID_ARG, "positions must be 4-byte aligned");
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return qjl_set_error(QJL_ERR_CUDA, "cannot query the current device");
-  if (!qjl_error_flag(dev)) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  if (!qjl_error_flag(dev)) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   PageMap pm;
   pm.pos = positions;
   pm.table = block_table;
@@ -162,7 +162,7 @@ qjl_status qjl_decode_attention_paged(const qjl_projection* P, const uint32_t* b
     return qjl_set_error(QJL_ERR_WORKSPACE, "workspace smaller than qjl_decode_paged_workspace_bytes()");
   DeviceGuard g(P->device);
   if (!g.ok) return qjl_set_error(QJL_ERR_CUDA, "cannot select the projection's device");
-  if (!qjl_error_flag(P->device)) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  if (!qjl_error_flag(P->device)) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   PagedRead pr;
   pr.table = block_table;
   pr.seq_lens = seq_lens;

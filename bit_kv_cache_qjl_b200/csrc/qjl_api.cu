@@ -53,20 +53,23 @@ void qjl_log_launch(const char* kernel, int64_t grid, int block, size_t smem, in
             per_sm);
 }
 
+// The per-device error int is static device storage of this module, so no
+// call of the library allocates device memory for it: it exists on every
+// device from the moment the module is loaded there, zero-initialised. Its
+// device address is resolved once per device (with that device current) and
+// cached; it stays valid for the life of the device's primary context.
+static __device__ int g_kernel_error;
+
 int* qjl_error_flag(int device) {
   static std::mutex mu;
   static int* flags[64] = {};
-  std::lock_guard<std::mutex> lock(mu);
   if (device < 0 || device >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (!flags[device]) {
+    DeviceGuard g(device);
     void* p = nullptr;
-    if (cudaMalloc(&p, sizeof(int)) != cudaSuccess) {
+    if (!g.ok || cudaGetSymbolAddress(&p, g_kernel_error) != cudaSuccess || !p) {
       cudaGetLastError();
-      return nullptr;
-    }
-    if (cudaMemset(p, 0, sizeof(int)) != cudaSuccess) {
-      cudaGetLastError();
-      cudaFree(p);
       return nullptr;
     }
     flags[device] = (int*)p;
@@ -231,6 +234,7 @@ qjl_status qjl_make_projection(uint64_t seed, int d, int m, qjl_kind kind, const
     }
     if (o.s_bf16) st = dev_upload(&P->S_bf16, sb.data(), md);
     if (st == QJL_OK) st = dev_upload(&P->St_f32, st_f.data(), md);
+    if (st == QJL_OK && o.s_bf16) dense_tc_prepare(P);
   } else {
     const int nb = m / d;
     const size_t cnt = (size_t)nb * d;

@@ -23,6 +23,10 @@ struct qjl_projection {
   int32_t* perm = nullptr;
   float* D_g = nullptr;
   float* ktab = nullptr;        // key-kernel tables, per block (fqjl_key_tables)
+  // the tensor map of S_bf16 for the tcgen05 quantize kernel (a CUtensorMap),
+  // encoded once when the projection is made; s_map_ok is false if that failed
+  alignas(64) unsigned char s_map[128] = {};
+  bool s_map_ok = false;
   // host copies for export
   float* h_S = nullptr;
   float* h_D_r = nullptr;
@@ -95,6 +99,8 @@ bool project_mma_supported(const qjl_projection* P, const float* q, int64_t ld, 
 qjl_status launch_project_mma(const qjl_projection* P, const float* q, int64_t nq, int64_t ld, float* out,
                               cudaStream_t st);
 bool dense_tc_supported(const qjl_projection* P, int dtype, const void* keys, int64_t ld);
+// encodes P->s_map (called once by qjl_make_projection for a bf16 dense S)
+void dense_tc_prepare(qjl_projection* P);
 qjl_status launch_dense_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld,
                            uint32_t* bits, float* norms, cudaStream_t st);
 qjl_status launch_fqjl_queries(const qjl_projection* P, const float* q, int64_t nq, int64_t ld,
@@ -104,9 +110,6 @@ qjl_status launch_fqjl_keys(const qjl_projection* P, const void* keys, int dtype
                             uint64_t first_token, uint32_t* bits, float* norms, cudaStream_t st,
                             const PageMap& pm = PageMap());
 bool scores_mma_supported(int m);
-bool scores_tc_supported(int m, int J);
-qjl_status launch_scores_tc(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t groups,
-                            int64_t N, const float* sq, int J, float* scores, cudaStream_t st);
 qjl_status launch_scores(const qjl_projection* P, const uint32_t* bits, const float* norms,
                          int64_t groups, int64_t N, const float* sq, int J, float* scores,
                          cudaStream_t st);
@@ -128,15 +131,16 @@ qjl_status launch_decode(const qjl_projection* P, const uint32_t* bits, const fl
 
 // Bits of the per-device error int (read by qjl_device_errors). Bits 1..32 mark
 // bounded waits that expired (each kernel's producer, drain, consumer and, in
-// the tcgen05 kernels, MMA, TMEM and norm-warp waits).
+// the tcgen05 kernel, MMA, TMEM and norm-warp waits).
 enum : int {
   QJL_DEVERR_WAITS = 63,   // bits 1, 2, 4, 8, 16, 32: a bounded wait expired
   QJL_DEVERR_PAGE = 64,    // a paged-cache position or block-table entry was out of range and skipped
   QJL_DEVERR_SELFTEST = 128  // qjl_selftest_bounded_wait's wait expired, as it should
 };
 
-// Per-device int the kernels set when a bounded wait expires (qjl_api.cu).
-// It is allocated on first use and never freed.
+// Per-device int the kernels set when a bounded wait expires (qjl_api.cu):
+// static device storage whose address is resolved on first use, so no call
+// allocates for it. nullptr if the address cannot be resolved.
 int* qjl_error_flag(int device);
 
 // When the environment variable QJL_LOG_LAUNCH is set, print a launch's

@@ -35,7 +35,6 @@
 
 #include <algorithm>
 #include <type_traits>
-#include <string.h>
 
 #include "qjl_internal.h"
 #include "mbarrier.cuh"
@@ -770,7 +769,7 @@ qjl_status launch_mma(const qjl_projection* P, const uint32_t* bits, const float
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess || per_sm < 1)
     return qjl_check_launch("scores_stream_kernel occupancy");
   int* err = qjl_error_flag(P->device);
-  if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  if (!err) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   const int64_t total = G * ((N + kStageKeys - 1) / kStageKeys);
   const int64_t slots = (int64_t)qjl_num_sms(P->device) * per_sm;
   const int64_t grid = std::min<int64_t>(total, slots);
@@ -797,7 +796,7 @@ qjl_status launch_decode_fast(const qjl_projection* P, const uint32_t* bits, con
   const int regs_per_cta = ((fa.numRegs * 32 + 255) / 256) * 256 * (kDecThreads / 32);
   const int per_sm = std::max(1, std::min(65536 / std::max(regs_per_cta, 1), (int)((228u * 1024u) / (smem + 1024))));
   int* err = qjl_error_flag(P->device);
-  if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  if (!err) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   const int64_t total = G * ((N + kDecStageKeys - 1) / kDecStageKeys);
   const int64_t slots = (int64_t)qjl_num_sms(P->device) * per_sm;
   const int64_t grid = std::min<int64_t>(total, slots);
@@ -823,7 +822,7 @@ qjl_status launch_digit(const qjl_projection* P, const uint32_t* bits, const flo
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, smem) != cudaSuccess || per_sm < 1)
     return qjl_check_launch("scores_digit_kernel occupancy");
   int* err = qjl_error_flag(P->device);
-  if (!err) return qjl_set_error(QJL_ERR_OOM, "cannot allocate the kernel error flag");
+  if (!err) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   const int64_t total = G * ((N + SKT - 1) / SKT);
   const int64_t slots = (int64_t)qjl_num_sms(P->device) * per_sm;
   const int64_t grid = std::min<int64_t>(total, slots);
@@ -852,22 +851,12 @@ qjl_status launch_scores(const qjl_projection* P, const uint32_t* bits, const fl
                          int64_t G, int64_t N, const float* sq, int J, float* scores, cudaStream_t st) {
   // At m = 256 or 512, one or two queries per group take the shift-window
   // digit kernel and three or four the class kernel (half the MMAs of two
-  // digit column tiles). The tcgen05 variant (QJL_SCORES_KERNEL=tc) computes
-  // the same sums on the 5th-gen tensor cores, but at about 48 cycles per
-  // 128x8x32 MMA its A-operand reads (one byte per sign bit) cap it below the
-  // mma.sync path; it is kept for comparison. QJL_SCORES_KERNEL=stream selects
-  // the generic streaming kernel.
-  static const int choice = [] {
-    const char* v = getenv("QJL_SCORES_KERNEL");
-    if (v && strcmp(v, "tc") == 0) return 1;
-    if (v && strcmp(v, "stream") == 0) return 2;
-    return 0;
-  }();
-  if (choice == 1 && scores_tc_supported(P->m, J)) return launch_scores_tc(P, bits, norms, G, N, sq, J, scores, st);
-  if (choice == 0 && J <= 2 && (P->m == 256 || P->m == 512))
+  // digit column tiles); more queries, or m = 1024, the generic streaming
+  // kernel.
+  if (J <= 2 && (P->m == 256 || P->m == 512))
     return P->m == 256 ? launch_digit_w<8>(P, bits, norms, G, N, sq, J, scores, st)
                        : launch_digit_w<16>(P, bits, norms, G, N, sq, J, scores, st);
-  if (choice == 0 && J <= 4 && (P->m == 256 || P->m == 512))
+  if (J <= 4 && (P->m == 256 || P->m == 512))
     return P->m == 256 ? launch_decode_fast<8>(P, bits, norms, G, N, sq, J, scores, st)
                        : launch_decode_fast<16>(P, bits, norms, G, N, sq, J, scores, st);
   const int NTR = J > 4 ? 2 : 1;

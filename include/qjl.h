@@ -227,8 +227,11 @@ qjl_status qjl_decode_attention(const qjl_projection* proj, const uint32_t* bits
  *   - Returns QJL_ERR_WORKSPACE, launching nothing, when
  *     qjl_decode_workspace_bytes(groups, q_per_group, N, d) exceeds that size.
  *   - The first call on each device resolves the array's device address
- *     (cudaGetSymbolAddress, with that device current). Make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress, with that device current), and that of the
+ *     kernels' error int, which is static device storage as well. Make that
+ *     first call before any stream capture. The cached addresses stay valid
+ *     for the life of the device's primary context: after cudaDeviceReset
+ *     the library must be reloaded.
  *   - All calls share the one array. Calls that overlap on the GPU (for
  *     example on two streams) race and give undefined results. Serialise
  *     them. Earlier calls' contents need no clearing: every workspace entry
@@ -384,11 +387,13 @@ qjl_status qjl_kivi_key_scores(const uint32_t* codes, const uint16_t* scale, con
 /*
  * Device-side errors. Kernels never trap. A bounded wait that expires (4 s of
  * wall time), or a paged-cache entry that is out of range, sets a bit in a
- * per-device int and the kernel winds down. The bits are:
+ * per-device int and the kernel winds down. The int is static device storage
+ * of the library (zero when the library loads on a device); no call allocates
+ * it. The bits are:
  *   1, 2, 4, 8, 16, 32  a bounded wait expired (1: a producer's wait for a
  *        free stage; 2: a final wait for a CTA's own copies; 4: a consumer's
- *        wait for a full stage; 8, 16, 32: the tcgen05 kernels' MMA-completion,
- *        TMEM and norm-warp waits)
+ *        wait for a full stage; 8, 16, 32: the tcgen05 quantize kernel's
+ *        MMA-completion, TMEM and norm-warp waits)
  *   64   a paged-cache position or block-table entry was out of range (skipped)
  *   128  qjl_selftest_bounded_wait's wait expired (as it should)
  * qjl_device_errors synchronises `device`, stores the int in *flags and, if

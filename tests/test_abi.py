@@ -108,3 +108,23 @@ def test_paged_and_prefill_calls_reject_a_null_projection(L):
     assert L.qjl_decode_attention_paged(None, z, z, z, z, z, z, 1, 16, 1, z, 1, 16, z, 1.0, z, z, 0, None) == -1
     assert L.qjl_prefill_attention(None, z, z, z, z, z, 1, 16, z, 1.0, z, None) == -1
     assert b"NULL" in L.qjl_last_error_message() or b"projection" in L.qjl_last_error_message()
+
+
+def test_only_projection_upload_allocates_device_memory():
+    """The library's one device allocation site is the projection's parameter upload.
+
+    Every other call works on caller-owned buffers, the fixed no-alloc scratch and
+    the static error int. A new cudaMalloc (or an allocating runtime call) anywhere
+    else in the sources fails this check.
+    """
+    import glob
+    import os
+    import re
+    csrc = os.path.join(os.path.dirname(_lib.__file__), "csrc")
+    sites = []
+    for path in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.h*"))):
+        for i, line in enumerate(open(path), 1):
+            code = line.split("//")[0]
+            if re.search(r"\bcuda(Malloc\w*|MallocAsync|MallocManaged|HostAlloc)\s*\(", code):
+                sites.append((os.path.basename(path), i))
+    assert len(sites) == 1 and sites[0][0] == "qjl_api.cu", sites
