@@ -38,11 +38,30 @@ def test_division_by_three_sampled():
         assert rn32(Fraction(float(q[i])) + Fraction(float(r[i])) * Fraction(float(THIRD))) == want[i]
 
 
+def _f32_midpoint(x64):
+    """True where a float64 value lies exactly halfway between two adjacent float32 values."""
+    x32 = x64.astype(np.float32)
+    lo = np.where(x32.astype(np.float64) > x64, np.nextafter(x32, np.float32(-np.inf)), x32)
+    hi = np.nextafter(lo, np.float32(np.inf))
+    return (lo.astype(np.float64) + hi.astype(np.float64)) * 0.5 == x64
+
+
 def test_reciprocal_step_all_fp16():
-    s_all = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float32)[::7]
-    for sv in s_all:
-        sv = np.float32(sv)
-        y = rn32(Fraction(1) / Fraction(float(sv)))
-        for y0 in (np.nextafter(y, np.float32(0)), y, np.nextafter(y, np.float32(np.inf))):
-            e = rn32(Fraction(1) - Fraction(float(sv)) * Fraction(float(y0)))
-            assert rn32(Fraction(float(y0)) + Fraction(float(e)) * Fraction(float(y0))) == y
+    """Every positive finite fp16 s, with y0 at RN(1/s) and both neighbours.
+
+    1 - s y0 is exact in float64 (an 11-bit by 24-bit product near 1), so e = RN32 of
+    it is exact too. y0 + e y0 is formed in float64 and rounded to float32; a case
+    whose float64 sum is a float32 midpoint (where double rounding could mislead) or
+    that disagrees is settled with exact rationals.
+    """
+    s = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float32)
+    y = np.float32(1.0) / s                                                 # IEEE RN(1/s)
+    for y0 in (np.nextafter(y, np.float32(0)), y, np.nextafter(y, np.float32(np.inf))):
+        e = (1.0 - s.astype(np.float64) * y0.astype(np.float64)).astype(np.float32)
+        t64 = y0.astype(np.float64) + e.astype(np.float64) * y0.astype(np.float64)
+        t = t64.astype(np.float32)
+        check = np.nonzero((t != y) | _f32_midpoint(t64))[0]
+        for i in check:
+            ee = rn32(Fraction(1) - Fraction(float(s[i])) * Fraction(float(y0[i])))
+            assert ee == e[i]
+            assert rn32(Fraction(float(y0[i])) + Fraction(float(ee)) * Fraction(float(y0[i]))) == y[i]
