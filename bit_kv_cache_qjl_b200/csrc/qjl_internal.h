@@ -109,7 +109,11 @@ std::vector<float> fqjl_key_tables(int d, int m, const float* D_r, const int32_t
 qjl_status launch_fqjl_keys(const qjl_projection* P, const void* keys, int dtype, int64_t n, int64_t ld,
                             uint64_t first_token, uint32_t* bits, float* norms, cudaStream_t st,
                             const PageMap& pm = PageMap());
-bool scores_mma_supported(int m);
+// many-query scores on tcgen05 (scores_many.cu): m in {256, 512, 1024}, J <= 64, N < 2^31 - 128
+// (a call of more keys than that in all is split by groups)
+bool scores_many_supported(int m, int64_t N);
+qjl_status launch_scores_many(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t G,
+                              int64_t N, const float* sq, int J, float* scores, cudaStream_t st);
 qjl_status launch_scores(const qjl_projection* P, const uint32_t* bits, const float* norms,
                          int64_t groups, int64_t N, const float* sq, int J, float* scores,
                          cudaStream_t st);

@@ -46,221 +46,6 @@ using namespace qjl_sign;
 
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
-constexpr int kConsumerWarps = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStageKeys = 256;
-constexpr int kTilesPerWarp = kStageKeys / 16 / kConsumerWarps;  // 4
-static_assert(kTilesPerWarp % 2 == 0, "tiles are consumed in pairs");
-
-// KT 16-key tiles of one stage (tiles tile0, tile0 + 8, ...), their MMAs
-// interleaved, written straight to `scores` from registers.
-template <int W, int NTR, int KT>
-__device__ __forceinline__ void consume_tiles(int tile0, const uint32_t* __restrict__ sb,
-                                              const float* __restrict__ sn, const float* __restrict__ nsrc,
-                                              bool nbulk, int cnt, const uint2* __restrict__ Btab,
-                                              const float* __restrict__ s_mul, const int* __restrict__ s_qsum,
-                                              int npass, int J, int64_t N, int64_t g, int64_t n0,
-                                              float* __restrict__ scores) {
-  const int lane = threadIdx.x & 31;
-  const int gq = lane >> 2, q = lane & 3;
-    int rr[KT][2];
-    uint32_t w0[KT][W / 4], w1[KT][W / 4];
-    float nrm[KT][2];
-#pragma unroll
-    for (int t2 = 0; t2 < KT; ++t2) {
-      const int tl = tile0 + t2 * kConsumerWarps;
-      rr[t2][0] = tl * 16 + gq;
-      rr[t2][1] = rr[t2][0] + 8;
-#pragma unroll
-      for (int kk = 0; kk < W / 8; ++kk) {
-        const uint2 a = (rr[t2][0] < cnt) ? *reinterpret_cast<const uint2*>(sb + rr[t2][0] * W + q * (W / 4) + 2 * kk)
-                                          : make_uint2(0, 0);
-        const uint2 b = (rr[t2][1] < cnt) ? *reinterpret_cast<const uint2*>(sb + rr[t2][1] * W + q * (W / 4) + 2 * kk)
-                                          : make_uint2(0, 0);
-        w0[t2][2 * kk] = a.x; w0[t2][2 * kk + 1] = a.y;
-        w1[t2][2 * kk] = b.x; w1[t2][2 * kk + 1] = b.y;
-      }
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-        nrm[t2][r] = rr[t2][r] < cnt ? (nbulk ? sn[rr[t2][r]] : __ldg(nsrc + rr[t2][r])) : 0.f;
-    }
-    if (tile0 * 16 < cnt) {
-      for (int pass = 0; pass < npass; ++pass) {
-        int acc[KT][NTR][4][4];
-#pragma unroll
-        for (int t2 = 0; t2 < KT; ++t2)
-#pragma unroll
-          for (int a = 0; a < NTR; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-#pragma unroll
-              for (int c = 0; c < 4; ++c) acc[t2][a][b][c] = 0;
-#pragma unroll
-        for (int p = 0; p < W / 8; ++p) {
-#pragma unroll
-          for (int sh = 0; sh < 2; ++sh) {
-            uint32_t x[KT][4];
-#pragma unroll
-            for (int t2 = 0; t2 < KT; ++t2) {
-              x[t2][0] = w0[t2][2 * p] >> sh;
-              x[t2][1] = w1[t2][2 * p] >> sh;
-              x[t2][2] = w0[t2][2 * p + 1] >> sh;
-              x[t2][3] = w1[t2][2 * p + 1] >> sh;
-            }
-#pragma unroll
-            for (int Ji = 0; Ji < 4; ++Ji) {
-              const uint32_t M = 0x01010101u << (2 * Ji);
-              const int mu = 8 * p + 2 * Ji + sh;
-#pragma unroll
-              for (int nt = 0; nt < NTR; ++nt) {
-                const uint2 bb = Btab[((pass * NTR + nt) * W + mu) * 32 + lane];
-#pragma unroll
-                for (int t2 = 0; t2 < KT; ++t2)
-                  mma_u8s8(acc[t2][nt][Ji], x[t2][0] & M, x[t2][1] & M, x[t2][2] & M, x[t2][3] & M, bb.x, bb.y);
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int nt = 0; nt < NTR; ++nt) {
-          const int jq = (pass * NTR + nt) * 4 + q;
-          if (jq >= J) continue;
-          const float mul = s_mul[jq] * 0.03125f;
-          const float qs32 = 32.f * (float)s_qsum[jq];
-          float* orow = scores + (g * J + jq) * N + n0;
-#pragma unroll
-          for (int t2 = 0; t2 < KT; ++t2) {
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const int row = rr[t2][r];
-              if (row >= cnt) continue;
-              const int hi = ((acc[t2][nt][0][2 * r] * 4 + acc[t2][nt][1][2 * r]) * 4 + acc[t2][nt][2][2 * r]) * 4 +
-                             acc[t2][nt][3][2 * r];
-              const int lo = ((acc[t2][nt][0][2 * r + 1] * 4 + acc[t2][nt][1][2 * r + 1]) * 4 +
-                              acc[t2][nt][2][2 * r + 1]) * 4 + acc[t2][nt][3][2 * r + 1];
-              // 32 * sum (2b - 1) Q in fp32: |hi| < 2^24 is exact, and the
-              // rounding of the sum is far below the 16-bit rounding of Sq
-              const float D = fmaf((float)hi, 256.f, (float)lo) - qs32;
-              orow[row] = mul * nrm[t2][r] * D;
-            }
-          }
-        }
-      }
-    }
-}
-
-// Streaming kernel. Persistent CTAs each take a contiguous range of work
-// items (group g, chunk of kStageKeys keys), g-major, so a CTA crosses at most
-// a few group boundaries. Warp 4 (one lane) is the producer. It moves each
-// chunk's packed bits, and its norms when they are 16-byte aligned, into an
-// NS-stage shared-memory ring with cp.async.bulk, completing on the stage's
-// mbarrier. Warps 0-3 consume: each takes four 16-key tiles of the stage,
-// runs the sign-sum MMAs against the group's B tables, and writes scores
-// straight from registers. At a group boundary the consumer warps rebuild
-// the tables behind a named barrier.
-template <int W, int NTR, int KT>
-__global__ void __launch_bounds__(kThreads, W == 8 ? 3 : 1) scores_stream_kernel(
-    const uint32_t* __restrict__ bits, const float* __restrict__ norms, const float* __restrict__ sq,
-    int64_t G, int64_t N, int J, int NS, float est_scale, int64_t items_per_cta, float* __restrict__ scores,
-    int* __restrict__ err) {
-  using namespace qjl_sync;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int NT = (J + 3) / 4;
-  const int npass = (NT + NTR - 1) / NTR;
-  const int NTP = npass * NTR;
-  float* s_inv = reinterpret_cast<float*>(smem_raw);
-  float* s_mul = s_inv + 64;
-  int* s_qsum = reinterpret_cast<int*>(s_mul + 64);
-  uint2* Btab = reinterpret_cast<uint2*>(smem_raw + 3 * 64 * 4);
-  uint32_t* sbits = reinterpret_cast<uint32_t*>(Btab + (size_t)NTP * W * 32);   // [NS][kStageKeys * W]
-  float* snorm = reinterpret_cast<float*>(sbits + (size_t)NS * kStageKeys * W); // [NS][kStageKeys]
-  uint64_t* full = reinterpret_cast<uint64_t*>(snorm + (size_t)NS * kStageKeys);
-  uint64_t* empty = full + NS;
-
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t cpg = (N + kStageKeys - 1) / kStageKeys;
-  const int64_t total = G * cpg;
-  const int64_t i0 = (int64_t)blockIdx.x * items_per_cta;
-  const int64_t i1 = min(total, i0 + items_per_cta);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
-    }
-    mbar_fence_init();
-  }
-  __syncthreads();
-
-  if (warp == kConsumerWarps) {
-    if (lane == 0) {
-      // incremental (group, chunk) and (stage, phase): no 64-bit division in the loop
-      int64_t g = i0 / cpg, c = i0 - (i0 / cpg) * cpg;
-      int s = 0;
-      uint32_t ph = 0;
-      int64_t issued = 0;
-      for (int64_t it = i0; it < i1; ++it, ++issued) {
-        if (!mbar_wait(&empty[s], ph ^ 1u)) { atomicOr(err, 1); break; }
-        const int64_t n0 = c * kStageKeys;
-        const int cnt = (int)(N - n0 < kStageKeys ? N - n0 : kStageKeys);
-        const float* nsrc = norms + g * N + n0;
-        const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
-        const uint32_t bbytes = (uint32_t)cnt * W * 4;
-        mbar_expect_tx(&full[s], bbytes + (nbulk ? (uint32_t)cnt * 4 : 0u));
-        bulk_g2s(sbits + (size_t)s * kStageKeys * W, bits + (g * N + n0) * W, bbytes, &full[s]);
-        if (nbulk) bulk_g2s(snorm + (size_t)s * kStageKeys, nsrc, (uint32_t)cnt * 4, &full[s]);
-        if (++c == cpg) { c = 0; ++g; }
-        if (++s == NS) { s = 0; ph ^= 1u; }
-      }
-      // every copy issued into a stage has landed before the CTA exits: the
-      // most recent phase of each used stage is waited on again
-      const int used = issued < NS ? (int)issued : NS;
-      for (int j = 0; j < used; ++j) {
-        // stage (s - 1 - j) mod NS; its last phase parity flips when we wrap back past 0
-        int st = s - 1 - j;
-        uint32_t p = ph;
-        if (st < 0) { st += NS; p ^= 1u; }
-        if (!mbar_wait(&full[st], p)) atomicOr(err, 2);
-      }
-    }
-    return;
-  }
-
-  // consumers
-  int64_t cur_g = -1;
-  int64_t g = i0 / cpg, c = i0 - (i0 / cpg) * cpg;
-  int s = 0;
-  uint32_t ph = 0;
-  bool dead = false;  // a timed-out wait: keep the loop's barriers, skip the work
-  for (int64_t it = i0; it < i1; ++it) {
-    const int64_t n0 = c * kStageKeys;
-    const int cnt = (int)(N - n0 < kStageKeys ? N - n0 : kStageKeys);
-    if (g != cur_g) {
-      named_sync(1, kConsumerWarps * 32);
-      build_tables<W>(sq + g * (int64_t)J * (32 * W), J, NTP, est_scale, s_inv, s_mul, s_qsum, Btab,
-                      kConsumerWarps, 1);
-      cur_g = g;
-    }
-    if (!dead && !__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { atomicOr(err, 4); dead = true; }
-    if (!dead) {
-    const float* nsrc = norms + g * N + n0;
-    const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
-    const uint32_t* sb = sbits + (size_t)s * kStageKeys * W;
-    const float* sn = snorm + (size_t)s * kStageKeys;
-    // this warp's tiles of the stage, KT at a time (KT = 2 interleaves two
-    // tiles' MMAs for ILP where registers allow)
-#pragma unroll 1
-    for (int i = 0; i < kTilesPerWarp; i += KT)
-      consume_tiles<W, NTR, KT>(warp + i * kConsumerWarps, sb, sn, nsrc, nbulk, cnt, Btab, s_mul, s_qsum, npass, J,
-                                N, g, n0, scores);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-    if (++c == cpg) { c = 0; ++g; }
-    if (++s == NS) { s = 0; ph ^= 1u; }
-  }
-}
-
 // Decode fast path: at most 4 queries per group (one n8 column tile), so each
 // consumer thread keeps its B fragments in registers (2 W of them), loaded
 // from the shared table once per group. The first MMA of each accumulator
@@ -495,6 +280,14 @@ __device__ __forceinline__ void digit_epilogue(const int (&acc)[KT][NT][4], int 
 
 // PAGED reads group g's tokens t < seq_lens[g] through the block table
 // (PagedRead); N is then the bound max_len, and the row stride of scores.
+//
+// Shared memory: the per-query constants, the B fragments, NS stages of
+// [SK keys x W words] bits and [SK] norms, one slot for a group's Sq rows
+// ([J][m] fp32) and the barriers. The producer copies each new group's Sq
+// rows into the slot with that group's first stage, once the consumers have
+// signalled (slot_free) that the previous group's table is built; the table
+// build then reuses the slot for its packed digits and the B fragments'
+// space for the quantised Sq.
 template <int W, int NT, bool DUP, int KT, int SKT, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
     const uint32_t* __restrict__ bits, const float* __restrict__ norms, const float* __restrict__ sq,
@@ -502,44 +295,58 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
     int* __restrict__ err, PagedRead pr) {
   using namespace qjl_sync;
   constexpr int SK = SKT;
+  constexpr int m = 32 * W;
   constexpr int TPW = SK / 16 / kDecConsumers;  // tiles per consumer warp per stage
   static_assert(!DUP || NT == 1, "DUP is the one-query layout");
   static_assert(TPW % KT == 0 && (KT == 2 || KT == 4), "KT tiles per batch");
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* s_inv = reinterpret_cast<float*>(smem_raw);
-  float* s_mul = s_inv + 64;
+  float* s_mul = reinterpret_cast<float*>(smem_raw);
   int* s_qsum = reinterpret_cast<int*>(s_mul + 64);
-  uint2* Btab = reinterpret_cast<uint2*>(smem_raw + 3 * 64 * 4 + 256);       // [NT][W][32]
+  uint2* Btab = reinterpret_cast<uint2*>(s_qsum + 64);                       // [NT][W][32]
   uint32_t* sbits = reinterpret_cast<uint32_t*>(Btab + (size_t)NT * W * 32);  // [NS][SK * W]
   float* snorm = reinterpret_cast<float*>(sbits + (size_t)NS * SK * W);     // [NS][SK]
-  uint64_t* full = reinterpret_cast<uint64_t*>(snorm + (size_t)NS * SK);
+  float* ssq = snorm + (size_t)NS * SK;                                      // [J * m]
+  uint64_t* full = reinterpret_cast<uint64_t*>(ssq + (size_t)J * m);
   uint64_t* empty = full + NS;
+  uint64_t* slot_free = empty + NS;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t cpg = (N + SK - 1) / SK;
   const int64_t total = G * cpg;
   const int64_t i0 = (int64_t)blockIdx.x * items_per_cta;
   const int64_t i1 = min(total, i0 + items_per_cta);
+  const uint32_t sq_bytes = (uint32_t)J * m * 4;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kDecConsumers);
     }
+    mbar_init(slot_free, 1);
     mbar_fence_init();
   }
   __syncthreads();
 
   if (warp == kDecConsumers) {
     if (lane == 0) {
-      // items newest first (see the consumer loop)
-      int64_t g = (i1 - 1) / cpg, c = (i1 - 1) - ((i1 - 1) / cpg) * cpg;
+      int64_t g = i0 / cpg, c = i0 - (i0 / cpg) * cpg;
+      int64_t prev_g = -1;
+      uint32_t sph = 0;  // parity of the slot's next release
       int s = 0;
       uint32_t ph = 0;
       int64_t issued = 0;
       for (int64_t it = i0; it < i1; ++it, ++issued) {
         if (!mbar_wait(&empty[s], ph ^ 1u)) { atomicOr(err, 1); break; }
         const int64_t n0 = c * SK;
+        // the first stage of each group this CTA visits also brings the group's Sq rows,
+        // into the slot the previous group's table build has released
+        const bool new_group = g != prev_g;
+        prev_g = g;
+        if (new_group) {
+          if (!mbar_wait(slot_free, sph ^ 1u)) { atomicOr(err, 1); break; }
+          sph ^= 1u;
+        }
+        const uint32_t tx_sq = new_group ? sq_bytes : 0u;
         if constexpr (PAGED) {
           // the stage's tokens [n0, n0 + cnt) of group g, one copy per page segment, each
           // rounded up to 4 tokens (16 bytes of norms; never past the page, which holds a
@@ -547,9 +354,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
           const int64_t Lg = min64(max64(__ldg(pr.seq_lens + g), 0), N);
           const int cnt = (int)max64(0, min64(SK, Lg - n0));
           const int T = pr.page_tokens;
-          uint32_t tx = 0;
+          uint32_t tx = tx_sq;
           for (int pass = 0; pass < 2; ++pass) {
-            if (pass == 1) mbar_expect_tx(&full[s], tx);
+            if (pass == 1) {
+              mbar_expect_tx(&full[s], tx);
+              if (new_group) bulk_g2s(ssq, sq + g * (int64_t)J * m, sq_bytes, &full[s]);
+            }
             for (int64_t lo = n0; lo < n0 + cnt;) {
               const int64_t pi = lo / T;
               const int64_t hi = min64(n0 + cnt, (pi + 1) * T);
@@ -574,11 +384,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
           const float* nsrc = norms + g * N + n0;
           const bool nbulk = (((uintptr_t)nsrc & 15u) == 0) && (cnt % 4 == 0);
           const uint32_t bbytes = (uint32_t)cnt * W * 4;
-          mbar_expect_tx(&full[s], bbytes + (nbulk ? (uint32_t)cnt * 4 : 0u));
+          mbar_expect_tx(&full[s], bbytes + (nbulk ? (uint32_t)cnt * 4 : 0u) + tx_sq);
           bulk_g2s(sbits + (size_t)s * SK * W, bits + (g * N + n0) * W, bbytes, &full[s]);
           if (nbulk) bulk_g2s(snorm + (size_t)s * SK, nsrc, (uint32_t)cnt * 4, &full[s]);
+          if (new_group) bulk_g2s(ssq, sq + g * (int64_t)J * m, sq_bytes, &full[s]);
         }
-        if (c == 0) { c = cpg - 1; --g; } else { --c; }
+        if (++c == cpg) { c = 0; ++g; }
         if (++s == NS) { s = 0; ph ^= 1u; }
       }
       const int used = issued < NS ? (int)issued : NS;
@@ -593,13 +404,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
   }
 
   const int gq = lane >> 2, q = lane & 3, par = q & 1, half = q >> 1;
-  // Each CTA walks its items newest first. When the keys were sketched just
-  // before (a whole-cache quantize, then scores), the tail of the bits array
-  // is still in L2, and reading it first takes it before the next reads
-  // evict it. Stage bookkeeping is incremental and 32-bit where it can be:
-  // chunk c of group g, with the norms and output pointers stepped per stage.
-  int64_t g = (i1 - 1) / cpg;
-  int c = (int)((i1 - 1) - g * cpg);
+  // Each CTA walks its contiguous range of (group, stage) items in order.
+  // Stage bookkeeping is incremental and 32-bit where it can be: chunk c of
+  // group g, with the norms and output pointers stepped per stage.
+  int64_t g = i0 / cpg;
+  int c = (int)(i0 - g * cpg);
   const int cpg32 = (int)cpg;
   const int last_cnt = (int)(N - (cpg - 1) * SK);
   const bool groups_aligned = ((((uintptr_t)norms) & 15u) == 0) && (N % 4 == 0);
@@ -618,10 +427,14 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
     if (PAGED && g != cur_g) Lg = min64(max64(__ldg(pr.seq_lens + g), 0), N);
     const int cnt = PAGED ? (int)max64(0, min64(SK, Lg - (int64_t)c * SK))
                           : (c == cpg32 - 1 ? last_cnt : SK);
+    if (!dead && !__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { atomicOr(err, 4); dead = true; }
     if (g != cur_g) {
+      // every consumer warp takes part (dead or not), so the named barriers stay matched
       named_sync(1, kDecConsumers * 32);
-      build_tables_dig<W>(sq + g * (int64_t)J * (32 * W), J, NT, DUP, est_scale, s_inv, s_mul, s_qsum, Btab,
-                          kDecConsumers, 1);
+      // the slot's Sq rows become the digit scratch, Btab's space holds Q until phase 3
+      build_tables_dig_smem<W>(ssq, J, NT, DUP, est_scale, s_mul, s_qsum, reinterpret_cast<int*>(Btab),
+                               reinterpret_cast<uint32_t*>(ssq), Btab, kDecConsumers, 1);
+      if (threadIdx.x == 0) mbar_arrive(slot_free);  // the build's last barrier: nobody reads the slot now
       if constexpr (NT == 1) {
 #pragma unroll
         for (int mu = 0; mu < W; ++mu) breg[mu] = Btab[mu * 32 + lane];
@@ -634,7 +447,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
       }
       cur_g = g;
     }
-    if (!dead && !__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { atomicOr(err, 4); dead = true; }
     if (!dead) {
       // the producer bulk-copied the norms exactly when they were 16-byte aligned
       // and a multiple of 4; otherwise they are read from global memory
@@ -708,15 +520,14 @@ __global__ void __launch_bounds__(kDecThreads, 2) scores_digit_kernel(
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-    if (c == 0) {
-      c = cpg32 - 1;
-      --g;
-      nsrc = norms + g * N + (int64_t)c * SK;
-      gout = scores + g * (int64_t)J * N + (int64_t)c * SK;
+    if (++c == cpg32) {
+      c = 0;
+      ++g;
+      nsrc = norms + g * N;
+      gout = scores + g * (int64_t)J * N;
     } else {
-      --c;
-      nsrc -= SK;
-      gout -= SK;
+      nsrc += SK;
+      gout += SK;
     }
     if (++s == NS) { s = 0; ph ^= 1u; }
   }
@@ -746,38 +557,6 @@ __global__ void __launch_bounds__(256) scores_simt_kernel(
       if (lane == 0) scores[(gi * J + j) * N + row] = est_scale * nrm * acc;
     }
   }
-}
-
-size_t stream_smem(int W, int NTP, int NS) {
-  return 3 * 64 * 4 + (size_t)NTP * W * 32 * sizeof(uint2) + (size_t)NS * kStageKeys * (W + 1) * 4 +
-         (size_t)2 * NS * 8;
-}
-
-template <int W, int NTR>
-qjl_status launch_mma(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t G,
-                      int64_t N, const float* sq, int J, float* scores, cudaStream_t st) {
-  const int NT = (J + 3) / 4;
-  const int NTP = ((NT + NTR - 1) / NTR) * NTR;
-  int NS = W <= 8 ? 4 : (W <= 16 ? 3 : 2);
-  while (NS > 2 && stream_smem(W, NTP, NS) > 200 * 1024) --NS;
-  const size_t smem = stream_smem(W, NTP, NS);
-  auto kern = scores_stream_kernel<W, NTR, (W <= 16 && NTR == 1) ? 2 : 1>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
-      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
-    return qjl_check_launch("scores_stream_kernel smem attribute");
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess || per_sm < 1)
-    return qjl_check_launch("scores_stream_kernel occupancy");
-  int* err = qjl_error_flag(P->device);
-  if (!err) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
-  const int64_t total = G * ((N + kStageKeys - 1) / kStageKeys);
-  const int64_t slots = (int64_t)qjl_num_sms(P->device) * per_sm;
-  const int64_t grid = std::min<int64_t>(total, slots);
-  const int64_t ipc = (total + grid - 1) / grid;
-  const int64_t nblk = (total + ipc - 1) / ipc;
-  qjl_log_launch("scores_stream_kernel", nblk, kThreads, smem, per_sm);
-  kern<<<(unsigned)nblk, kThreads, smem, st>>>(bits, norms, sq, G, N, J, NS, P->est_scale, ipc, scores, err);
-  return qjl_check_launch("scores_stream_kernel");
 }
 
 template <int W>
@@ -811,9 +590,11 @@ template <int W, int NT, bool DUP, int KT, int SKT, bool PAGED = false>
 qjl_status launch_digit(const qjl_projection* P, const uint32_t* bits, const float* norms, int64_t G, int64_t N,
                         const float* sq, int J, float* scores, cudaStream_t st, const PagedRead& pr = PagedRead()) {
   // ring depth: as many stages as keep two CTAs per SM within shared memory
-  const int NS = SKT * (W + 1) * 4 * 4 <= 80 * 1024 ? 4 : (SKT * (W + 1) * 4 * 3 <= 110 * 1024 ? 3 : 2);
-  const size_t smem = 3 * 64 * 4 + 256 + (size_t)NT * W * 32 * sizeof(uint2) + (size_t)NS * SKT * (W + 1) * 4 +
-                      (size_t)2 * NS * 8;
+  const size_t stage = (size_t)SKT * (W + 1) * 4;  // bits and norms
+  const int NS = stage * 4 <= 80 * 1024 ? 4 : (stage * 3 <= 110 * 1024 ? 3 : 2);
+  const size_t smem = 2 * 64 * 4 + (size_t)NT * W * 32 * sizeof(uint2) + (size_t)NS * stage +
+                      (size_t)J * 32 * W * 4 + (size_t)(2 * NS + 1) * 8;
+  static_assert((size_t)NT * W * 32 * sizeof(uint2) >= (size_t)2 * 32 * W * 4, "Q scratch fits in Btab (J <= 2)");
   auto kern = scores_digit_kernel<W, NT, DUP, KT, SKT, PAGED>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
@@ -845,30 +626,20 @@ qjl_status launch_digit_w(const qjl_projection* P, const uint32_t* bits, const f
 
 }  // namespace
 
-bool scores_mma_supported(int m) { return m == 256 || m == 512 || m == 1024; }
-
 qjl_status launch_scores(const qjl_projection* P, const uint32_t* bits, const float* norms,
                          int64_t G, int64_t N, const float* sq, int J, float* scores, cudaStream_t st) {
   // At m = 256 or 512, one or two queries per group take the shift-window
   // digit kernel and three or four the class kernel (half the MMAs of two
-  // digit column tiles); more queries, or m = 1024, the generic streaming
-  // kernel.
+  // digit column tiles). More queries, or m = 1024, are a contraction for the
+  // tcgen05 kernel (scores_many.cu). Other m, and one group of more than 2^31
+  // keys, take the SIMT kernel.
   if (J <= 2 && (P->m == 256 || P->m == 512))
     return P->m == 256 ? launch_digit_w<8>(P, bits, norms, G, N, sq, J, scores, st)
                        : launch_digit_w<16>(P, bits, norms, G, N, sq, J, scores, st);
   if (J <= 4 && (P->m == 256 || P->m == 512))
     return P->m == 256 ? launch_decode_fast<8>(P, bits, norms, G, N, sq, J, scores, st)
                        : launch_decode_fast<16>(P, bits, norms, G, N, sq, J, scores, st);
-  const int NTR = J > 4 ? 2 : 1;
-  switch (scores_mma_supported(P->m) ? P->m : 0) {
-    case 256: return NTR == 1 ? launch_mma<8, 1>(P, bits, norms, G, N, sq, J, scores, st)
-                              : launch_mma<8, 2>(P, bits, norms, G, N, sq, J, scores, st);
-    case 512: return NTR == 1 ? launch_mma<16, 1>(P, bits, norms, G, N, sq, J, scores, st)
-                              : launch_mma<16, 2>(P, bits, norms, G, N, sq, J, scores, st);
-    case 1024: return NTR == 1 ? launch_mma<32, 1>(P, bits, norms, G, N, sq, J, scores, st)
-                               : launch_mma<32, 2>(P, bits, norms, G, N, sq, J, scores, st);
-    default: break;
-  }
+  if (scores_many_supported(P->m, N)) return launch_scores_many(P, bits, norms, G, N, sq, J, scores, st);
   const int64_t want = (G * N + 7) / 8;
   const int blocks = (int)std::min<int64_t>(want, (int64_t)qjl_num_sms(P->device) * 16);
   scores_simt_kernel<<<blocks, 256, 0, st>>>(bits, norms, sq, G, N, J, P->m / 32, P->est_scale, scores);

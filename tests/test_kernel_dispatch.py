@@ -62,9 +62,14 @@ def test_scores_and_projection_kernels(cuda_ok):
     # three or four: the weight-class kernel
     sq4 = torch.ones((4, 4, 256), device="cuda")
     assert _has(_kernels(lambda: qjl.scores(P, bits, norms, sq4)), "scores_decode_kernel")
-    # more than 4 queries per group take the streaming mma.sync kernel
+    # more than 4 queries per group are a contraction for the tcgen05 kernel
     sq8 = torch.ones((4, 8, 256), device="cuda")
-    assert _has(_kernels(lambda: qjl.scores(P, bits, norms, sq8)), "scores_stream_kernel")
+    assert _has(_kernels(lambda: qjl.scores(P, bits, norms, sq8)), "scores_many_kernel")
+    # and so is any query count at m = 1024
+    P1k = qjl.Projection(2, 128, 1024, "dense")
+    b1k = torch.zeros((4, 1000, 32), dtype=torch.int32, device="cuda")
+    sq1 = torch.ones((4, 1, 1024), device="cuda")
+    assert _has(_kernels(lambda: qjl.scores(P1k, b1k, norms, sq1)), "scores_many_kernel")
 
 
 def test_values_and_decode_kernels(cuda_ok):

@@ -1,8 +1,9 @@
 """Estimator kernels vs the oracle, fed the oracle's bits and norms.
 
 Tolerance: |gpu - oracle| <= 1e-3 * c * alpha * ||k|| * ||Sq||_1 per score.
-Covers the tensor-core kernel (m = 256, 512, 1024) and the SIMT kernel for
-other m, with 1..64 queries per group, several groups, ragged N and N = 1.
+Covers the mma.sync kernels (one to four queries per group at m = 256, 512),
+the tcgen05 kernel (more queries, or m = 1024) and the SIMT kernel for other
+m, with 1..64 queries per group, several groups, ragged N and N = 1.
 """
 
 import numpy as np
@@ -47,6 +48,17 @@ def _case(kind, d, m, G, J, N, seed=0):
                                      (512, 2, 2, 1030), (256, 7, 1, 2051)])
 def test_scores_tensor_core(cuda_ok, m, G, J, N):
     _case("dense", 128, m, G, J, N)
+
+
+# the tcgen05 many-query kernel (more than four queries per group, or m = 1024): every column
+# width (8, 16, 32, 64 query slots), ragged tiles, N = 1, and more tiles than CTAs so that a CTA
+# spans several groups and rebuilds its tables (two table buffers at m <= 512, one at m = 1024
+# with 64 query slots)
+@pytest.mark.parametrize("m,G,J,N", [(256, 300, 33, 200), (1024, 200, 64, 130), (512, 7, 12, 1000),
+                                     (1024, 3, 5, 4096), (256, 3, 64, 1), (512, 1, 64, 2049),
+                                     (1024, 1, 2, 130), (512, 400, 20, 129), (256, 2, 8, 127)])
+def test_scores_tcgen05_many(cuda_ok, m, G, J, N):
+    _case("dense", 128, m, G, J, N, seed=m + G + J + N)
 
 
 @pytest.mark.parametrize("m,G,J,N", [(64, 2, 3, 100), (128, 1, 1, 50), (320, 1, 2, 41)])
