@@ -37,6 +37,7 @@
 
 #include <mutex>
 
+#include "cache_hint.cuh"
 #include "qjl_internal.h"
 
 namespace {
@@ -363,11 +364,11 @@ __global__ void __launch_bounds__(kThreads, 1) dense_tc_kernel(const __grid_cons
           uint32_t wq[4];
           tmem_ld128_pack(taddr, wq);
           if (row < prm.n)
-            *reinterpret_cast<uint4*>(prm.bits + row * W + c * 8 + half * 4) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+            qjl_hint::st_v4(prm.bits + row * W + c * 8 + half * 4, wq[0], wq[1], wq[2], wq[3], qjl_hint::evict_first());
         } else {
           uint32_t w0, w1;
           tmem_ld64_pack(taddr, w0, w1);
-          if (row < prm.n) *reinterpret_cast<uint2*>(prm.bits + row * W + c * 8 + half * 2) = make_uint2(w0, w1);
+          if (row < prm.n) qjl_hint::st_v2(prm.bits + row * W + c * 8 + half * 2, w0, w1, qjl_hint::evict_first());
         }
         tc_fence_before();
         __syncwarp();
@@ -409,7 +410,9 @@ __global__ void __launch_bounds__(kThreads, 1) dense_tc_kernel(const __grid_cons
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int64_t row = t * BM + r0 + 64 * j;
-        if (row < prm.n) prm.norms[row] = sqrtf((acc[j][0] + acc[j][1]) + (acc[j][2] + acc[j][3]));
+        if (row < prm.n)
+          qjl_hint::st_f32(prm.norms + row, sqrtf((acc[j][0] + acc[j][1]) + (acc[j][2] + acc[j][3])),
+                           qjl_hint::evict_first());
       }
       if (++s == NS) { s = 0; ph ^= 1u; }
     }

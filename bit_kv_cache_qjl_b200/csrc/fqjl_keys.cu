@@ -48,6 +48,7 @@
 
 #include "mbarrier.cuh"
 #include "philox.h"
+#include "cache_hint.cuh"
 #include "qjl_internal.h"
 
 namespace {
@@ -423,11 +424,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
             const float y = (r < E / 2) ? V[r].x : V[r - E / 2].y;
             acc = __funnelshift_l(__float_as_uint(y), acc, 1);
           }
-          out[w] = ~acc;
+          qjl_hint::st_u32(out + w, ~acc, qjl_hint::evict_first());
         }
       }
     }
-    if (valid && s == 0 && a.norms) a.norms[orow] = norm;
+    if (valid && s == 0 && a.norms) qjl_hint::st_f32(a.norms + orow, norm, qjl_hint::evict_first());
     // fetch the next batch into the same buffer (issuing it at the end of the batch measured
     // faster than right after the last read of the staged rows)
     __syncwarp();

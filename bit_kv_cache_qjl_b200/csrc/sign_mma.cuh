@@ -325,4 +325,90 @@ __device__ void build_tables_dig(const float* __restrict__ sqg, int J, int NT, b
   named_barrier_or_sync(bar_id, nthreads);
 }
 
+// build_tables_dig from a shared-memory copy of the group's Sq rows (sSq,
+// [J][m] fp32), quantising each value once. Scratch: sQ and sDig, [J][m]
+// 32-bit words each; sDig may be sSq itself (phase 2 starts after the last
+// read of sSq), and sQ may share Btab's space (phase 3 reads only sDig).
+// Three phases, each closed by the named barrier:
+//   1. per query (one warp each): max |Sq|, the grid scale, Q for every
+//      coordinate into sQ, and sum Q;
+//   2. per coordinate i: the residue B_i (mod 2^32) of its window, stored as
+//      its four balanced base-256 digits, digit dg in byte dg of sDig;
+//   3. per B fragment entry: eight digit bytes gathered from sDig.
+// The entries are those of build_tables_dig (same layout and values).
+template <int W>
+__device__ void build_tables_dig_smem(const float* sSq, int J, int NT, bool dup, float est_scale, float* s_mul,
+                                      int* s_qsum, int* sQ, uint32_t* sDig, uint2* Btab, int nwarps, int bar_id) {
+  static_assert(W % 8 == 0, "whole MMA k-steps");
+  constexpr int m = 32 * W;
+  constexpr int Qm = qmax_dig(m);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nthreads = 32 * nwarps;
+  for (int j = warp; j < J; j += nwarps) {
+    const float* row = sSq + j * m;
+    float mx = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < W; ++k) mx = fmaxf(mx, fabsf(row[32 * k + lane]));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float inv = mx > 0.f ? (float)Qm / mx : 0.f;
+    int qs = 0;
+#pragma unroll 4
+    for (int k = 0; k < W; ++k) {
+      const int q = quant_dig(row[32 * k + lane], inv, Qm);
+      sQ[j * m + 32 * k + lane] = q;
+      qs += q;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+    if (lane == 0) {
+      s_mul[j] = est_scale * (mx > 0.f ? mx / (float)Qm : 0.f);
+      s_qsum[j] = qs;
+    }
+  }
+  named_barrier_or_sync(bar_id, nthreads);
+  for (int idx = threadIdx.x; idx < J * m; idx += nthreads) {
+    const int i = idx & 31;              // coordinate within its sign word
+    const int* Qw = sQ + (idx - i);      // that word's 32 values
+    uint32_t B = 0u;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int t = i - 8 * k;
+      if (t < 0) break;
+      const int v = Qw[t] - (t > 0 ? 2 * Qw[t - 1] : 0);
+      B += (uint32_t)v << (8 * k);
+    }
+    uint32_t packed = 0u;
+#pragma unroll
+    for (int dg = 0; dg < 4; ++dg) {
+      const int d = (int)(int8_t)(B & 0xFFu);
+      packed |= ((uint32_t)d & 0xFFu) << (8 * dg);
+      B = (B - (uint32_t)d) >> 8;
+    }
+    sDig[idx] = packed;
+  }
+  named_barrier_or_sync(bar_id, nthreads);
+  const int entries = NT * W * 32;
+  for (int idx = threadIdx.x; idx < entries; idx += nthreads) {
+    const int ln = idx & 31;
+    const int mu = (idx >> 5) % W;
+    const int nt = (idx >> 5) / W;
+    const int n = ln >> 2, qq = ln & 3;
+    const int jq = dup ? 0 : nt * 2 + (n >> 2);
+    const int dg = n & 3;
+    const int p = mu >> 3, s = mu & 7;
+    uint32_t b[2] = {0u, 0u};
+    if (jq < J) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const uint32_t* Dw = sDig + jq * m + 32 * (qq * (W / 4) + 2 * p + r);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) b[r] |= ((Dw[8 * e + s] >> (8 * dg)) & 0xFFu) << (8 * e);
+      }
+    }
+    Btab[idx] = make_uint2(b[0], b[1]);
+  }
+  named_barrier_or_sync(bar_id, nthreads);
+}
+
 }  // namespace qjl_sign
