@@ -78,53 +78,90 @@ def ncu_traffic(kernel, workload, src):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled around a timed region.
+
+    A reader thread collects samples every `period_ms`. Entering waits (up to 5 s) for the first
+    sample, so the region is never timed before sampling runs; mark() records the region's start
+    and end on the host clock, and leaving waits for one sample past the end. The summary takes the
+    samples that fall in the region plus the last one before it and the first one after it, so a
+    region shorter than the period is still bracketed by two samples under load.
+    """
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
+    def __init__(self, index, period_ms=50):
+        self.index, self.period_ms = index, period_ms
+        self.proc, self.samples, self.marks = None, [], []
+        import threading
+        self._cv = threading.Condition()
 
-    def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
-                                          "--format=csv,noheader,nounits", "-lms", "20"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-        return self
-
-    def __exit__(self, *a):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
-
-    def summary(self):
-        mhz, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
-            f = [x.strip() for x in l.split(",")]
+    def _reader(self):
+        for line in self.proc.stdout:
+            f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
             try:
-                mhz.append(float(f[1]))
-                mx = float(f[2])
+                mhz, mx = float(f[1]), float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(mhz)}
+            reasons = [n for n, v in zip(self.NAMES, f[5:9]) if v.lower() == "active"]
+            with self._cv:
+                self.samples.append((time.monotonic(), mhz, mx, reasons))
+                self._cv.notify_all()
+
+    def _wait_for(self, count, timeout):
+        with self._cv:
+            self._cv.wait_for(lambda: len(self.samples) >= count, timeout=timeout)
+
+    def __enter__(self):
+        import threading
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return self
+        threading.Thread(target=self._reader, daemon=True).start()
+        self._wait_for(1, 5.0)
+        return self
+
+    def mark(self):
+        """Record the host time of a region boundary (call after a synchronize)."""
+        self.marks.append(time.monotonic())
+
+    def __exit__(self, *a):
+        if self.proc is None:
+            return
+        with self._cv:
+            n = len(self.samples)
+        self._wait_for(n + 1, 2.0)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+
+    def summary(self):
+        with self._cv:
+            smp = list(self.samples)
+        if len(self.marks) >= 2:
+            t0, t1 = self.marks[0], self.marks[-1]
+            inside = [s for s in smp if t0 <= s[0] <= t1]
+            before = [s for s in smp if s[0] < t0][-1:]
+            after = [s for s in smp if s[0] > t1][:1]
+            use = before + inside + after
+            region_ms = 1e3 * (t1 - t0)
+        else:
+            use, inside, region_ms = smp, smp, None
+        reasons = sorted({r for s in use for r in s[3]})
+        return {"sm_mhz": statistics.median([s[1] for s in use]) if use else None,
+                "sm_max_mhz": use[-1][2] if use else None, "reasons": reasons, "samples": len(use),
+                "samples_inside": len(inside), "region_ms": region_ms, "period_ms": self.period_ms,
+                "rule": "samples inside the timed region plus the last before and the first after it"}
 
 
 def dist_setup(backend=None):
@@ -170,26 +207,124 @@ def job_throughput(units_per_rank, world, ms_step_max):
     return world * units_per_rank / (ms_step_max * 1e-3)
 
 
-def cpu_oracle_rate(sample_keys, seconds_hint=None):
-    """Time the oracle (as it stands) on `sample_keys` keys of the workload: keys/s, threads."""
+_ORACLE_PROJ = {}
+
+
+def oracle_prepare(name, units):
+    """The oracle's path over a `units`-sized slice of workload `name`, ready to run: the projection
+    is drawn and the inputs generated here (setup, not timed). Returns (run, units): run() takes
+    every step of that workload's path in the fp64 oracle, as it stands."""
     import numpy as np
-    from threadpoolctl import threadpool_info
 
     import oracle
     from bit_kv_cache_qjl_b200 import workloads as wl
-    O = oracle.params.make_projection(2, D, M, oracle.params.KIND_DENSE, s_bf16=True)
-    heads = max(1, sample_keys // N)
-    per = min(N, sample_keys)
-    keys = wl.llama_keys("cpu", B=1, H=heads, N=per).reshape(heads, per, D).to("cpu").float().numpy()
-    q = wl.llama_queries("cpu", B=1, H=heads).reshape(heads, D).numpy()
-    t0 = time.perf_counter()
-    for h in range(heads):
-        words, norms, _ = oracle.qjl.quantize_keys(O, keys[h].astype(np.float64))
-        sq = oracle.qjl.project_queries(O, q[h:h + 1].astype(np.float64))
-        oracle.qjl.scores(O, words[None], norms[None], sq[None])
-    dt = time.perf_counter() - t0
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return heads * per / dt, dt, threads, heads * per
+
+    class P:                                       # the oracle's projections, drawn once per process
+        KIND_DENSE, KIND_DFQJL, KIND_PFQJL = (oracle.params.KIND_DENSE, oracle.params.KIND_DFQJL,
+                                              oracle.params.KIND_PFQJL)
+
+        @staticmethod
+        def make_projection(*a, **k):
+            key = (a, tuple(sorted(k.items())))
+            if key not in _ORACLE_PROJ:
+                _ORACLE_PROJ[key] = oracle.params.make_projection(*a, **k)
+            return _ORACLE_PROJ[key]
+    if name == "dense_1head":
+        O = P.make_projection(1, D, M, P.KIND_DENSE, s_bf16=False)
+        n = max(16, min(units, 4096))
+        keys, q = wl.dense_1head("cpu", n=n)
+        keys, q = keys.double().numpy(), q.double().numpy()
+
+        def run():
+            words, norms, _ = oracle.qjl.quantize_keys(O, keys)
+            sq = oracle.qjl.project_queries(O, q)
+            oracle.qjl.scores(O, words[None], norms[None], sq[None])
+        return run, n
+    if name in ("decode_llama7b", "gqa_decode"):
+        dense = name == "decode_llama7b"
+        m, J = (M, 1) if dense else (512, 4)
+        O = P.make_projection(2 if dense else 3, D, m, P.KIND_DENSE, s_bf16=True)
+        n = max(64, min(units, N if dense else 131072))
+        if dense:
+            keys = wl.llama_keys("cpu", B=1, H=1, N=n).reshape(n, D)
+            q = wl.llama_queries("cpu", B=1, H=1).reshape(1, D)
+        else:
+            keys = wl.gqa_keys("cpu", B=1, Hkv=1, N=n).reshape(n, D)
+            q = wl.gqa_queries("cpu", B=1, Hq=J).reshape(J, D)
+        keys, q = keys.double().numpy(), q.double().numpy()
+
+        def run():
+            words, norms, _ = oracle.qjl.quantize_keys(O, keys)
+            sq = oracle.qjl.project_queries(O, q)
+            oracle.qjl.scores(O, words[None], norms[None], sq[None])
+        return run, n
+    if name in ("pfqjl_bulk_m256", "pfqjl_bulk_m1024"):
+        m = 256 if name.endswith("256") else 1024
+        O = P.make_projection(4, 256, m, P.KIND_PFQJL)
+        n = max(256, min(units, 1 << 16))
+        keys = wl.bulk_keys("cpu", n=n, d=256).double().numpy()
+        q = wl.bulk_queries("cpu", nq=64, d=256).double().numpy()
+        ns = max(1, n // 16)                       # the workload scores 2^20 of its 2^24 keys
+
+        def run():
+            words, norms, _ = oracle.qjl.quantize_keys(O, keys)
+            sq = oracle.qjl.project_queries(O, q)
+            oracle.qjl.scores(O, words[None, :ns], norms[None, :ns], sq[None])
+        return run, n
+    if name == "dfqjl_decode":
+        O = P.make_projection(5, D, M, P.KIND_DFQJL, sigma_rel=0.5)
+        n = max(64, min(units, 16384))
+        keys, vals = wl.decode_kv("cpu", B=1, H=1, N=n, d=D)
+        keys, vals = keys.reshape(n, D).double().numpy(), vals.reshape(n, D).float().numpy()
+        q = wl.decode_queries("cpu", B=1, H=1).reshape(1, D).double().numpy()
+
+        def run():
+            words, norms, _ = oracle.qjl.quantize_keys(O, keys)
+            codes, sc, zr = oracle.kivi.quantize_values_2bit(vals)
+            sq = oracle.qjl.project_queries(O, q)
+            est = oracle.qjl.scores(O, words[None], norms[None], sq[None])
+            vhat = oracle.kivi.dequantize_values(codes, sc, zr, D)[None]
+            oracle.attention.decode_attention(est, vhat, 1.0 / math.sqrt(D))
+        return run, n
+    raise ValueError(name)
+
+
+ORACLE_UNIT = {"dense_1head": "keys/s", "decode_llama7b": "keys/s", "gqa_decode": "keys/s",
+               "pfqjl_bulk_m256": "vectors/s", "pfqjl_bulk_m1024": "vectors/s", "dfqjl_decode": "tokens/s"}
+
+
+def _timed(run, threads, warm=None):
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=threads):
+        (warm or run)()                                    # warm: BLAS threads, caches, allocations
+        t0 = time.perf_counter()
+        run()
+        return time.perf_counter() - t0
+
+
+# oracle slice per config: one head (or the whole small config), or a key count that takes a few seconds
+ORACLE_SAMPLE = {"dense_1head": 4096, "decode_llama7b": N, "gqa_decode": 16384, "pfqjl_bulk_m256": 32768,
+                 "pfqjl_bulk_m1024": 8192, "dfqjl_decode": 16384}
+
+
+def cpu_baseline(name):
+    """The oracle timed on this host's cores over a fixed slice of workload `name` (ORACLE_SAMPLE), in
+    two modes: one BLAS thread, and as many threads as the process may run on. Each mode takes one
+    untimed warm call on a 512-unit slice, then one timed pass."""
+    affinity = len(os.sched_getaffinity(0))
+    small, _ = oracle_prepare(name, 512)
+    run, units = oracle_prepare(name, ORACLE_SAMPLE[name])
+    res = {"kind": "oracle", "unit": ORACLE_UNIT[name], "nproc": os.cpu_count(), "affinity": affinity}
+    for mode, threads in (("all_cores", affinity), ("single_thread", 1)):
+        dt = _timed(run, threads, warm=small)
+        res[mode] = {"value": units / dt, "cores": threads, "seconds": dt}
+    res["value"] = res["all_cores"]["value"]
+    res["cores"] = affinity
+    res["sample"] = ("%d %s of the workload (one head or key slice, same shapes and generators on the host); "
+                     "the fp64 oracle's quantize, projection and scoring (and, for the fused decode, values "
+                     "and attention), one timed pass per mode after a 512-unit warm call" %
+                     (units, ORACLE_UNIT[name].split("/")[0]))
+    return res
 
 
 def default_desc():
@@ -210,21 +345,25 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    sample = args.ref_sample
-    for _ in range(args.warmup):
-        cpu_oracle_rate(sample)
-    total_keys, total_t = 0, 0.0
-    threads = 1
-    for _ in range(args.steps):
-        rate, dt, threads, k = cpu_oracle_rate(sample)
-        total_keys += k
-        total_t += dt
+    threads = len(os.sched_getaffinity(0))
+    run, sample = oracle_prepare(WORKLOAD, args.ref_sample)
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=threads):
+        for _ in range(args.warmup):
+            run()
+        total_keys, total_t = 0, 0.0
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            run()
+            total_t += time.perf_counter() - t0
+            total_keys += sample
     value = total_keys / total_t
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": run_config(default_desc(), B * H * N, world),
             "cpu_baseline": {"value": value, "unit": "keys/s", "cores": threads, "kind": "oracle",
+                             "nproc": os.cpu_count(),
                              "sample": "%d keys (one head slice of the workload) per step: oracle quantize + "
                                        "project + score" % sample},
             "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -259,6 +398,14 @@ def profile_case(case, n):
         bits, norms = qjl.quantize_keys(P, keys)
         sq = qjl.project_queries(P, wl.llama_queries(dev, B=1, H=G, d=D).reshape(-1, D))
         run = lambda: qjl.scores(P, bits.view(G, N, M // 32), norms.view(G, N), sq.view(G, 1, M))
+    elif case in ("many256", "many1024"):
+        # many-query scores: 2^18 keys against 64 queries (a quarter of the bulk workload's scored keys)
+        m = 256 if case == "many256" else 1024
+        P = qjl.Projection(4, 256, m, "pfqjl")
+        keys = wl.bulk_keys(dev, n=n, d=256)
+        bits, norms = qjl.quantize_keys(P, keys)
+        sq = qjl.project_queries(P, wl.bulk_queries(dev, nq=64, d=256))
+        run = lambda: qjl.scores(P, bits.view(1, n, m // 32), norms.view(1, n), sq.view(1, 64, m))
     elif case == "values":
         v = wl.normal((n, D), 506, dev, torch.bfloat16)
         run = lambda: qjl.quantize_values_2bit(v)
@@ -295,8 +442,11 @@ class Stage:
     """One library call of a step: name, callable, units it processes, algorithmic bytes (and flops) per unit."""
 
     def __init__(self, name, fn, units, bytes_per_unit, flops_per_unit=0, kernel=None, src=None, bound="hbm",
-                 launches=1):
+                 launches=1, peak_scale=1.0):
+        # peak_scale: the stage's tensor peak relative to the measured bf16 one (2 for an int8
+        # contraction: the nominal int8 : bf16 dense ratio)
         self.name, self.fn, self.units, self.launches = name, fn, units, launches
+        self.peak_scale = peak_scale
         self.bytes_per_unit, self.flops_per_unit = bytes_per_unit, flops_per_unit
         self.kernel, self.src, self.bound = kernel, src, bound
 
@@ -316,7 +466,7 @@ def build_workload(name, dev, qjl, wl, torch):
         stages = [
             Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), G * N,
                   2 * D + M // 8 + 4, 2 * D * M, "dense_tc_kernel", "dense_tc.cu"),
-            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * M),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * M, bound="launch"),
             Stage("scores", lambda: qjl.scores(P, bits.view(G, N, M // 32), norms.view(G, N), sq.view(G, 1, M), out=out),
                   G * N, M // 8 + 4 + 4, 0, "scores_digit_kernel", "scores.cu"),
         ]
@@ -334,7 +484,7 @@ def build_workload(name, dev, qjl, wl, torch):
         stages = [
             Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), G * Nq,
                   2 * D + m // 8 + 4, 2 * D * m, "dense_tc_kernel", "dense_tc.cu", "tensor"),
-            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G * J, 4 * D + 4 * m),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G * J, 4 * D + 4 * m, bound="launch"),
             Stage("scores", lambda: qjl.scores(P, bits.view(G, Nq, m // 32), norms.view(G, Nq), sq.view(G, J, m),
                                                out=out), G * Nq, m // 8 + 4 + 4 * J, 0, "scores_decode_kernel",
                   "scores.cu"),
@@ -352,10 +502,10 @@ def build_workload(name, dev, qjl, wl, torch):
         out = torch.empty((1, J, n), dtype=torch.float32, device=dev)
         stages = [
             Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), n, 4 * D + M // 8 + 4,
-                  2 * D * M, "dense_simt_kernel", "dense_simt.cu"),
-            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), J, 4 * D + 4 * M),
+                  2 * D * M, "dense_simt_kernel", "dense_simt.cu", "launch"),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), J, 4 * D + 4 * M, bound="launch"),
             Stage("scores", lambda: qjl.scores(P, bits.view(1, n, M // 32), norms.view(1, n), sq.view(1, J, M), out=out),
-                  n, M // 8 + 4 + 4 * J, 0, "scores_stream_kernel", "scores.cu"),
+                  n, M // 8 + 4 + 4 * J, 0, "scores_many_kernel", "scores_many.cu", "launch"),
         ]
         W.update(units=n, unit="keys/s", inputs=[keys, q], outputs=[out], dtype="f32",
                  desc="%s: 4096 fp32 keys, 16 queries, d=128, m=256 fp32 S (launch-bound)" % name)
@@ -372,10 +522,10 @@ def build_workload(name, dev, qjl, wl, torch):
         stages = [
             Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), n,
                   2 * d + m // 8 + 4, fqjl_flops_per_key(d, m), "fqjl_keys_kernel", "fqjl_keys.cu", "alu"),
-            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), J, 4 * d + 4 * m),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), J, 4 * d + 4 * m, bound="launch"),
             Stage("scores", lambda: qjl.scores(P, bits[:ns].view(1, ns, m // 32), norms[:ns].view(1, ns),
-                                               sq.view(1, J, m), out=out), ns, m // 8 + 4 + 4 * J, 0,
-                  "scores_stream_kernel", "scores.cu"),
+                                               sq.view(1, J, m), out=out), ns, m // 8 + 4 + 4 * J, 2 * J * m,
+                  "scores_many_kernel", "scores_many.cu", "hbm" if m == 256 else "tensor", peak_scale=2.0),
         ]
         W.update(units=n, unit="vectors/s", inputs=[keys, q], outputs=[out], dtype="bf16",
                  desc="%s: P-FQJL, 2^24 keys d=256 bf16, m=%d; quantize all, project 64 queries, score the first "
@@ -401,7 +551,7 @@ def build_workload(name, dev, qjl, wl, torch):
                   2 * D + m // 8 + 4, fqjl_flops_per_key(D, m), "fqjl_keys_kernel", "fqjl_keys.cu", "alu"),
             Stage("quantize_values", lambda: qjl.quantize_values_2bit(vals, codes=codes, scale=sc, zero=zr), G * Nd,
                   2 * D + D // 4 + D // 8, 0, "values_2bit_kernel", "values.cu"),
-            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * m),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * m, bound="launch"),
             Stage("decode_attention", lambda: qjl.decode_attention(
                 P, bits.view(G, Nd, m // 32), norms.view(G, Nd), codes.view(G, Nd, D // 16), sc.view(G, Nd, D // 32),
                 zr.view(G, Nd, D // 32), sq.view(G, 1, m), smx, out=out, workspace=ws), G * Nd,
@@ -448,9 +598,10 @@ def build_workload(name, dev, qjl, wl, torch):
         smx = 1.0 / math.sqrt(D)
         stages = [
             Stage("append_keys", lambda: qjl.append_keys(P, cache, newk, pos), G, 2 * D + m // 8 + 4,
-                  fqjl_flops_per_key(D, m)),
-            Stage("append_values", lambda: qjl.append_values_2bit(cache, newv, pos), G, 2 * D + D // 4 + D // 8),
-            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * m),
+                  fqjl_flops_per_key(D, m), bound="launch"),
+            Stage("append_values", lambda: qjl.append_values_2bit(cache, newv, pos), G, 2 * D + D // 4 + D // 8,
+                  bound="launch"),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * m, bound="launch"),
             Stage("decode_attention_paged", lambda: qjl.decode_attention_paged(P, cache, sq, Nd, smx, out=out,
                                                                                workspace=ws), G * Nd,
                   m // 8 + 4 + D // 4 + D // 8, 0, "decode_stream_kernel", "decode.cu", launches=2),
@@ -480,7 +631,8 @@ def build_workload(name, dev, qjl, wl, torch):
                   2 * D + m // 8 + 4, 2 * D * m, "dense_tc_kernel", "dense_tc.cu"),
             Stage("quantize_values", lambda: qjl.quantize_values_2bit(vals, codes=codes, scale=sc, zero=zr), Gp * Lp,
                   2 * D + D // 4 + D // 8),
-            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), Gp * Lp, 4 * D + 4 * m),
+            Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), Gp * Lp, 4 * D + 4 * m,
+                  kernel="project_mma_kernel", src="project_mma.cu"),
             # work per (query, key) pair: 2 d flops of P.V plus 2 m of sign-dot multiply-adds
             Stage("prefill_attention", lambda: qjl.prefill_attention(
                 P, bits.view(Gp, Lp, -1), norms.view(Gp, Lp), codes.view(Gp, Lp, -1), sc.view(Gp, Lp, -1),
@@ -541,23 +693,124 @@ def build_workload(name, dev, qjl, wl, torch):
     return W
 
 
+PER_CONFIG = ["dense_1head", "gqa_decode", "pfqjl_bulk_m256", "pfqjl_bulk_m1024", "dfqjl_decode"]
+
+
+def stage_roof(st, ms, pk):
+    """A stage's achieved rate on its binding roof: HBM bytes, bf16 tensor flops or fp32 lane operations."""
+    t = ms * 1e-3
+    gbs = st.units * st.bytes_per_unit / t / 1e9
+    e = {"ms": ms, "units_per_s": st.units / t, "gbs": gbs, "frac_hbm_measured": gbs / pk["hbm_gbs"],
+         "frac_8tbs": gbs / 8000.0, "bytes_per_unit": st.bytes_per_unit, "bound": st.bound}
+    if st.flops_per_unit:
+        e["flops_per_unit"] = st.flops_per_unit
+        e["tflops"] = st.units * st.flops_per_unit / t / 1e12
+    if st.bound == "tensor":
+        e["frac"] = e["tflops"] / (st.peak_scale * pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+        e["frac_of"] = ("bf16 tensor peak (sustained, measured)" if st.peak_scale == 1.0 else
+                        "int8 tensor peak: measured bf16 (sustained) x 2, the nominal int8 : bf16 ratio")
+        e["frac_burst"] = e["tflops"] / (st.peak_scale * pk["bf16_tflops"])
+    elif st.bound == "alu":
+        e["frac"] = e["tflops"] / FP32_TFLOPS
+        e["frac_of"] = "FP32 lane ceiling (derived: 148 SMs x 128 lanes x 1.965 GHz)"
+    elif st.bound == "launch":
+        e["frac"] = None
+        e["frac_of"] = "launch-bound (microseconds of work)"
+    else:
+        e["frac"] = e["frac_hbm_measured"]
+        e["frac_of"] = "HBM copy bandwidth (measured)"
+    return e
+
+
+def time_region(stages, steps, stream, torch, world, local, period_ms=50):
+    """Time `steps` whole steps (events around every stage) between barriers, with clocks sampled."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local, period_ms) as clk:
+        clk.mark()
+        t_start.record(stream)
+        for i in range(steps):
+            for j, st in enumerate(stages):
+                evs[i][j].record(stream)
+                st.fn()
+            evs[i][len(stages)].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        clk.mark()
+    barrier(world)
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), world)
+    k_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(len(stages))]
+    return ms_total / steps, k_ms, clk.summary()
+
+
+def analyse(Wk, k_ms, pk, workload):
+    stages = Wk["stages"]
+    kernels = {st.name: stage_roof(st, ms, pk) for st, ms in zip(stages, k_ms)}
+    dom = max(range(len(stages)), key=lambda i: k_ms[i])
+    ds = stages[dom]
+    e = kernels[ds.name]
+    roof = {"bound": "hbm", "kernel": "%s (%s)" % (ds.kernel, ds.name), "achieved": e["gbs"],
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": e["frac_hbm_measured"], "peak_kind": pk["kind"],
+            "traffic": ncu_traffic(ds.kernel, workload, ds.src) if ds.src else None,
+            "bytes_per_launch": ds.units * ds.bytes_per_unit}
+    if ds.bound == "alu":
+        roof.update({"bound": "alu", "achieved": e["tflops"], "peak": FP32_TFLOPS, "unit": "TFLOP/s",
+                     "frac": e["frac"], "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 1.965 GHz",
+                     "flops_per_launch": ds.units * ds.flops_per_unit, "hbm_gbs": e["gbs"],
+                     "hbm_frac": e["frac_hbm_measured"]})
+    elif ds.bound == "tensor":
+        roof.update({"bound": "tensor", "achieved": e["tflops"],
+                     "peak": ds.peak_scale * pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+                     "unit": "TFLOP/s", "frac": e["frac"], "peak_kind": pk["kind"] + " (bf16, sustained)",
+                     "flops_per_launch": ds.units * ds.flops_per_unit, "hbm_gbs": e["gbs"],
+                     "hbm_frac": e["frac_hbm_measured"]})
+    elif ds.flops_per_unit:
+        roof["tensor_tflops"] = e["tflops"]
+        roof["tensor_frac_of_sustained"] = e["tflops"] / pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    return kernels, roof
+
+
+def cold_leg(stage, torch, stream, reps=20):
+    """One stage timed alone, L2 flushed before every call by reading a 256 MB buffer. A read flush
+    leaves L2 full of clean lines: a write flush would leave dirty ones whose write-back the timed
+    call would pay for (and the earlier calls' own dirty outputs are written back during the flush)."""
+    flush = torch.ones((64 << 20,), dtype=torch.float32, device=torch.cuda.current_device())
+    ts = []
+    for r in range(reps + 3):
+        flush.sum()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        stage.fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if r >= 3:
+            ts.append(a.elapsed_time(b))
+    del flush
+    return statistics.median(ts), statistics.mean(ts), reps
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=["decode_llama7b", "gqa_decode", "dense_1head", "pfqjl_bulk_m256", "pfqjl_bulk_m1024",
                              "dfqjl_decode", "paged_decode", "kivi_keys_decode", "prefill_causal"])
     ap.add_argument("--ref-sample", type=int, default=4096)
-    ap.add_argument("--cpu-sample", type=int, default=1 << 21)
     ap.add_argument("--profile-case", default=None,
-                    choices=["quantize", "scores", "fqjl", "fqjl1024", "dfqjl", "values", "decode", "prefill"],
+                    choices=["quantize", "scores", "fqjl", "fqjl1024", "dfqjl", "values", "decode", "prefill",
+                             "many256", "many1024"],
                     help="run one small case of a single kernel (3 launches after 2 warm-ups) for ncu")
     ap.add_argument("--profile-keys", type=int, default=1 << 20)
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--sustained-seconds", type=float, default=2.5,
+                    help="length of the sustained leg (the headline step repeated under the power cap)")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the other configs (single-GPU runs only)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -573,37 +826,41 @@ def main():
     import bit_kv_cache_qjl_b200 as qjl
     from bit_kv_cache_qjl_b200 import workloads as wl
 
-    Wk = build_workload(args.workload, dev, qjl, wl, torch)
-    stages = Wk["stages"]
+    pk, pk_kind = peaks()
+    pk = dict(pk, kind=pk_kind)
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
-        for i, st in enumerate(stages):
-            if ev is not None:
-                ev[i].record(stream)
+    Wk = build_workload(args.workload, dev, qjl, wl, torch)
+    stages = Wk["stages"]
+
+    def step():
+        for st in stages:
             st.fn()
-        if ev is not None:
-            ev[len(stages)].record(stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    ms_total = max_over_ranks(t_start.elapsed_time(t_end), world)
-    ms_step = ms_total / args.steps
-    k_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(len(stages))]
+    ms_step, k_ms, clocks = time_region(stages, args.steps, stream, torch, world, local)
     units = Wk["units"]
     value = job_throughput(units, world, ms_step)
+    kernels, roof = analyse(Wk, k_ms, pk, args.workload)
+
+    # the score stage alone, L2 flushed before every call: its HBM fraction without any L2-resident
+    # tail of the bits that the quantize stage has just written
+    cold = None
+    sc_stage = next((st for st in stages if st.name == "scores"), None)
+    if sc_stage is not None:
+        med, mean, reps = cold_leg(sc_stage, torch, stream)
+        cold = dict(stage_roof(sc_stage, med, pk), kernel=sc_stage.kernel, reps=reps, ms_mean=mean,
+                    rule="median of %d calls, each after a 256 MB read that flushes L2 (clean lines)" % reps)
+
+    # sustained: the same step repeated for a few seconds, long enough for the 1 kW power cap to act
+    n_sus = max(args.steps, int(math.ceil(args.sustained_seconds * 1e3 / ms_step)))
+    s_ms, s_k, s_clk = time_region(stages, n_sus, stream, torch, world, local, period_ms=100)
+    s_kern, s_roof = analyse(Wk, s_k, pk, args.workload)
+    sustained = {"steps": n_sus, "ms_per_step": s_ms, "value": job_throughput(units, world, s_ms),
+                 "kernels": {k: {"ms": v["ms"], "frac": v["frac"], "frac_of": v["frac_of"]} for k, v in s_kern.items()},
+                 "roofline_frac": s_roof["frac"], "clocks": s_clk}
 
     # end to end through the same calls with host buffers (pinned), copies inside the timed region
     h_in = []
@@ -633,64 +890,59 @@ def main():
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
     h2d = sum(h.numel() * h.element_size() for h in h_in)
     d2h = sum(h.numel() * h.element_size() for h in h_out)
-
-    pk, pk_kind = peaks()
-    hbm = pk["hbm_gbs"]
-    tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-    kernels = {}
-    for st, ms in zip(stages, k_ms):
-        gbs = st.units * st.bytes_per_unit / (ms * 1e-3) / 1e9
-        e = {"ms": ms, "units_per_s": st.units / (ms * 1e-3), "gbs": gbs, "frac_hbm_measured": gbs / hbm,
-             "frac_8tbs": gbs / 8000.0, "bytes_per_unit": st.bytes_per_unit}
-        if st.flops_per_unit:
-            e["tflops"] = st.units * st.flops_per_unit / (ms * 1e-3) / 1e12
-        kernels[st.name] = e
-    dom = max(range(len(stages)), key=lambda i: k_ms[i])
-    ds = stages[dom]
-    d_gbs = kernels[ds.name]["gbs"]
-    roof = {"bound": "hbm", "kernel": "%s (%s)" % (ds.kernel, ds.name), "achieved": d_gbs, "peak": hbm,
-            "unit": "GB/s", "frac": d_gbs / hbm, "peak_kind": pk_kind,
-            "traffic": ncu_traffic(ds.kernel, args.workload, ds.src) if ds.src else None,
-            "bytes_per_launch": ds.units * ds.bytes_per_unit}
-    if ds.bound == "alu":
-        # the Walsh-Hadamard transform is bound by fp32 issue, not by HBM: report its fp32 operation
-        # rate against the FP32 lane ceiling, and keep the HBM fraction beside it
-        tfl = kernels[ds.name]["tflops"]
-        roof.update({"bound": "alu", "achieved": tfl, "peak": FP32_TFLOPS, "unit": "TFLOP/s",
-                     "frac": tfl / FP32_TFLOPS, "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 1.965 GHz",
-                     "flops_per_launch": ds.units * ds.flops_per_unit, "hbm_gbs": d_gbs, "hbm_frac": d_gbs / hbm})
-    elif ds.bound == "tensor":
-        tfl = kernels[ds.name]["tflops"]
-        roof.update({"bound": "tensor", "achieved": tfl, "peak": tf, "unit": "TFLOP/s", "frac": tfl / tf,
-                     "peak_kind": pk_kind + " (bf16, sustained)", "flops_per_launch": ds.units * ds.flops_per_unit,
-                     "hbm_gbs": d_gbs, "hbm_frac": d_gbs / hbm})
-    elif ds.flops_per_unit:
-        roof["tensor_tflops"] = kernels[ds.name]["tflops"]
-        roof["tensor_frac_of_sustained"] = kernels[ds.name]["tflops"] / tf
-    clocks = clk.summary()
+    accuracy = Wk["accuracy"]() if "accuracy" in Wk and rank == 0 else None
+    w_unit, w_dtype, w_desc = Wk["unit"], Wk["dtype"], Wk["desc"]
+    launches = sum(st.launches for st in stages) * args.steps
+    del Wk, stages, h_in, h_out
+    torch.cuda.empty_cache()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu and args.workload == WORKLOAD:
-        rate, dt, threads, k = cpu_oracle_rate(args.cpu_sample)
-        cpu = {"value": rate, "unit": "keys/s", "cores": threads, "kind": "oracle",
-               "sample": "%d keys of the workload (%d head slices of %d keys): oracle quantize + project + "
-                         "score, %.1f s" % (k, max(1, k // N), min(N, k), dt)}
+    if rank == 0 and world == 1 and not args.no_cpu and args.workload in ORACLE_UNIT:
+        cpu = cpu_baseline(args.workload)
+
+    # the other configs, each timed the same way in this process, with the oracle beside it
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        per_config = {}
+        for name in PER_CONFIG:
+            if name == args.workload:
+                continue
+            W2 = build_workload(name, dev, qjl, wl, torch)
+            st2 = W2["stages"]
+            for _ in range(args.warmup):
+                for st in st2:
+                    st.fn()
+            torch.cuda.synchronize()
+            ms2, k2, clk2 = time_region(st2, args.steps, stream, torch, world, local)
+            kern2, roof2 = analyse(W2, k2, pk, name)
+            q = kern2.get("quantize_keys")
+            per_config[name] = {
+                "workload": W2["desc"], "value": W2["units"] / (ms2 * 1e-3), "unit": W2["unit"],
+                "ms_per_step": ms2, "steps": args.steps, "kernels": kern2, "roofline": roof2,
+                "quantize_vectors_per_s": q["units_per_s"] if q else None, "clocks": clk2,
+                "cpu_baseline": None if args.no_cpu else cpu_baseline(name)}
+            del W2, st2
+            torch.cuda.empty_cache()
 
     line = {
-        "metric": METRIC, "value": value, "unit": Wk["unit"], "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": w_unit,
+        "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": Wk["dtype"], "data": "synthetic",
-        "config": run_config(Wk["desc"], units, world),
+        "vs_baseline": None, "dtype": w_dtype, "data": "synthetic",
+        "config": run_config(w_desc, units, world),
         "roofline": roof,
         "kernels": kernels,
-        "e2e": {"value": world * units / (e2e_ms * 1e-3), "unit": Wk["unit"], "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": sum(st.launches for st in stages) * args.steps,
+        "scores_cold": cold,
+        "sustained": sustained,
+        "e2e": {"value": world * units / (e2e_ms * 1e-3), "unit": w_unit,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
         "clocks": clocks,
         "cpu_baseline": cpu,
+        "per_config": per_config,
     }
-    if "accuracy" in Wk and rank == 0:
-        line["accuracy"] = Wk["accuracy"]()
+    if accuracy is not None:
+        line["accuracy"] = accuracy
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
