@@ -637,7 +637,7 @@ def build_workload(name, dev, qjl, wl, torch):
             Stage("prefill_attention", lambda: qjl.prefill_attention(
                 P, bits.view(Gp, Lp, -1), norms.view(Gp, Lp), codes.view(Gp, Lp, -1), sc.view(Gp, Lp, -1),
                 zr.view(Gp, Lp, -1), sq.view(Gp, Lp, m), 1.0 / math.sqrt(D), out=out), pairs, 0, 2 * D + 2 * m,
-                "prefill_kernel", "prefill.cu", "tensor"),
+                "prefill_tc_kernel", "prefill.cu", "tensor"),
         ]
         W.update(units=pairs, unit="query-key pairs/s", inputs=[keys, vals, q], outputs=[out], dtype="bf16",
                  desc="%s: 32 heads x 4096 tokens, d=128, m=256 dense bf16 S; quantize keys and 2-bit values, project "

@@ -23,7 +23,7 @@
 // A lives in TMEM rather than shared memory: expanding m bits into m bytes
 // per key and reading them back through shared memory would take more
 // shared-memory bandwidth than the MMAs leave. Persistent kernel, one CTA
-// per SM, 14 warps:
+// per SM, 22 warps:
 //   warp 0      bulk-copy producer: each 128-key tile's sign words into a
 //               ring of shared-memory stages.
 //   warp 1      allocates TMEM (two D buffers of 128 columns, then A
@@ -32,8 +32,9 @@
 //   warps 2-5   expanders: thread r of lane quarter r / 32 owns key row r; it
 //               turns its words into A columns with tcgen05.st, KC words per
 //               A buffer.
-//   warps 6-13  epilogue: two warps per lane quarter, each half of the
-//               queries; tcgen05.ld of D, the estimate, coalesced stores of
+//   warps 6-21  epilogue: four warps per lane quarter, each a quarter of the
+//               queries; tcgen05.ld of D, the estimate (pairs of queries in
+//               packed f32x2 arithmetic), coalesced stores of
 //               scores[g][j][n]. They also build each group's B table: a
 //               group's table goes into a buffer once the last tile that read
 //               that buffer has left the epilogue (so its MMAs are complete).
@@ -61,7 +62,7 @@ using namespace qjl_sync;
 
 constexpr int kTile = 128;             // keys per MMA tile (M)
 constexpr int kExpWarps = 4;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;
 constexpr int kThreads = (2 + kExpWarps + kEpiWarps) * 32;
 constexpr int kTmemCols = 512;
 constexpr int kDStride = 128;          // columns per D buffer
@@ -85,70 +86,56 @@ struct ManyParams {
 
 // Table of one group into `tab` (2 JP rows x m bytes, K-major slices of 32
 // bytes per sign word) and its per-query constants. Run by the epilogue
-// warps (kEpiWarps * 32 threads, named barrier 1).
+// warps (kEpiWarps * 32 threads, named barrier 1). A warp takes whole query
+// rows: lane l holds coordinate 32 k + l of the row for every word k, loaded
+// at once, so one pass finds max |Sq| and a second quantises and writes the
+// two digit bytes of each coordinate to its K position (4 s + e for bit
+// 8 e + s of the word). Rows j >= J are zero.
 template <int W, int JP>
 __device__ void build_table(const float* __restrict__ sqg, int J, float est_scale, unsigned char* tab,
-                            float* s_mul, int* s_qs, int tid) {
+                            float2* s_cst, int tid) {
   constexpr int m = 32 * W;
   constexpr int nthr = kEpiWarps * 32;
   constexpr int N = 2 * JP;
-  __shared__ float s_inv[JP];
   const int lane = tid & 31, wq = tid >> 5;
+  const int kpos = 4 * (lane & 7) + (lane >> 3);  // K position of bit `lane` within its word's slice
   // every epilogue warp is done with the buffer's previous constants
   named_sync(1, nthr);
-  // per query: max |Sq| (the fixed-point scale) and the sum of Q
   for (int j = wq; j < JP; j += kEpiWarps) {
+    float v[W];
+#pragma unroll
+    for (int k = 0; k < W; ++k) v[k] = j < J ? __ldg(sqg + (int64_t)j * m + 32 * k + lane) : 0.f;
     float mx = 0.f;
-    if (j < J)
-      for (int i = lane; i < m; i += 32) mx = fmaxf(mx, fabsf(__ldg(sqg + (int64_t)j * m + i)));
+#pragma unroll
+    for (int k = 0; k < W; ++k) mx = fmaxf(mx, fabsf(v[k]));
 #pragma unroll
     for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     const float inv = mx > 0.f ? (float)kQmax / mx : 0.f;
     int qs = 0;
-    if (j < J)
-      for (int i = lane; i < m; i += 32) {
-        const float q = rintf(__ldg(sqg + (int64_t)j * m + i) * inv);
-        qs += (int)fminf(fmaxf(q, (float)-kQmax), (float)kQmax);
-      }
+    unsigned char* hi_row = tab + qjl_tc::kmajor_ofs(j, kpos);
+    unsigned char* lo_row = tab + qjl_tc::kmajor_ofs(JP + j, kpos);
+#pragma unroll
+    for (int k = 0; k < W; ++k) {
+      const int Q = (int)fminf(fmaxf(rintf(v[k] * inv), (float)-kQmax), (float)kQmax);
+      qs += Q;
+      const int l = (int)(int8_t)(Q & 0xFF);
+      hi_row[k * N * 32] = (unsigned char)((Q - l) >> 8);
+      lo_row[k * N * 32] = (unsigned char)l;
+    }
 #pragma unroll
     for (int o = 16; o; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
     if (lane == 0) {
-      s_inv[j] = inv;
-      s_mul[j] = est_scale * (mx > 0.f ? mx / (float)kQmax : 0.f);
-      s_qs[j] = qs;
+      // the estimate is c1 * (sum b Q) + c0, times ||k||
+      const float mul = est_scale * (mx > 0.f ? mx / (float)kQmax : 0.f);
+      s_cst[j] = make_float2(2.f * mul, -mul * (float)qs);
     }
-  }
-  named_sync(1, nthr);
-  // one (query j, word w, shift s) per step: the digits of bits 8 e + s, e = 0..3,
-  // as one 32-bit word of row j (hi) and one of row JP + j (lo) at K positions 4 s .. 4 s + 3
-  for (int idx = tid; idx < JP * W * 8; idx += nthr) {
-    const int s = idx & 7;
-    const int w = (idx >> 3) % W;
-    const int j = (idx >> 3) / W;
-    uint32_t hi = 0u, lo = 0u;
-    if (j < J) {
-      const float inv = s_inv[j];
-      const float* src = sqg + (int64_t)j * m + 32 * w + s;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float q = rintf(__ldg(src + 8 * e) * inv);
-        const int Q = (int)fminf(fmaxf(q, (float)-kQmax), (float)kQmax);
-        const int l = (int)(int8_t)(Q & 0xFF);
-        const int h = (Q - l) >> 8;
-        hi |= ((uint32_t)h & 0xFFu) << (8 * e);
-        lo |= ((uint32_t)l & 0xFFu) << (8 * e);
-      }
-    }
-    unsigned char* slice = tab + (size_t)w * N * 32;
-    *reinterpret_cast<uint32_t*>(slice + qjl_tc::kmajor_ofs(j, 4 * s)) = hi;
-    *reinterpret_cast<uint32_t*>(slice + qjl_tc::kmajor_ofs(JP + j, 4 * s)) = lo;
   }
   // the MMAs read the table through the async proxy
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   named_sync(1, nthr);
 }
 
-// TMEM loads of NC consecutive columns (NC = 4, 8, 16 or 32) of this thread's lane, no wait.
+// TMEM loads of NC consecutive columns (NC = 2, 4, 8, 16 or 32) of this thread's lane, no wait.
 template <int NC>
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t* r) {
   if constexpr (NC == 32) {
@@ -161,11 +148,13 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t* r) {
         : "r"(taddr));
   } else if constexpr (NC == 8) {
     qjl_tc::ld8(taddr, r);
-  } else {
-    static_assert(NC == 4, "4, 8, 16 or 32 columns");
+  } else if constexpr (NC == 4) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(taddr));
+  } else {
+    static_assert(NC == 2, "2, 4, 8, 16 or 32 columns");
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr));
   }
 }
 
@@ -195,7 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
   constexpr int KC = kc_words(W);         // sign words per A buffer
   constexpr int NCH = W / KC;             // A buffers per tile
   constexpr int NA = n_abuf(W);
-  constexpr int JH = JP / 2;              // queries per epilogue warp
+  constexpr int JH = JP / (kEpiWarps / 4);  // queries per epilogue warp (even)
+  static_assert(JH % 2 == 0, "query pairs");
   constexpr uint32_t TAB = (uint32_t)NCOL * 32 * W;
   constexpr uint32_t STAGE = (uint32_t)kTile * W * 4;
   static_assert(W % KC == 0 && NA >= 2, "A buffers");
@@ -204,9 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_dyn + 1023) & ~(uintptr_t)1023);
   unsigned char* sbits = base;                                                // [NS] stages
   unsigned char* tabs = sbits + (size_t)P.NS * STAGE;                         // [ntab] tables
-  float* s_mul = reinterpret_cast<float*>(tabs + (size_t)P.ntab * TAB);       // [2][64]
-  int* s_qs = reinterpret_cast<int*>(s_mul + 128);                            // [2][64]
-  uint64_t* full = reinterpret_cast<uint64_t*>(s_qs + 128);
+  float2* s_cst = reinterpret_cast<float2*>(tabs + (size_t)P.ntab * TAB);   // [2][64] per-query (c1, c0)
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_cst + 128);
   uint64_t* empty = full + P.NS;
   uint64_t* afull = empty + P.NS;    // [NA]
   uint64_t* aempty = afull + NA;     // [NA]
@@ -321,19 +310,22 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
     uint32_t ph = 0, apar = 0;
     for (int64_t it = i0; it < i1; ++it) {
       if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { atomicOr(P.err, 4); break; }
-      uint32_t words[W];
       const unsigned char* stg = sbits + (size_t)s * STAGE;
-#pragma unroll
-      for (int k = 0; k < W / 4; ++k) {
-        const uint4 v = *reinterpret_cast<const uint4*>(stg + swz_ofs<W>(r, k));
-        words[4 * k] = v.x; words[4 * k + 1] = v.y; words[4 * k + 2] = v.z; words[4 * k + 3] = v.w;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      if (++s == NS) { s = 0; ph ^= 1u; }
       bool ok = true;
 #pragma unroll
       for (int ch = 0; ch < NCH; ++ch) {
+        // this chunk's KC words of row r (16-byte pieces at their swizzled offsets)
+        uint32_t words[KC];
+#pragma unroll
+        for (int k = 0; k < KC / 4; ++k) {
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + swz_ofs<W>(r, ch * (KC / 4) + k));
+          words[4 * k] = v.x; words[4 * k + 1] = v.y; words[4 * k + 2] = v.z; words[4 * k + 3] = v.w;
+        }
+        if (ch == NCH - 1) {
+          // the stage is read: hand it back to the producer
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
+        }
         if (!__all_sync(0xffffffffu, mbar_wait(&aempty[ab], apar ^ 1u))) { atomicOr(P.err, 4); ok = false; break; }
         qjl_tc::fence_after();
         const uint32_t a_addr = tmem_base + lane_off + (uint32_t)(kAcol0 + ab * 8 * KC);
@@ -343,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
           uint32_t a[32];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const uint32_t w = words[ch * KC + t4 + u];
+            const uint32_t w = words[t4 + u];
 #pragma unroll
             for (int sh = 0; sh < 8; ++sh) a[8 * u + sh] = (w >> sh) & 0x01010101u;
           }
@@ -355,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
         if (lane == 0) mbar_arrive(&afull[ab]);
         if (++ab == NA) { ab = 0; apar ^= 1u; }
       }
+      if (++s == NS) { s = 0; ph ^= 1u; }
       if (!ok) break;
     }
   } else {
@@ -362,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
     const int ew = warp - 2 - kExpWarps;   // 0..7
     const int tid = ew * 32 + lane;        // 0..255, named barrier 1
     const int quarter = warp & 3;
-    const int hq = ew >> 2;                // which half of the queries
+    const int hq = ew >> 2;                // which share of the queries
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int J = P.J;
@@ -370,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
     const int64_t ngroups = i1 > i0 ? (i1 - 1) / tpg - g_first + 1 : 0;
     for (int k = 0; k < ntab && k < ngroups; ++k) {
       build_table<W, JP>(P.sq + (g_first + k) * (int64_t)J * m, J, P.est_scale, tabs + (size_t)k * TAB,
-                         s_mul + 64 * k, s_qs + 64 * k, tid);
+                         s_cst + 64 * k, tid);
       if (tid == 0) mbar_arrive(&tfull[k]);
     }
     const uint64_t pol = qjl_hint::evict_first();
@@ -387,6 +380,8 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
       }
       const int64_t n0 = c * kTile;
       const int cnt = (int)(N - n0 < kTile ? N - n0 : kTile);
+      // the tile's norm is fetched before the wait for its accumulator
+      const float nrm = r < cnt ? __ldg(P.norms + g * N + n0 + r) : 0.f;
       if (!dead && !__all_sync(0xffffffffu, mbar_wait(&dfull[db], dpar))) { atomicOr(P.err, 16); dead = true; }
       if (!dead) {
         qjl_tc::fence_after();
@@ -400,17 +395,23 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
         if (lane == 0) mbar_arrive(&dempty[db]);
         if (r < cnt) {
           const int64_t n = n0 + r;
-          const float nrm = __ldg(P.norms + g * N + n);
           float* out = P.scores + (g * J + hq * JH) * N + n;
-          const float* mul = s_mul + 64 * tb + hq * JH;
-          const int* qs = s_qs + 64 * tb + hq * JH;
+          const float2* cst = s_cst + 64 * tb + hq * JH;
 #pragma unroll
-          for (int jj = 0; jj < JH; ++jj) {
-            if (hq * JH + jj < J) {
-              // sum b Q = 256 D_hi + D_lo, exact in int32 (|.| <= m * 32639 < 2^31)
-              const int D = (int)hi[jj] * 256 + (int)lo[jj];
-              qjl_hint::st_f32(out + (int64_t)jj * N, mul[jj] * nrm * (float)(2 * D - qs[jj]), pol);
-            }
+          for (int jj = 0; jj < JH; jj += 2) {
+            // sum b Q = 256 D_hi + D_lo, exact in int32 (|.| <= m * 32639 < 2^31); two queries at once
+            const float4 cc = *reinterpret_cast<const float4*>(cst + jj);  // (c1, c0) of queries jj, jj + 1
+            const float d0 = (float)((int)hi[jj] * 256 + (int)lo[jj]);
+            const float d1 = (float)((int)hi[jj + 1] * 256 + (int)lo[jj + 1]);
+            float e0, e1;
+            asm("{\n\t.reg .b64 a, b, c;\n\t"
+                "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+                "fma.rn.f32x2 a, a, b, c;\n\tmov.b64 b, {%8, %8};\n\tmul.rn.f32x2 a, a, b;\n\t"
+                "mov.b64 {%0, %1}, a;\n\t}"
+                : "=f"(e0), "=f"(e1)
+                : "f"(cc.x), "f"(cc.z), "f"(d0), "f"(d1), "f"(cc.y), "f"(cc.w), "f"(nrm));
+            if (hq * JH + jj < J) qjl_hint::st_f32(out + (int64_t)jj * N, e0, pol);
+            if (hq * JH + jj + 1 < J) qjl_hint::st_f32(out + (int64_t)(jj + 1) * N, e1, pol);
           }
         }
       }
@@ -420,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
       const bool last = (c + 1 == tpg) || (it + 1 == i1);
       if (last && gi + ntab < ngroups) {
         build_table<W, JP>(P.sq + (g_first + gi + ntab) * (int64_t)J * m, J, P.est_scale, tabs + (size_t)tb * TAB,
-                           s_mul + 64 * tb, s_qs + 64 * tb, tid);
+                           s_cst + 64 * tb, tid);
         if (tid == 0) mbar_arrive(&tfull[tb]);
       }
       if (++c == tpg) { c = 0; ++g; }

@@ -98,3 +98,16 @@ def test_many_query_projection_kernels(cuda_ok):
     assert _has(_kernels(lambda: qjl.project_queries(Pb, q)), "project_mma_kernel")
     Pf = qjl.Projection(2, 128, 256, "dense", s_bf16=False)
     assert _has(_kernels(lambda: qjl.project_queries(Pf, q)), "dense_simt_kernel")
+
+
+def test_prefill_uses_tcgen05_kernel(cuda_ok):
+    P = qjl.Projection(2, 128, 256, "dense")
+    G, L = 2, 200
+    bits = torch.zeros((G, L, 8), dtype=torch.int32, device="cuda")
+    norms = torch.ones((G, L), device="cuda")
+    codes = torch.zeros((G, L, 8), dtype=torch.int32, device="cuda")
+    sc = torch.ones((G, L, 4), dtype=torch.float16, device="cuda")
+    zr = torch.zeros((G, L, 4), dtype=torch.float16, device="cuda")
+    sq = torch.ones((G, L, 256), device="cuda")
+    names = _kernels(lambda: qjl.prefill_attention(P, bits, norms, codes, sc, zr, sq, 0.1))
+    assert _has(names, "prefill_tc_kernel"), names

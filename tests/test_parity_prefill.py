@@ -4,8 +4,11 @@ The GPU is given the oracle's bits, norms, codes, scales and zeros, and Sq, so
 only the kernel's arithmetic is compared. Tolerance:
 |gpu - oracle| <= 2e-3 * sum_j p_ij |v_hat_j| + 1e-6. P and v_hat enter the
 fp16 tensor cores rounded to binary16 (2^-11 relative each); the products
-and sums run in fp32, and the 23-bit rounding of Sq moves the scores by
-far less. Shapes cover one and several 16-query tiles, ragged L, and D-FQJL.
+and sums run in fp32, and the 16-bit rounding of Sq moves the scores by
+far less. Shapes cover one and several 128-query tiles (a CTA's tile of
+queries and of keys), ragged and exact multiples of 128, L = 1, D-FQJL and
+P-FQJL, and keys scaled up so that the running max moves by more than 2^8
+between key tiles (the output accumulator is then rescaled in TMEM).
 """
 
 import math
@@ -21,14 +24,16 @@ from helpers import host, oracle_projection
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("kind,G,L", [("dense", 2, 16), ("dense", 3, 100), ("dfqjl", 2, 257), ("dense", 1, 1),
-                                      ("pfqjl", 2, 48)])
-def test_prefill(cuda_ok, kind, G, L):
+@pytest.mark.parametrize("kind,G,L,kscale", [("dense", 2, 16, 1.0), ("dense", 3, 100, 1.0), ("dfqjl", 2, 257, 1.0),
+                                             ("dense", 1, 1, 1.0), ("pfqjl", 2, 48, 1.0), ("dense", 1, 128, 1.0),
+                                             ("dense", 2, 129, 1.0), ("dense", 1, 700, 6.0), ("dfqjl", 2, 384, 4.0),
+                                             ("dense", 1, 1000, 1.0)])
+def test_prefill(cuda_ok, kind, G, L, kscale):
     d, m = 128, 256
     P = qjl.Projection(41, d, m, kind)
     O = oracle_projection(P)
     rng = np.random.default_rng(3)
-    keys = rng.standard_normal((G * L, d)).astype(np.float32)
+    keys = (kscale * rng.standard_normal((G * L, d))).astype(np.float32)
     vals = rng.standard_normal((G * L, d)).astype(np.float32)
     words, norms, _ = oracle.qjl.quantize_keys(O, keys)
     c, s, z = oracle.kivi.quantize_values_2bit(vals)

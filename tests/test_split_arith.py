@@ -132,3 +132,41 @@ def test_shift_window_digits_give_the_exact_sign_sum():
             assert tot == int((bits * Q).sum())
             # the estimator's signed sum: 2 tot - sum Q = sum (2 b - 1) Q
             assert 2 * tot - int(Q.sum()) == int(((2 * bits - 1) * Q).sum())
+
+
+def test_integer_pv_weight_rounding_model():
+    """The rounding of a P.V computed as an integer contraction (a design study for the fused decode).
+
+    The weights w_t = p_t * s_t of one 512-token stage are rounded to a (8 nd - 1)-bit
+    grid scaled by the stage's max weight, the code sums are exact integers, and the
+    zero term is added in float. Over softmaxes from flat to one dominant token, the
+    worst error against exact fp64, relative to the fused decode's bound
+    1e-3 * sum_t p_t |v_hat_t| + 1e-6, is about 0.5 % (under 1 %) with three int8 digit
+    rows and between 1 % and 60 % with two: why three rows were costed.
+    """
+    rng = np.random.default_rng(0)
+    d, N, stage = 128, 16384, 512
+    worst = {2: 0.0, 3: 0.0}
+    for trial in range(20):
+        x = rng.standard_normal(N) * (1.0 + 3.0 * (trial % 4))
+        if trial % 5 == 0:
+            x[rng.integers(N)] += 30
+        p = np.exp(x - x.max())
+        codes = rng.integers(0, 4, size=(N, d))
+        s = np.abs(rng.standard_normal(N)) * 0.5 + 0.1
+        z = rng.standard_normal(N)
+        vhat = codes * s[:, None] + z[:, None]
+        exact = (p[:, None] * vhat).sum(0)
+        bound = 1e-3 * (p[:, None] * np.abs(vhat)).sum(0) + 1e-6
+        for nd in (2, 3):
+            qmax = (1 << (8 * nd - 1)) - 1
+            acc = np.zeros(d)
+            for st in range(0, N, stage):
+                w = p[st:st + stage] * s[st:st + stage]
+                W = w.max()
+                wq = np.rint(w / W * qmax)
+                acc += (wq[:, None] * codes[st:st + stage]).sum(0) * (W / qmax)
+            acc += (p * z).sum()
+            worst[nd] = max(worst[nd], (np.abs(acc - exact) / bound).max())
+    assert worst[3] < 0.01, worst
+    assert 0.01 < worst[2] < 0.6, worst
