@@ -44,6 +44,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "mbarrier.cuh"
 #include "qjl_internal.h"
 #include "tcgen05.cuh"
@@ -240,23 +242,55 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillPa
       qjl_tc::fence_after();
       const float* nb = snorm + kb * kT;
       const int64_t k0 = (int64_t)kt * kT;
-      // key j of the tile is visible to this row iff k0 + j <= qi and k0 + j < L
+      // key j of the tile is visible to this row iff k0 + j <= qi and k0 + j < L; only the last
+      // tile (the diagonal one, the only one that can reach past L) needs the check
       const int64_t jmax = min(qi, L - 1) - k0;  // last visible j (< 0: none)
-      // ---- pass 1: the tile's row max
-      float mt = -INFINITY;
+      const bool masked = kt == nkt - 1;
+      // one pass over the row: the scores, their max, and (unless the max must be found first)
+      // p = 2^(s - m) against the running max, written as fp16 pairs into P buffer pb
+      auto pass = [&](auto mask_c, auto write_c, float mref, float& mt, float& lt) {
+        constexpr bool MASK = decltype(mask_c)::value;
+        constexpr bool WRITE = decltype(write_c)::value;
 #pragma unroll 1
-      for (int ch = 0; ch < kT / 32; ++ch) {
-        uint32_t hi[32], lo[32];
-        qjl_tc::ld32(tmem + lane_off + kColShi + 32 * ch, hi);
-        qjl_tc::ld32(tmem + lane_off + kColSlo + 32 * ch, lo);
-        qjl_tc::wait_ld();
+        for (int ch = 0; ch < kT / 32; ++ch) {
+          uint32_t hi[32], lo[32];
+          qjl_tc::ld32(tmem + lane_off + kColShi + 32 * ch, hi);
+          qjl_tc::ld32(tmem + lane_off + kColSlo + 32 * ch, lo);
+          qjl_tc::wait_ld();
+          uint32_t pk[16];
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int j = 32 * ch + jj;
-          const int t = 2 * ((int)hi[jj] * 256 + (int)lo[jj]) - qsum;
-          const float s = mul * nb[j] * (float)t;
-          mt = (j <= jmax) ? fmaxf(mt, s) : mt;
+          for (int jj = 0; jj < 32; jj += 2) {
+            float p2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int j = 32 * ch + jj + u;
+              const int t = 2 * ((int)hi[jj + u] * 256 + (int)lo[jj + u]) - qsum;
+              float sc = mul * nb[j] * (float)t;
+              if (MASK && j > jmax) sc = -INFINITY;
+              mt = fmaxf(mt, sc);
+              p2[u] = WRITE ? exp2f(sc - mref) : 0.f;
+              lt += p2[u];
+            }
+            if (WRITE) {
+              const __half2 h = __floats2half2_rn(p2[0], p2[1]);
+              pk[jj / 2] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+          }
+          if (WRITE) st16(tmem + lane_off + kColP + 64 * pb + 16 * ch, pk);
         }
+      };
+      // P buffer pb is free once the P.V two tiles back has read it
+      if (!__all_sync(0xffffffffu, mbar_wait(&pfree[pb], (uint32_t)(((kt >> 1) & 1) ^ 1))))
+        { atomicOr(P.err, 16); ok = false; break; }
+      qjl_tc::fence_after();
+      const bool fresh = __any_sync(0xffffffffu, m_run == -INFINITY);  // the first visible tile
+      float mt = -INFINITY, lt = 0.f;
+      if (fresh) {
+        if (masked) pass(std::true_type(), std::false_type(), 0.f, mt, lt);
+        else pass(std::false_type(), std::false_type(), 0.f, mt, lt);
+      } else {
+        if (masked) pass(std::true_type(), std::true_type(), m_run, mt, lt);
+        else pass(std::false_type(), std::true_type(), m_run, mt, lt);
       }
       // ---- lazy rescale: a row's running max moves only when the tile's exceeds it by more than
       // 2^kTau (or on its first visible key). Rows decide on their own; the O rescale in TMEM is
@@ -265,10 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillPa
       const bool scale_o = move && m_run != -INFINITY;  // this row's O holds earlier tiles
       float f = 1.f;
       if (move) {
-        if (scale_o) {
-          f = exp2f(m_run - mt);
-          l_run *= f;
-        }
+        if (scale_o) f = exp2f(m_run - mt);
         m_run = mt;
       }
       if (__any_sync(0xffffffffu, scale_o)) {
@@ -286,37 +317,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillPa
           for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
           qjl_tc::st32(tmem + lane_off + kColO + 32 * ch, o);
         }
+      }
+      if (fresh || __any_sync(0xffffffffu, move)) {
+        // p against the final max (rows that kept theirs get the same values again); the first
+        // pass's P stores complete before these overwrite them
         qjl_tc::wait_st();
+        const float mref = m_run == -INFINITY ? 0.f : m_run;
+        float mt2 = -INFINITY;
+        lt = 0.f;
+        if (masked) pass(std::true_type(), std::true_type(), mref, mt2, lt);
+        else pass(std::false_type(), std::true_type(), mref, mt2, lt);
       }
-      const float mref = m_run == -INFINITY ? 0.f : m_run;
-      // ---- pass 2: p = 2^(s - m) as fp16 pairs into P buffer pb, once the P.V two tiles back has read it
-      if (!__all_sync(0xffffffffu, mbar_wait(&pfree[pb], (uint32_t)(((kt >> 1) & 1) ^ 1))))
-        { atomicOr(P.err, 16); ok = false; break; }
-      qjl_tc::fence_after();
-#pragma unroll 1
-      for (int ch = 0; ch < kT / 32; ++ch) {
-        uint32_t hi[32], lo[32];
-        qjl_tc::ld32(tmem + lane_off + kColShi + 32 * ch, hi);
-        qjl_tc::ld32(tmem + lane_off + kColSlo + 32 * ch, lo);
-        qjl_tc::wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int jj = 0; jj < 32; jj += 2) {
-          float p2[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int j = 32 * ch + jj + u;
-            const int t = 2 * ((int)hi[jj + u] * 256 + (int)lo[jj + u]) - qsum;
-            const float s = mul * nb[j] * (float)t;
-            p2[u] = (j <= jmax) ? exp2f(s - mref) : 0.f;
-          }
-          const __half2 h = __floats2half2_rn(p2[0], p2[1]);
-          const float2 hf = __half22float2(h);
-          l_run += hf.x + hf.y;  // the sum of the rounded weights P.V uses
-          pk[jj / 2] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        st16(tmem + lane_off + kColP + 64 * pb + 16 * ch, pk);
-      }
+      l_run = l_run * f + lt;
       qjl_tc::wait_st();
       qjl_tc::fence_before();
       __syncwarp();
@@ -429,11 +441,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const PrefillPa
       const uint32_t cw[kCW] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
       unsigned char* vs = Vb + (size_t)kb * kVbytes + (r >> 4) * (kD * 32);  // the K slice of this key
       const int kbyte = 2 * (r & 15);
+      // channels c and c + 8 share a code word and a scale group: one shift and one mask-or give
+      // the fp16 pair (1024 + code_c, 1024 + code_c+8), an exact subtract leaves the codes, and one
+      // fp16x2 FMA forms both code * scale + zero with a single rounding each
 #pragma unroll
-      for (int c = 0; c < kD; ++c) {
-        const uint32_t code = (cw[c >> 4] >> (2 * (c & 15))) & 3u;
-        const __half vh = __hfma(__uint2half_rn(code), sc[c >> 5], zr[c >> 5]);
-        *reinterpret_cast<__half*>(vs + qjl_tc::kmajor_ofs(c, kbyte)) = vh;
+      for (int w = 0; w < kCW; ++w) {
+        const __half2 s2 = __half2half2(sc[w >> 1]), z2 = __half2half2(zr[w >> 1]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t x = ((cw[w] >> (2 * k)) & 0x00030003u) | 0x64006400u;
+          const __half2 v = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), __float2half2_rn(1024.f)), s2, z2);
+          *reinterpret_cast<__half*>(vs + qjl_tc::kmajor_ofs(16 * w + k, kbyte)) = __low2half(v);
+          *reinterpret_cast<__half*>(vs + qjl_tc::kmajor_ofs(16 * w + k + 8, kbyte)) = __high2half(v);
+        }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
