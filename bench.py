@@ -442,11 +442,12 @@ class Stage:
     """One library call of a step: name, callable, units it processes, algorithmic bytes (and flops) per unit."""
 
     def __init__(self, name, fn, units, bytes_per_unit, flops_per_unit=0, kernel=None, src=None, bound="hbm",
-                 launches=1, peak_scale=1.0):
+                 launches=1, peak_scale=1.0, alu_ops_per_unit=0):
         # peak_scale: the stage's tensor peak relative to the measured bf16 one (2 for an int8
-        # contraction: the nominal int8 : bf16 dense ratio)
+        # contraction: the nominal int8 : bf16 dense ratio). alu_ops_per_unit: fp32 lane operations
+        # a tensor-bound stage also runs (reported beside, against the FP32 lane ceiling)
         self.name, self.fn, self.units, self.launches = name, fn, units, launches
-        self.peak_scale = peak_scale
+        self.peak_scale, self.alu_ops_per_unit = peak_scale, alu_ops_per_unit
         self.bytes_per_unit, self.flops_per_unit = bytes_per_unit, flops_per_unit
         self.kernel, self.src, self.bound = kernel, src, bound
 
@@ -520,8 +521,11 @@ def build_workload(name, dev, qjl, wl, torch):
         sq = torch.empty((J, m), dtype=torch.float32, device=dev)
         out = torch.empty((1, J, ns), dtype=torch.float32, device=dev)
         stages = [
+            # the first Hadamard factor runs as an exact +-1 contraction on tcgen05 (2 d m flops per
+            # key), the second (D_g and d log2 d additions per block) on the FP32 lanes
             Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), n,
-                  2 * d + m // 8 + 4, fqjl_flops_per_key(d, m), "fqjl_keys_kernel", "fqjl_keys.cu", "alu"),
+                  2 * d + m // 8 + 4, 2 * d * m, "fqjl_tc_kernel", "fqjl_tc.cu", "tensor", launches=m // 256,
+                  alu_ops_per_unit=(m // d) * (d + d * int(math.log2(d)))),
             Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), J, 4 * d + 4 * m, bound="launch"),
             Stage("scores", lambda: qjl.scores(P, bits[:ns].view(1, ns, m // 32), norms[:ns].view(1, ns),
                                                sq.view(1, J, m), out=out), ns, m // 8 + 4 + 4 * J, 2 * J * m,
@@ -705,6 +709,10 @@ def stage_roof(st, ms, pk):
     if st.flops_per_unit:
         e["flops_per_unit"] = st.flops_per_unit
         e["tflops"] = st.units * st.flops_per_unit / t / 1e12
+    if st.alu_ops_per_unit:
+        e["alu_ops_per_unit"] = st.alu_ops_per_unit
+        e["alu_tops"] = st.units * st.alu_ops_per_unit / t / 1e12
+        e["alu_frac"] = e["alu_tops"] / FP32_TFLOPS
     if st.bound == "tensor":
         e["frac"] = e["tflops"] / (st.peak_scale * pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
         e["frac_of"] = ("bf16 tensor peak (sustained, measured)" if st.peak_scale == 1.0 else
@@ -764,8 +772,10 @@ def analyse(Wk, k_ms, pk, workload):
         roof.update({"bound": "tensor", "achieved": e["tflops"],
                      "peak": ds.peak_scale * pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
                      "unit": "TFLOP/s", "frac": e["frac"], "peak_kind": pk["kind"] + " (bf16, sustained)",
-                     "flops_per_launch": ds.units * ds.flops_per_unit, "hbm_gbs": e["gbs"],
+                     "flops_per_launch": ds.units * ds.flops_per_unit // ds.launches, "hbm_gbs": e["gbs"],
                      "hbm_frac": e["frac_hbm_measured"]})
+        if ds.alu_ops_per_unit:
+            roof.update({"alu_tops": e["alu_tops"], "alu_frac": e["alu_frac"]})
     elif ds.flops_per_unit:
         roof["tensor_tflops"] = e["tflops"]
         roof["tensor_frac_of_sustained"] = e["tflops"] / pk.get("bf16_tflops_sustained", pk["bf16_tflops"])

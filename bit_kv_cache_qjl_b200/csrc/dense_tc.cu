@@ -38,9 +38,12 @@
 #include <mutex>
 
 #include "cache_hint.cuh"
+#include "key_math.cuh"
 #include "qjl_internal.h"
 
 namespace {
+
+using qjl_km::sq_acc_bf16x2;
 
 constexpr int BM = 128;            // keys per tile (MMA M)
 constexpr int kEpiWarps = 8;
@@ -214,15 +217,6 @@ __device__ __forceinline__ void tmem_ld64_pack(uint32_t taddr, uint32_t& w0, uin
   uint32_t v[64];
   tmem_ld64(taddr, v);
   sign_words2(v, w0, w1);
-}
-
-// acc += lo^2 + hi^2 for the two bf16 halves of u, with sm_100's mixed-precision
-// FMA (bf16 operands widened exactly, fp32 accumulate): no unpacking.
-__device__ __forceinline__ void sq_acc_bf16x2(uint32_t u, float& acc) {
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tfma.rn.f32.bf16 %0, lo, lo, %0;\n\t"
-      "fma.rn.f32.bf16 %0, hi, hi, %0;\n\t}"
-      : "+f"(acc)
-      : "r"(u));
 }
 
 __device__ __forceinline__ void flag_error(int* err, int code) { atomicOr(err, code); }
@@ -479,6 +473,10 @@ bool dense_tc_supported(const qjl_projection* P, int dtype, const void* keys, in
 }
 
 static_assert(sizeof(CUtensorMap) == sizeof(qjl_projection::s_map), "CUtensorMap size");
+
+bool qjl_make_bf16_map(void* map, const void* ptr, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+  return make_map(reinterpret_cast<CUtensorMap*>(map), ptr, rows, cols, ld, box_rows);
+}
 
 void dense_tc_prepare(qjl_projection* P) {
   P->s_map_ok = P->S_bf16 && make_map(reinterpret_cast<CUtensorMap*>(P->s_map), P->S_bf16, (uint64_t)P->m,

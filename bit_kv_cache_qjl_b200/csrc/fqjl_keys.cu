@@ -48,6 +48,7 @@
 
 #include "mbarrier.cuh"
 #include "philox.h"
+#include "key_math.cuh"
 #include "cache_hint.cuh"
 #include "qjl_internal.h"
 
@@ -59,63 +60,13 @@ using qjl_sync::mbar_fence_init;
 using qjl_sync::mbar_init;
 using qjl_sync::mbar_wait;
 using qjl_sync::smem_u32;
+using namespace qjl_km;
 
 constexpr int kMaxWarps = 8;
 constexpr size_t kTableBudget = 24 * 1024;   // shared bytes for the per-block tables of one launch
 constexpr size_t kSmemLimit = 227 * 1024;
 
 enum { MODE_P = 0, MODE_D = 1 };
-
-// ---- packed fp32 pair arithmetic (sm_100 f32x2) ----------------------------------------------
-
-// (a, b) <- (a + b, a - b), both lanes of the pair
-__device__ __forceinline__ void bfly2(float2& a, float2& b) {
-  asm("{\n\t.reg .b64 x, y, s, d;\n\t"
-      "mov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
-      "add.rn.f32x2 s, x, y;\n\tsub.rn.f32x2 d, x, y;\n\t"
-      "mov.b64 {%0, %1}, s;\n\tmov.b64 {%2, %3}, d;\n\t}"
-      : "+f"(a.x), "+f"(a.y), "+f"(b.x), "+f"(b.y));
-}
-
-// a <- a * b
-__device__ __forceinline__ void mul2(float2& a, float2 b) {
-  asm("{\n\t.reg .b64 x, y;\n\t"
-      "mov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
-      "mul.rn.f32x2 x, x, y;\n\t"
-      "mov.b64 {%0, %1}, x;\n\t}"
-      : "+f"(a.x), "+f"(a.y)
-      : "f"(b.x), "f"(b.y));
-}
-
-// a <- fma(a, b, +0): the product, with an exact zero always +0
-__device__ __forceinline__ void mulz2(float2& a, float2 b) {
-  asm("{\n\t.reg .b64 x, y, z;\n\t"
-      "mov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\tmov.b64 z, {%4, %4};\n\t"
-      "fma.rn.f32x2 x, x, y, z;\n\t"
-      "mov.b64 {%0, %1}, x;\n\t}"
-      : "+f"(a.x), "+f"(a.y)
-      : "f"(b.x), "f"(b.y), "f"(0.f));
-}
-
-// a <- fma(sg, a, p) with the same sign sg on both lanes
-__device__ __forceinline__ void sfma2(float2& a, float sg, float2 p) {
-  asm("{\n\t.reg .b64 x, s, q;\n\t"
-      "mov.b64 x, {%0, %1};\n\tmov.b64 s, {%2, %2};\n\tmov.b64 q, {%3, %4};\n\t"
-      "fma.rn.f32x2 x, s, x, q;\n\t"
-      "mov.b64 {%0, %1}, x;\n\t}"
-      : "+f"(a.x), "+f"(a.y)
-      : "f"(sg), "f"(p.x), "f"(p.y));
-}
-
-// acc += a * a (pairwise)
-__device__ __forceinline__ void sq_acc2(float2& acc, float2 a) {
-  asm("{\n\t.reg .b64 x, c;\n\t"
-      "mov.b64 x, {%2, %3};\n\tmov.b64 c, {%0, %1};\n\t"
-      "fma.rn.f32x2 c, x, x, c;\n\t"
-      "mov.b64 {%0, %1}, c;\n\t}"
-      : "+f"(acc.x), "+f"(acc.y)
-      : "f"(a.x), "f"(a.y));
-}
 
 // ---- transform ----------------------------------------------------------------------------------
 
@@ -147,27 +98,6 @@ __device__ __forceinline__ void fwht(float2 (&V)[E / 2], int lane) {
       sfma2(V[t], sg, p);
     }
   }
-}
-
-// ---- dither ------------------------------------------------------------------------------------
-
-// Box-Muller on 23-bit draws, scaled by amp: (amp r cos 2 pi v, amp r sin 2 pi v) with
-// u = ((xr >> 9) + 1/2) 2^-23 and v = (xa >> 9) 2^-23. Both draws are exact fp32 values:
-// u = (1 + k 2^-23) - (1 - 2^-24) is an exact subtraction. The angle is taken as 2 pi (1 + v),
-// which has the same sine and cosine.
-__device__ __forceinline__ void box_muller23(uint32_t xr, uint32_t xa, float amp, float& c, float& s) {
-  const float u = __uint_as_float((xr >> 9) | 0x3f800000u) - __uint_as_float(0x3f7fffffu);
-  const float f = __uint_as_float((xa >> 9) | 0x3f800000u);
-  float l, rs, sn, cs;
-  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(u));
-  const float t = -1.38629436f * l;  // -2 ln u > 0
-  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(rs) : "f"(t));
-  const float r = t * rs * amp;
-  const float th = 6.28318548f * f;
-  asm("sin.approx.ftz.f32 %0, %1;" : "=f"(sn) : "f"(th));
-  asm("cos.approx.ftz.f32 %0, %1;" : "=f"(cs) : "f"(th));
-  c = r * cs;
-  s = r * sn;
 }
 
 // ---- staging ------------------------------------------------------------------------------------
@@ -243,22 +173,6 @@ __device__ __forceinline__ void load_x(const unsigned char* xrow, int s, float2 
       V[t].x = a.x; V[t + 1].x = a.y; V[t + 2].x = a.z; V[t + 3].x = a.w;
       V[t].y = c.x; V[t + 1].y = c.y; V[t + 2].y = c.z; V[t + 3].y = c.w;
     }
-  }
-}
-
-// Philox4x32-10 on four counters at once, rounds interleaved for instruction-level parallelism.
-__device__ __forceinline__ void philox_x4(qjl::U32x4 (&c)[4], uint32_t k0, uint32_t k1) {
-#pragma unroll
-  for (int r = 0; r < 10; ++r) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t hA, lA, hB, lB;
-      qjl::mul_hi_lo(0xD2511F53u, c[j].x, hA, lA);
-      qjl::mul_hi_lo(0xCD9E8D57u, c[j].z, hB, lB);
-      c[j] = qjl::U32x4{hB ^ c[j].y ^ k0, lB, hA ^ c[j].w ^ k1, lA};
-    }
-    k0 += 0x9E3779B9u;
-    k1 += 0xBB67AE85u;
   }
 }
 

@@ -1,0 +1,466 @@
+// FQJL key sketch with the first randomized Hadamard transform on the
+// 5th-generation tensor cores (tcgen05 + TMA).
+//
+// "Fast Quantized Johnson - Lindenstrauss Transforms" ("Key concepts", "The
+// paper" abstract): block b of the sketch is z = H D_g Pi H D_r x, up to a
+// positive factor, with H the unnormalised Sylvester matrix and Pi the
+// gather u'[i] = u[pi(i)]. Its first factor S1 = Pi H D_r has entries +-1:
+// row i is row pi(i) of H with its columns signed by D_r. With bf16 keys
+// every product k_c S1[i][c] is exact, so u' = S1 x is a dense contraction
+// with exact operands and fp32 sums, run like the dense sketch: S1 resident
+// in shared memory, keys streamed by TMA, tcgen05 MMAs into TMEM. The second
+// factor H D_g is not exact in bf16 and stays on the FP32 lanes. Each
+// epilogue thread reads one key's accumulator row from TMEM, scales it by
+// D_g and runs the Walsh-Hadamard butterflies in registers. For d = 256 the
+// top butterfly, which pairs the two halves of the block, is fused with D_g
+// in a first sweep over the accumulator row, and each half is then
+// transformed with 128 points. The D-FQJL dither (Philox and Box-Muller per
+// coordinate) outweighs the transform by far and stays with the register
+// kernel (fqjl_keys.cu), whose eight warps per SM share it; this kernel
+// serves P-FQJL and D-FQJL without dither.
+//
+// Persistent kernel, one CTA per SM, 12 warps:
+//   warp 0     TMA producer: this pass's 256 rows of S1 once, then the keys as
+//              128-row x 64-column bf16 boxes (one 128-byte swizzle atom
+//              each) through an NS-slot ring, d/64 slots per 128-key tile.
+//   warp 1     allocates 512 TMEM columns (two 128 x 256 fp32 accumulators);
+//              one lane issues M=128, N=256, K=16 MMAs, four per slot.
+//   warps 2-9  epilogue. Warp w reads TMEM lanes 32 (w % 4) .. + 31, so each
+//              thread owns one key; the two warps on a lane quarter take 128
+//              of the pass's 256 coordinates each (a block of d = 128, or an
+//              output half of d = 256).
+//   warps 10-11 ||x|| from the swizzled key slots (as in the dense sketch).
+// A pass covers 256 output coordinates (one block of d = 256 or two of
+// d = 128). The host runs m/256 passes; each reads the keys again.
+//
+// No output bit comes from a -0. D_g is applied as fma(g, u, +0), or for the
+// fused top butterfly as fma(g, a, fma(+-g', b, +0)), so an exact zero is
+// +0. Sums of values that are not -0 are not -0, so the stored bit is exactly
+// [z >= 0].
+//
+// Every mbarrier wait is bounded. On expiry the kernel records an error flag,
+// drains what it issued, frees TMEM and returns.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "cache_hint.cuh"
+#include "key_math.cuh"
+#include "mbarrier.cuh"
+#include "qjl_internal.h"
+#include "tcgen05.cuh"
+
+namespace {
+
+using namespace qjl_km;
+using qjl_sync::mbar_arrive;
+using qjl_sync::mbar_expect_tx;
+using qjl_sync::mbar_fence_init;
+using qjl_sync::mbar_init;
+using qjl_sync::mbar_wait;
+using qjl_sync::smem_u32;
+
+constexpr int BM = 128;                   // keys per tile (MMA M)
+constexpr int kPass = 256;                // output coordinates per pass (MMA N)
+constexpr int kEpiWarps = 8;
+constexpr int kNormWarps = 2;
+constexpr int kThreads = (2 + kEpiWarps + kNormWarps) * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSlotBytes = BM * 128;  // 128 keys x 64 bf16 channels
+constexpr size_t kSmemLimit = 227 * 1024;
+
+struct FtcParams {
+  int64_t n;
+  int W;                 // sign words per key row
+  int pass;              // output coordinates 256 pass .. 256 pass + 255
+  int ns;                // ring slots
+  const float* D_g;      // [m], all blocks
+  uint32_t* bits;
+  float* norms;          // the first pass only, else nullptr
+  int* err;
+};
+
+__device__ __forceinline__ void flag_error(int* err, int code) { atomicOr(err, code); }
+
+// 128-point unnormalised Walsh-Hadamard transform in place, V[t] = (v_2t, v_2t+1):
+// the pair stage within registers, then six stages of packed butterflies.
+__device__ __forceinline__ void fwht128(float2 (&V)[64]) {
+#pragma unroll
+  for (int t = 0; t < 64; ++t) {
+    const float a = V[t].x, b = V[t].y;
+    V[t].x = a + b;
+    V[t].y = a - b;
+  }
+#pragma unroll
+  for (int h = 1; h < 64; h <<= 1) {
+#pragma unroll
+    for (int t = 0; t < 64; ++t)
+      if (!(t & h)) bfly2(V[t], V[t + h]);
+  }
+}
+
+// Sign words of 128 values: bit k of word j is 1 iff element 32 j + k >= 0. Eight
+// independent funnel-shift chains of 16 elements each.
+__device__ __forceinline__ void sign_words128(const float2 (&V)[64], uint32_t (&w)[4]) {
+  uint32_t c[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) c[k] = 0u;
+#pragma unroll
+  for (int i = 7; i >= 0; --i) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      c[k] = __funnelshift_l(__float_as_uint(V[8 * k + i].y), c[k], 1);
+      c[k] = __funnelshift_l(__float_as_uint(V[8 * k + i].x), c[k], 1);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) w[j] = ~(c[2 * j] | (c[2 * j + 1] << 16));
+}
+
+__device__ __forceinline__ float2 as_f2(uint32_t a, uint32_t b) {
+  return make_float2(__uint_as_float(a), __uint_as_float(b));
+}
+
+// The epilogue warp is done reading accumulator buffer `bar`'s TMEM columns.
+__device__ __forceinline__ void release_tmem(uint64_t* bar, int lane) {
+  qjl_tc::fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                            const __grid_constant__ CUtensorMap tmS,
+                                                            const FtcParams prm) {
+  static_assert(D == 128 || D == 256, "d in {128, 256}");
+  constexpr int KA = D / 64;  // key slots (64-column atoms) per tile
+  extern __shared__ __align__(1024) unsigned char smem_dyn[];
+  unsigned char* base = (unsigned char*)(((uintptr_t)smem_dyn + 1023) & ~(uintptr_t)1023);
+  const int NS = prm.ns;
+  unsigned char* sS = base;                                     // KA atoms x 256 rows x 128 B
+  unsigned char* ring = sS + (size_t)KA * kPass * 128;          // NS slots
+  float* sG = reinterpret_cast<float*>(ring + (size_t)NS * kSlotBytes);  // [2][256]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sG + 2 * kPass);
+  uint64_t* empty = full + NS;
+  uint64_t* tfull = empty + NS;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* sbar = tempty + 2;
+  uint64_t* dbar = sbar + 1;
+  uint64_t* xbar = dbar + 1;  // [4]: the two epilogue warps of a lane quarter, first sweep done
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xbar + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ntiles = (prm.n + BM - 1) / BM;
+
+  // D_g of this pass's coordinates. Row h scales the upper 128 by (+1, -1)[h]: the fused
+  // top butterfly of d = 256 reads row h for output half h. d = 128 reads row 0 only.
+  for (int i = threadIdx.x; i < 2 * kPass; i += blockDim.x) {
+    const int h = i / kPass, c = i % kPass;
+    const float g = __ldg(prm.D_g + (size_t)kPass * prm.pass + c);
+    sG[i] = (h == 1 && c >= 128) ? -g : g;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + kNormWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kEpiWarps);
+    }
+    mbar_init(sbar, 1);
+    mbar_init(dbar, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&xbar[q], 2);
+    mbar_fence_init();
+  }
+  if (warp == 1) qjl_tc::alloc(tmem_holder, kTmemCols);
+  qjl_tc::fence_before();
+  __syncthreads();
+  qjl_tc::fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(sbar, (uint32_t)(KA * kPass * 128));
+      for (int a = 0; a < KA; ++a) qjl_tc::tma_load_2d(sS + (size_t)a * kPass * 128, &tmS, sbar, a * 64, kPass * prm.pass);
+      int64_t issued = 0;
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        for (int a = 0; a < KA; ++a, ++issued) {
+          if (!mbar_wait(&empty[s], ph ^ 1u)) { flag_error(prm.err, 1); ok = false; break; }
+          mbar_expect_tx(&full[s], kSlotBytes);
+          qjl_tc::tma_load_2d(ring + (size_t)s * kSlotBytes, &tmK, &full[s], a * 64, (int)(t * BM));
+          if (++s == NS) { s = 0; ph ^= 1u; }
+        }
+      }
+      // drain: the most recent phase of every used slot must have landed before exit
+      const int used = issued < NS ? (int)issued : NS;
+      for (int j = 0; j < used; ++j) {
+        int st = s - 1 - j;
+        uint32_t p = ph;
+        if (st < 0) { st += NS; p ^= 1u; }
+        if (!mbar_wait(&full[st], p)) flag_error(prm.err, 2);
+      }
+      if (!mbar_wait(sbar, 0)) flag_error(prm.err, 2);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = mbar_wait(sbar, 0);
+      if (!ok) flag_error(prm.err, 4);
+      const uint32_t idesc = qjl_tc::idesc_bf16(kPass);
+      const uint32_t sS_addr = smem_u32(sS);
+      uint32_t u = 0;
+      int s = 0;
+      uint32_t ph = 0;
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++u) {
+        const int buf = (int)(u & 1u);
+        if (!mbar_wait(&tempty[buf], ((u >> 1) & 1u) ^ 1u)) { flag_error(prm.err, 4); break; }
+        qjl_tc::fence_after();
+        const uint32_t dcol = tmem_base + (uint32_t)(buf * 256);
+        for (int a = 0; a < KA; ++a) {
+          if (!mbar_wait(&full[s], ph)) { flag_error(prm.err, 4); ok = false; break; }
+          qjl_tc::fence_after();
+          const uint32_t a_addr = smem_u32(ring + (size_t)s * kSlotBytes);
+          const uint32_t b_addr = sS_addr + (uint32_t)(a * kPass * 128);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            qjl_tc::mma_bf16_ss(dcol, qjl_tc::sw128_desc(a_addr + 32u * kk), qjl_tc::sw128_desc(b_addr + 32u * kk),
+                                idesc, (a | kk) ? 1u : 0u);
+          qjl_tc::commit(&empty[s]);
+          if (++s == NS) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        qjl_tc::commit(&tfull[buf]);
+      }
+      // every MMA this thread issued has completed before TMEM is released
+      qjl_tc::commit(dbar);
+      if (!mbar_wait(dbar, 0)) flag_error(prm.err, 8);
+    }
+  } else if (warp < 2 + kEpiWarps) {
+    const int quarter = warp & 3;
+    const int part = (warp - 2) >> 2;  // this warp's 128 coordinates of the pass
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_base = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    const uint64_t pol = qjl_hint::evict_first();
+    uint32_t u = 0;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++u) {
+      const int buf = (int)(u & 1u);
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (u >> 1) & 1u))) { flag_error(prm.err, 16); break; }
+      qjl_tc::fence_after();
+      const int64_t row = t * BM + r;
+      const uint32_t tb = lane_base + (uint32_t)(buf * 256);
+      if constexpr (D == 256) {
+        // One block of 256: output half h is the 128-point transform of
+        // v_h,i = g_i u'_i + (+-1)[h] g_{i+128} u'_{i+128}, i < 128. First sweep: this warp forms
+        // both halves for i in [64 part, 64 part + 64) and writes them back in place, v_0 over
+        // u'[0, 128) and v_1 over u'[128, 256), 32 columns at a time. Once the other warp of the
+        // quarter has done the same, it reads its half back whole.
+#pragma unroll 1
+        for (int rr = 0; rr < 2; ++rr) {
+          const int i0 = 64 * part + 32 * rr;
+          uint32_t A[32], B[32];
+          qjl_tc::ld32(tb + i0, A);
+          qjl_tc::ld32(tb + 128u + i0, B);
+          qjl_tc::wait_ld();
+#pragma unroll
+          for (int q = 0; q < 16; q += 2) {
+            const int c = i0 + 2 * q;
+            const float4 ga = *reinterpret_cast<const float4*>(sG + c);
+            const float4 gp = *reinterpret_cast<const float4*>(sG + 128 + c);          // +g_{i+128}
+            const float4 gn = *reinterpret_cast<const float4*>(sG + kPass + 128 + c);  // -g_{i+128}
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float2 g0 = e ? make_float2(ga.z, ga.w) : make_float2(ga.x, ga.y);
+              const float2 g1 = e ? make_float2(gp.z, gp.w) : make_float2(gp.x, gp.y);
+              const float2 g2 = e ? make_float2(gn.z, gn.w) : make_float2(gn.x, gn.y);
+              const int k = 2 * (q + e);
+              const float2 a = as_f2(A[k], A[k + 1]), b = as_f2(B[k], B[k + 1]);
+              float2 p = b, n = b, v0 = a, v1 = a;
+              mulz2(p, g1);
+              mulz2(n, g2);
+              fma2(v0, g0, p);
+              fma2(v1, g0, n);
+              A[k] = __float_as_uint(v0.x);
+              A[k + 1] = __float_as_uint(v0.y);
+              B[k] = __float_as_uint(v1.x);
+              B[k + 1] = __float_as_uint(v1.y);
+            }
+          }
+          qjl_tc::st32(tb + i0, A);
+          qjl_tc::st32(tb + 128u + i0, B);
+        }
+        qjl_tc::wait_st();
+        qjl_tc::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xbar[quarter]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&xbar[quarter], u & 1u))) { flag_error(prm.err, 16); break; }
+        qjl_tc::fence_after();
+      }
+      // this warp's 128 coordinates: columns 128 part .. 128 part + 127 (a block of d = 128 scaled
+      // by D_g here, or a half of d = 256 formed by the sweep)
+      uint32_t R[128];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) qjl_tc::ld32(tb + 128u * part + 32u * j, R + 32 * j);
+      qjl_tc::wait_ld();
+      release_tmem(&tempty[buf], lane);
+      float2 V[64];
+#pragma unroll
+      for (int q = 0; q < 64; ++q) V[q] = as_f2(R[2 * q], R[2 * q + 1]);
+      if constexpr (D == 128) {
+        const float* g = sG + 128 * part;
+#pragma unroll
+        for (int q = 0; q < 64; q += 2) {
+          const float4 gg = *reinterpret_cast<const float4*>(g + 2 * q);
+          mulz2(V[q], make_float2(gg.x, gg.y));
+          mulz2(V[q + 1], make_float2(gg.z, gg.w));
+        }
+      }
+      fwht128(V);
+      uint32_t w[4];
+      sign_words128(V, w);
+      if (row < prm.n) qjl_hint::st_v4(prm.bits + row * (int64_t)prm.W + 8 * prm.pass + 4 * part, w[0], w[1], w[2], w[3], pol);
+    }
+  } else {
+    // norm warps: ||x|| of rows r0 and r0 + 64 of each tile from the swizzled key slots
+    // (16-byte chunk c of row r sits at chunk c ^ (r % 8)), then the slot is released
+    // together with the MMAs' commit
+    const int r0 = (warp - 2 - kEpiWarps) * 32 + lane;
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      float acc[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[j][k] = 0.f;
+      for (int a = 0; a < KA; ++a) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { flag_error(prm.err, 32); ok = false; break; }
+        const unsigned char* slot = ring + (size_t)s * kSlotBytes;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int rr = r0 + 64 * j;
+            const uint4 v = *reinterpret_cast<const uint4*>(slot + rr * 128 + ((c ^ (rr & 7)) << 4));
+            sq_acc_bf16x2(v.x, acc[j][0]);
+            sq_acc_bf16x2(v.y, acc[j][1]);
+            sq_acc_bf16x2(v.z, acc[j][2]);
+            sq_acc_bf16x2(v.w, acc[j][3]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (++s == NS) { s = 0; ph ^= 1u; }
+      }
+      if (!ok || !prm.norms) continue;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int64_t row = t * BM + r0 + 64 * j;
+        if (row < prm.n)
+          qjl_hint::st_f32(prm.norms + row, sqrtf((acc[j][0] + acc[j][1]) + (acc[j][2] + acc[j][3])),
+                           qjl_hint::evict_first());
+      }
+    }
+  }
+  qjl_tc::fence_before();
+  __syncthreads();
+  qjl_tc::fence_after();
+  if (warp == 1) qjl_tc::dealloc(tmem_base, kTmemCols);
+}
+
+size_t smem_bytes(int d, int ns) {
+  return 1024 + (size_t)(d / 64) * kPass * 128 + (size_t)ns * kSlotBytes + 2 * kPass * 4 + (2 * ns + 10) * 8 + 16;
+}
+
+int pick_slots(int d) {
+  for (int ns = 8; ns >= 3; --ns)
+    if (smem_bytes(d, ns) <= kSmemLimit) return ns;
+  return 0;
+}
+
+}  // namespace
+
+bool fqjl_tc_shape(int d, int m, bool dg_outer) {
+  return (d == 128 || d == 256) && m % kPass == 0 && !dg_outer && pick_slots(d) > 0;
+}
+
+// S1 [m][d] as bf16 bit patterns: row b d + i is row pi_b(i) of H, column c times D_r^b[c];
+// H[p][c] = (-1)^popcount(p & c) (Sylvester order).
+std::vector<uint16_t> fqjl_tc_matrix(int d, int m, const float* D_r, const int32_t* perm) {
+  std::vector<uint16_t> s1((size_t)m * d);
+  for (int b = 0; b < m / d; ++b)
+    for (int i = 0; i < d; ++i) {
+      const int p = perm[(size_t)b * d + i];
+      uint16_t* row = s1.data() + ((size_t)b * d + i) * d;
+      for (int c = 0; c < d; ++c) {
+        const bool neg = (__builtin_popcount((unsigned)(p & c)) & 1) != (D_r[(size_t)b * d + c] < 0.f);
+        row[c] = neg ? 0xBF80u : 0x3F80u;
+      }
+    }
+  return s1;
+}
+
+void fqjl_tc_prepare(qjl_projection* P) {
+  P->s_map_ok = P->S1_bf16 && qjl_make_bf16_map(P->s_map, P->S1_bf16, (uint64_t)P->m, (uint64_t)P->d,
+                                                (uint64_t)P->d, (uint32_t)kPass);
+}
+
+bool fqjl_tc_supported(const qjl_projection* P, int dtype, int64_t n) {
+  // the D-FQJL dither stays with the register kernel
+  const bool dither = P->kind == QJL_DFQJL && P->dither_sigma != 0.f;
+  return P->kind != QJL_DENSE && !dither && P->S1_bf16 && P->s_map_ok && dtype == QJL_BF16 &&
+         fqjl_tc_shape(P->d, P->m, P->opt.dg_outer != 0) && n <= (int64_t)INT32_MAX - BM;
+}
+
+qjl_status launch_fqjl_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld, uint32_t* bits,
+                          float* norms, cudaStream_t st) {
+  if (n <= 0) return QJL_OK;
+  // the keys' map is cached per thread for the last (pointer, rows, ld, d), as in the dense sketch
+  struct KeyMapCache {
+    const void* ptr = nullptr;
+    int64_t n = -1, ld = -1;
+    int d = -1;
+    alignas(64) unsigned char map[128];
+  };
+  static thread_local KeyMapCache kc;
+  if (kc.ptr != keys || kc.n != n || kc.ld != ld || kc.d != P->d) {
+    kc.ptr = nullptr;
+    if (!qjl_make_bf16_map(kc.map, keys, (uint64_t)n, (uint64_t)P->d, (uint64_t)ld, BM))
+      return qjl_set_error(QJL_ERR_CUDA, "cuTensorMapEncodeTiled failed for the keys");
+    kc.ptr = keys;
+    kc.n = n;
+    kc.ld = ld;
+    kc.d = P->d;
+  }
+  CUtensorMap tmK, tmS;
+  memcpy(&tmK, kc.map, sizeof(tmK));
+  memcpy(&tmS, P->s_map, sizeof(tmS));
+  int* err = qjl_error_flag(P->device);
+  if (!err) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
+  const int ns = pick_slots(P->d);
+  const size_t smem = smem_bytes(P->d, ns);
+  void (*kern)(CUtensorMap, CUtensorMap, FtcParams) = P->d == 128 ? fqjl_tc_kernel<128> : fqjl_tc_kernel<256>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return qjl_check_launch("fqjl_tc_kernel smem attribute");
+  const int64_t ntiles = (n + BM - 1) / BM;
+  const int grid = (int)std::min<int64_t>(ntiles, qjl_num_sms(P->device));
+  FtcParams prm{n, P->m / 32, 0, ns, P->D_g, bits, norms, err};
+  for (int pass = 0; pass < P->m / kPass; ++pass) {
+    prm.pass = pass;
+    prm.norms = pass == 0 ? norms : nullptr;
+    qjl_log_launch("fqjl_tc_kernel", grid, kThreads, smem, 1);
+    kern<<<grid, kThreads, smem, st>>>(tmK, tmS, prm);
+    const qjl_status s = qjl_check_launch("fqjl_tc_kernel");
+    if (s != QJL_OK) return s;
+  }
+  return QJL_OK;
+}

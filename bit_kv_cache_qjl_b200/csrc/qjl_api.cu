@@ -142,6 +142,7 @@ void free_projection(qjl_projection* P) {
   cudaFree(P->perm);
   cudaFree(P->D_g);
   cudaFree(P->ktab);
+  cudaFree(P->S1_bf16);
   free(P->h_S);
   free(P->h_D_r);
   free(P->h_perm);
@@ -274,6 +275,11 @@ qjl_status qjl_make_projection(uint64_t seed, int d, int m, qjl_kind kind, const
       const std::vector<float> kt = fqjl_key_tables(d, m, P->h_D_r, P->h_perm, P->h_D_g);
       st = dev_upload(&P->ktab, kt.data(), kt.size());
     }
+    if (st == QJL_OK && fqjl_tc_shape(d, m, o.dg_outer != 0)) {
+      const std::vector<uint16_t> s1 = fqjl_tc_matrix(d, m, P->h_D_r, P->h_perm);
+      st = dev_upload(&P->S1_bf16, s1.data(), s1.size());
+      if (st == QJL_OK) fqjl_tc_prepare(P);
+    }
   }
   if (st != QJL_OK) {
     free_projection(P);
@@ -339,6 +345,7 @@ qjl_status qjl_quantize_keys(const qjl_projection* P, const void* keys, qjl_dtyp
     if (dense_tc_supported(P, dtype, keys, ld)) return launch_dense_tc(P, keys, n, ld, bits, norms, st);
     return launch_dense_simt(P, keys, dtype, n, ld, bits, norms, nullptr, st);
   }
+  if (fqjl_tc_supported(P, dtype, n)) return launch_fqjl_tc(P, keys, n, ld, bits, norms, st);
   return launch_fqjl_keys(P, keys, dtype, n, ld, first_token, bits, norms, st);
 }
 

@@ -23,8 +23,10 @@ struct qjl_projection {
   int32_t* perm = nullptr;
   float* D_g = nullptr;
   float* ktab = nullptr;        // key-kernel tables, per block (fqjl_key_tables)
-  // the tensor map of S_bf16 for the tcgen05 quantize kernel (a CUtensorMap),
-  // encoded once when the projection is made; s_map_ok is false if that failed
+  uint16_t* S1_bf16 = nullptr;  // [m][d] bf16 +-1: row b*d + i is row pi_b(i) of H times D_r^b (fqjl_tc.cu)
+  // the tensor map of S_bf16 (dense) or S1_bf16 (FQJL) for the tcgen05 quantize
+  // kernels (a CUtensorMap), encoded once when the projection is made;
+  // s_map_ok is false if that failed
   alignas(64) unsigned char s_map[128] = {};
   bool s_map_ok = false;
   // host copies for export
@@ -103,6 +105,22 @@ bool dense_tc_supported(const qjl_projection* P, int dtype, const void* keys, in
 void dense_tc_prepare(qjl_projection* P);
 qjl_status launch_dense_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld,
                            uint32_t* bits, float* norms, cudaStream_t st);
+// 2-D bf16 tensor map (a CUtensorMap written to `map`, 128 bytes, 64-byte
+// aligned): rows x cols, row stride ld elements, boxes of 64 columns x
+// box_rows rows with 128-byte swizzle. False if the encoder is unavailable or
+// rejects the arguments.
+bool qjl_make_bf16_map(void* map, const void* ptr, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows);
+// FQJL keys with the first randomized Hadamard transform on tcgen05
+// (fqjl_tc.cu): bf16 keys, d in {128, 256}, m a multiple of 256, the default
+// order, no dither, not a paged append. When the projection is made, fqjl_tc_shape
+// decides whether it gets S1 (fqjl_tc_matrix, uploaded to S1_bf16), and
+// fqjl_tc_prepare encodes S1's tensor map into s_map.
+bool fqjl_tc_shape(int d, int m, bool dg_outer);
+std::vector<uint16_t> fqjl_tc_matrix(int d, int m, const float* D_r, const int32_t* perm);
+void fqjl_tc_prepare(qjl_projection* P);
+bool fqjl_tc_supported(const qjl_projection* P, int dtype, int64_t n);
+qjl_status launch_fqjl_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld, uint32_t* bits,
+                          float* norms, cudaStream_t st);
 qjl_status launch_fqjl_queries(const qjl_projection* P, const float* q, int64_t nq, int64_t ld,
                                float* out, cudaStream_t st);
 std::vector<float> fqjl_key_tables(int d, int m, const float* D_r, const int32_t* perm, const float* D_g);

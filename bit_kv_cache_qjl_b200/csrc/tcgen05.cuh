@@ -68,6 +68,42 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// Shared-memory descriptor of a K-major operand in 128-byte swizzled atoms
+// (8 rows x 128 bytes, 1024 bytes per 8-row group), as a 2-D TMA load with
+// 128-byte swizzle writes it. A K slice inside the atom is addressed by
+// advancing the start address by its byte offset.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t desc = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  desc |= (uint64_t)1u << 16;
+  desc |= (uint64_t)(1024u >> 4) << 32;
+  desc |= (uint64_t)1u << 46;
+  desc |= (uint64_t)2u << 61;
+  return desc;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B (K-major), fp32 D, M = 128, N columns.
+__host__ __device__ constexpr uint32_t idesc_bf16(int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] . B[smem], kind::f16, cta_group::1.
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// 2-D tiled TMA load (no multicast) of the box at (x, y), completion counted on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+          "r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
 // This thread's TMEM lane, 32 consecutive 32-bit columns from `taddr`.
 __device__ __forceinline__ void st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(

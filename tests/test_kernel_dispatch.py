@@ -42,9 +42,26 @@ def test_fp32_keys_use_simt_kernel(cuda_ok):
 
 
 def test_fqjl_kernels(cuda_ok):
+    # bf16 keys with d in {128, 256} and m a multiple of 256: the tcgen05 kernel, one launch per 256 coordinates
     P = qjl.Projection(4, 256, 1024, "pfqjl")
     keys = wl.normal((512, 256), 1, "cuda", torch.bfloat16)
-    assert _has(_kernels(lambda: qjl.quantize_keys(P, keys)), "fqjl_keys_kernel")
+    names = _kernels(lambda: qjl.quantize_keys(P, keys))
+    assert sum("fqjl_tc_kernel" in n for n in names) == 4, names
+    assert not _has(names, "fqjl_keys_kernel")
+    D0 = qjl.Projection(5, 128, 256, "dfqjl", dither_sigma_rel=0.0)
+    names = _kernels(lambda: qjl.quantize_keys(D0, wl.normal((300, 128), 3, "cuda", torch.bfloat16)))
+    assert sum("fqjl_tc_kernel" in n for n in names) == 1, names
+    # the dither, fp32 keys, other widths and the literal order keep the register Walsh-Hadamard kernel
+    D = qjl.Projection(5, 128, 256, "dfqjl")
+    assert _has(_kernels(lambda: qjl.quantize_keys(D, wl.normal((300, 128), 3, "cuda", torch.bfloat16))),
+                "fqjl_keys_kernel")
+    assert _has(_kernels(lambda: qjl.quantize_keys(P, keys.float())), "fqjl_keys_kernel")
+    E = qjl.Projection(4, 512, 1024, "pfqjl")
+    assert _has(_kernels(lambda: qjl.quantize_keys(E, wl.normal((64, 512), 4, "cuda", torch.bfloat16))),
+                "fqjl_keys_kernel")
+    F = qjl.Projection(4, 128, 256, "pfqjl", dg_outer=True)
+    assert _has(_kernels(lambda: qjl.quantize_keys(F, wl.normal((64, 128), 5, "cuda", torch.bfloat16))),
+                "fqjl_keys_kernel")
     q = wl.normal((3, 256), 2, "cuda")
     assert _has(_kernels(lambda: qjl.project_queries(P, q)), "fqjl_query_kernel")
 

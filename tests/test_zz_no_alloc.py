@@ -114,7 +114,7 @@ sys.path.insert(0, sys.argv[1])
 import bit_kv_cache_qjl_b200 as qjl
 from bit_kv_cache_qjl_b200 import lib
 torch.cuda.init()
-P = qjl.Projection(5, 128, 256, "dfqjl")       # its four parameter uploads are the only ones allowed
+P = qjl.Projection(5, 128, 256, "dfqjl")       # its five parameter uploads are the only ones allowed
 G, N, J, d, m = 8, 1500, 1, 128, 256
 g = torch.Generator(device="cuda").manual_seed(77)
 bits = torch.randint(-2**31, 2**31 - 1, (G, N, m // 32), dtype=torch.int32, device="cuda", generator=g)
@@ -145,7 +145,7 @@ print("fresh-process no-alloc ok")
 
 
 def test_noalloc_first_call_in_fresh_process_with_allocations_refused(cuda_ok):
-    env = dict(os.environ, QJL_FAIL_ALLOC_AFTER="4")
+    env = dict(os.environ, QJL_FAIL_ALLOC_AFTER="5")
     r = subprocess.run([sys.executable, "-c", _FRESH, ROOT], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-3000:]
     assert "fresh-process no-alloc ok" in r.stdout
