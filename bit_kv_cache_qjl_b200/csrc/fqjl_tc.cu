@@ -70,7 +70,12 @@ constexpr int BM = 128;                   // keys per tile (MMA M)
 constexpr int kPass = 256;                // output coordinates per pass (MMA N)
 constexpr int kEpiWarps = 8;
 constexpr int kNormWarps = 2;
-constexpr int kThreads = (2 + kEpiWarps + kNormWarps) * 32;
+constexpr int kThreads = (2 + kNormWarps + kEpiWarps) * 32;  // 384: 168 registers a thread at launch
+// Register split by warpgroup (setmaxnreg, d = 128; it measured slower for d = 256): the
+// producer, MMA and norm warps give theirs up for the epilogue's 128-value rows: 128 x 56 + 256 x 224 = 64512, the launch's 384 x 168.
+constexpr int kRegsLow = 56;
+constexpr int kRegsHigh = 224;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * 168, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotBytes = BM * 128;  // 128 keys x 64 bf16 channels
 constexpr size_t kSmemLimit = 227 * 1024;
@@ -81,6 +86,9 @@ struct FtcParams {
   int pass;              // output coordinates 256 pass .. 256 pass + 255
   int ns;                // ring slots
   const float* D_g;      // [m], all blocks
+  float sigma;           // D-FQJL dither sigma_rel (the dithered instantiation)
+  uint32_t k0, k1;       // the seed as the Philox key
+  uint64_t first_token;  // token index of row 0 (the dither's counter)
   uint32_t* bits;
   float* norms;          // the first pass only, else nullptr
   int* err;
@@ -123,6 +131,32 @@ __device__ __forceinline__ void sign_words128(const float2 (&V)[64], uint32_t (&
   for (int j = 0; j < 4; ++j) w[j] = ~(c[2 * j] | (c[2 * j + 1] << 16));
 }
 
+// D-FQJL dither of coordinates e0 .. e0 + 127 of token tok, scaled by amp, added to V: the
+// register kernel's draw (fqjl_keys.cu). Coordinate e comes from the Philox4x32-10 block at
+// counter (e/4, tok_lo, tok_hi, dither stream): words (0, 1) give coordinates 4c, 4c + 1 and
+// words (2, 3) give 4c + 2, 4c + 3, by Box-Muller on 23-bit draws.
+__device__ __forceinline__ void add_dither(float2 (&V)[64], uint32_t e0, uint64_t tok, float amp, uint32_t k0,
+                                           uint32_t k1) {
+  const uint32_t cb = e0 >> 2, tlo = (uint32_t)tok, thi = (uint32_t)(tok >> 32);
+#pragma unroll
+  for (int c = 0; c < 32; c += 4) {
+    qjl::U32x4 w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) w[j] = qjl::U32x4{cb + c + j, tlo, thi, qjl::kStreamDither};
+    philox_x4(w, k0, k1);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float xi[4];
+      box_muller23(w[j].x, w[j].y, amp, xi[0], xi[1]);
+      box_muller23(w[j].z, w[j].w, amp, xi[2], xi[3]);
+      V[2 * (c + j)].x += xi[0];
+      V[2 * (c + j)].y += xi[1];
+      V[2 * (c + j) + 1].x += xi[2];
+      V[2 * (c + j) + 1].y += xi[3];
+    }
+  }
+}
+
 __device__ __forceinline__ float2 as_f2(uint32_t a, uint32_t b) {
   return make_float2(__uint_as_float(a), __uint_as_float(b));
 }
@@ -134,11 +168,12 @@ __device__ __forceinline__ void release_tmem(uint64_t* bar, int lane) {
   if (lane == 0) mbar_arrive(bar);
 }
 
-template <int D>
+template <int D, bool DITHER>
 __global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                             const __grid_constant__ CUtensorMap tmS,
                                                             const FtcParams prm) {
   static_assert(D == 128 || D == 256, "d in {128, 256}");
+  static_assert(!DITHER || D == 128, "the dithered instantiation is d = 128");
   constexpr int KA = D / 64;  // key slots (64-column atoms) per tile
   extern __shared__ __align__(1024) unsigned char smem_dyn[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_dyn + 1023) & ~(uintptr_t)1023);
@@ -185,68 +220,114 @@ __global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_const
   qjl_tc::fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_expect_tx(sbar, (uint32_t)(KA * kPass * 128));
-      for (int a = 0; a < KA; ++a) qjl_tc::tma_load_2d(sS + (size_t)a * kPass * 128, &tmS, sbar, a * 64, kPass * prm.pass);
-      int64_t issued = 0;
+  if (warp < 4) {
+    if constexpr (D == 128) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+    if (warp == 0) {
+      if (lane == 0) {
+        mbar_expect_tx(sbar, (uint32_t)(KA * kPass * 128));
+        for (int a = 0; a < KA; ++a) qjl_tc::tma_load_2d(sS + (size_t)a * kPass * 128, &tmS, sbar, a * 64, kPass * prm.pass);
+        int64_t issued = 0;
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+          for (int a = 0; a < KA; ++a, ++issued) {
+            if (!mbar_wait(&empty[s], ph ^ 1u)) { flag_error(prm.err, 1); ok = false; break; }
+            mbar_expect_tx(&full[s], kSlotBytes);
+            qjl_tc::tma_load_2d(ring + (size_t)s * kSlotBytes, &tmK, &full[s], a * 64, (int)(t * BM));
+            if (++s == NS) { s = 0; ph ^= 1u; }
+          }
+        }
+        // drain: the most recent phase of every used slot must have landed before exit
+        const int used = issued < NS ? (int)issued : NS;
+        for (int j = 0; j < used; ++j) {
+          int st = s - 1 - j;
+          uint32_t p = ph;
+          if (st < 0) { st += NS; p ^= 1u; }
+          if (!mbar_wait(&full[st], p)) flag_error(prm.err, 2);
+        }
+        if (!mbar_wait(sbar, 0)) flag_error(prm.err, 2);
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {
+        bool ok = mbar_wait(sbar, 0);
+        if (!ok) flag_error(prm.err, 4);
+        const uint32_t idesc = qjl_tc::idesc_bf16(kPass);
+        const uint32_t sS_addr = smem_u32(sS);
+        uint32_t u = 0;
+        int s = 0;
+        uint32_t ph = 0;
+        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++u) {
+          const int buf = (int)(u & 1u);
+          if (!mbar_wait(&tempty[buf], ((u >> 1) & 1u) ^ 1u)) { flag_error(prm.err, 4); break; }
+          qjl_tc::fence_after();
+          const uint32_t dcol = tmem_base + (uint32_t)(buf * 256);
+          for (int a = 0; a < KA; ++a) {
+            if (!mbar_wait(&full[s], ph)) { flag_error(prm.err, 4); ok = false; break; }
+            qjl_tc::fence_after();
+            const uint32_t a_addr = smem_u32(ring + (size_t)s * kSlotBytes);
+            const uint32_t b_addr = sS_addr + (uint32_t)(a * kPass * 128);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              qjl_tc::mma_bf16_ss(dcol, qjl_tc::sw128_desc(a_addr + 32u * kk), qjl_tc::sw128_desc(b_addr + 32u * kk),
+                                  idesc, (a | kk) ? 1u : 0u);
+            qjl_tc::commit(&empty[s]);
+            if (++s == NS) { s = 0; ph ^= 1u; }
+          }
+          if (!ok) break;
+          qjl_tc::commit(&tfull[buf]);
+        }
+        // every MMA this thread issued has completed before TMEM is released
+        qjl_tc::commit(dbar);
+        if (!mbar_wait(dbar, 0)) flag_error(prm.err, 8);
+      }
+    } else {
+      // norm warps: ||x|| of rows r0 and r0 + 64 of each tile from the swizzled key slots
+      // (16-byte chunk c of row r sits at chunk c ^ (r % 8)), then the slot is released
+      // together with the MMAs' commit
+      const int r0 = (warp - 2) * 32 + lane;
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        for (int a = 0; a < KA; ++a, ++issued) {
-          if (!mbar_wait(&empty[s], ph ^ 1u)) { flag_error(prm.err, 1); ok = false; break; }
-          mbar_expect_tx(&full[s], kSlotBytes);
-          qjl_tc::tma_load_2d(ring + (size_t)s * kSlotBytes, &tmK, &full[s], a * 64, (int)(t * BM));
-          if (++s == NS) { s = 0; ph ^= 1u; }
-        }
-      }
-      // drain: the most recent phase of every used slot must have landed before exit
-      const int used = issued < NS ? (int)issued : NS;
-      for (int j = 0; j < used; ++j) {
-        int st = s - 1 - j;
-        uint32_t p = ph;
-        if (st < 0) { st += NS; p ^= 1u; }
-        if (!mbar_wait(&full[st], p)) flag_error(prm.err, 2);
-      }
-      if (!mbar_wait(sbar, 0)) flag_error(prm.err, 2);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      bool ok = mbar_wait(sbar, 0);
-      if (!ok) flag_error(prm.err, 4);
-      const uint32_t idesc = qjl_tc::idesc_bf16(kPass);
-      const uint32_t sS_addr = smem_u32(sS);
-      uint32_t u = 0;
-      int s = 0;
-      uint32_t ph = 0;
-      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++u) {
-        const int buf = (int)(u & 1u);
-        if (!mbar_wait(&tempty[buf], ((u >> 1) & 1u) ^ 1u)) { flag_error(prm.err, 4); break; }
-        qjl_tc::fence_after();
-        const uint32_t dcol = tmem_base + (uint32_t)(buf * 256);
-        for (int a = 0; a < KA; ++a) {
-          if (!mbar_wait(&full[s], ph)) { flag_error(prm.err, 4); ok = false; break; }
-          qjl_tc::fence_after();
-          const uint32_t a_addr = smem_u32(ring + (size_t)s * kSlotBytes);
-          const uint32_t b_addr = sS_addr + (uint32_t)(a * kPass * 128);
+        float acc[2][4];
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            qjl_tc::mma_bf16_ss(dcol, qjl_tc::sw128_desc(a_addr + 32u * kk), qjl_tc::sw128_desc(b_addr + 32u * kk),
-                                idesc, (a | kk) ? 1u : 0u);
-          qjl_tc::commit(&empty[s]);
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc[j][k] = 0.f;
+        for (int a = 0; a < KA; ++a) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { flag_error(prm.err, 32); ok = false; break; }
+          const unsigned char* slot = ring + (size_t)s * kSlotBytes;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int rr = r0 + 64 * j;
+              const uint4 v = *reinterpret_cast<const uint4*>(slot + rr * 128 + ((c ^ (rr & 7)) << 4));
+              sq_acc_bf16x2(v.x, acc[j][0]);
+              sq_acc_bf16x2(v.y, acc[j][1]);
+              sq_acc_bf16x2(v.z, acc[j][2]);
+              sq_acc_bf16x2(v.w, acc[j][3]);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
           if (++s == NS) { s = 0; ph ^= 1u; }
         }
-        if (!ok) break;
-        qjl_tc::commit(&tfull[buf]);
+        if (!ok || !prm.norms) continue;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int64_t row = t * BM + r0 + 64 * j;
+          if (row < prm.n)
+            qjl_hint::st_f32(prm.norms + row, sqrtf((acc[j][0] + acc[j][1]) + (acc[j][2] + acc[j][3])),
+                             qjl_hint::evict_first());
+        }
       }
-      // every MMA this thread issued has completed before TMEM is released
-      qjl_tc::commit(dbar);
-      if (!mbar_wait(dbar, 0)) flag_error(prm.err, 8);
     }
-  } else if (warp < 2 + kEpiWarps) {
+  } else {
+    if constexpr (D == 128) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
     const int quarter = warp & 3;
-    const int part = (warp - 2) >> 2;  // this warp's 128 coordinates of the pass
+    const int part = (warp - 4) >> 2;  // this warp's 128 coordinates of the pass
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = tmem_base + ((uint32_t)(quarter * 32) << 16);
     const uint64_t pol = qjl_hint::evict_first();
@@ -314,6 +395,14 @@ __global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_const
       float2 V[64];
 #pragma unroll
       for (int q = 0; q < 64; ++q) V[q] = as_f2(R[2 * q], R[2 * q + 1]);
+      float amp = 0.f;
+      if constexpr (DITHER) {
+        // ||S1 x||^2 = d ||x||^2 over a block, so sqrt(d) sigma_rel ||x|| = sigma_rel ||u'||
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 64; ++q) sq_acc2(acc, V[q]);
+        amp = prm.sigma * sqrtf(acc.x + acc.y);
+      }
       if constexpr (D == 128) {
         const float* g = sG + 128 * part;
 #pragma unroll
@@ -324,51 +413,12 @@ __global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_const
         }
       }
       fwht128(V);
+      if (DITHER && amp != 0.f)
+        add_dither(V, (uint32_t)(kPass * prm.pass + 128 * part), prm.first_token + (uint64_t)row, amp, prm.k0,
+                   prm.k1);
       uint32_t w[4];
       sign_words128(V, w);
       if (row < prm.n) qjl_hint::st_v4(prm.bits + row * (int64_t)prm.W + 8 * prm.pass + 4 * part, w[0], w[1], w[2], w[3], pol);
-    }
-  } else {
-    // norm warps: ||x|| of rows r0 and r0 + 64 of each tile from the swizzled key slots
-    // (16-byte chunk c of row r sits at chunk c ^ (r % 8)), then the slot is released
-    // together with the MMAs' commit
-    const int r0 = (warp - 2 - kEpiWarps) * 32 + lane;
-    int s = 0;
-    uint32_t ph = 0;
-    bool ok = true;
-    for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-      float acc[2][4];
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[j][k] = 0.f;
-      for (int a = 0; a < KA; ++a) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) { flag_error(prm.err, 32); ok = false; break; }
-        const unsigned char* slot = ring + (size_t)s * kSlotBytes;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int rr = r0 + 64 * j;
-            const uint4 v = *reinterpret_cast<const uint4*>(slot + rr * 128 + ((c ^ (rr & 7)) << 4));
-            sq_acc_bf16x2(v.x, acc[j][0]);
-            sq_acc_bf16x2(v.y, acc[j][1]);
-            sq_acc_bf16x2(v.z, acc[j][2]);
-            sq_acc_bf16x2(v.w, acc[j][3]);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-        if (++s == NS) { s = 0; ph ^= 1u; }
-      }
-      if (!ok || !prm.norms) continue;
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int64_t row = t * BM + r0 + 64 * j;
-        if (row < prm.n)
-          qjl_hint::st_f32(prm.norms + row, sqrtf((acc[j][0] + acc[j][1]) + (acc[j][2] + acc[j][3])),
-                           qjl_hint::evict_first());
-      }
     }
   }
   qjl_tc::fence_before();
@@ -415,14 +465,14 @@ void fqjl_tc_prepare(qjl_projection* P) {
 }
 
 bool fqjl_tc_supported(const qjl_projection* P, int dtype, int64_t n) {
-  // the D-FQJL dither stays with the register kernel
+  // the D-FQJL dither runs here for d = 128 only
   const bool dither = P->kind == QJL_DFQJL && P->dither_sigma != 0.f;
-  return P->kind != QJL_DENSE && !dither && P->S1_bf16 && P->s_map_ok && dtype == QJL_BF16 &&
+  return P->kind != QJL_DENSE && (!dither || P->d == 128) && P->S1_bf16 && P->s_map_ok && dtype == QJL_BF16 &&
          fqjl_tc_shape(P->d, P->m, P->opt.dg_outer != 0) && n <= (int64_t)INT32_MAX - BM;
 }
 
-qjl_status launch_fqjl_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld, uint32_t* bits,
-                          float* norms, cudaStream_t st) {
+qjl_status launch_fqjl_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld, uint64_t first_token,
+                          uint32_t* bits, float* norms, cudaStream_t st) {
   if (n <= 0) return QJL_OK;
   // the keys' map is cached per thread for the last (pointer, rows, ld, d), as in the dense sketch
   struct KeyMapCache {
@@ -448,12 +498,15 @@ qjl_status launch_fqjl_tc(const qjl_projection* P, const void* keys, int64_t n, 
   if (!err) return qjl_set_error(QJL_ERR_CUDA, "cannot resolve the kernel error flag");
   const int ns = pick_slots(P->d);
   const size_t smem = smem_bytes(P->d, ns);
-  void (*kern)(CUtensorMap, CUtensorMap, FtcParams) = P->d == 128 ? fqjl_tc_kernel<128> : fqjl_tc_kernel<256>;
+  const bool dither = P->kind == QJL_DFQJL && P->dither_sigma != 0.f;
+  void (*kern)(CUtensorMap, CUtensorMap, FtcParams) =
+      P->d == 256 ? fqjl_tc_kernel<256, false> : (dither ? fqjl_tc_kernel<128, true> : fqjl_tc_kernel<128, false>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return qjl_check_launch("fqjl_tc_kernel smem attribute");
   const int64_t ntiles = (n + BM - 1) / BM;
   const int grid = (int)std::min<int64_t>(ntiles, qjl_num_sms(P->device));
-  FtcParams prm{n, P->m / 32, 0, ns, P->D_g, bits, norms, err};
+  FtcParams prm{n, P->m / 32, 0, ns, P->D_g, P->dither_sigma, (uint32_t)P->seed, (uint32_t)(P->seed >> 32),
+                first_token, bits, norms, err};
   for (int pass = 0; pass < P->m / kPass; ++pass) {
     prm.pass = pass;
     prm.norms = pass == 0 ? norms : nullptr;

@@ -345,7 +345,7 @@ qjl_status qjl_quantize_keys(const qjl_projection* P, const void* keys, qjl_dtyp
     if (dense_tc_supported(P, dtype, keys, ld)) return launch_dense_tc(P, keys, n, ld, bits, norms, st);
     return launch_dense_simt(P, keys, dtype, n, ld, bits, norms, nullptr, st);
   }
-  if (fqjl_tc_supported(P, dtype, n)) return launch_fqjl_tc(P, keys, n, ld, bits, norms, st);
+  if (fqjl_tc_supported(P, dtype, n)) return launch_fqjl_tc(P, keys, n, ld, first_token, bits, norms, st);
   return launch_fqjl_keys(P, keys, dtype, n, ld, first_token, bits, norms, st);
 }
 

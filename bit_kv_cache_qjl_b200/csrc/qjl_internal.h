@@ -112,15 +112,15 @@ qjl_status launch_dense_tc(const qjl_projection* P, const void* keys, int64_t n,
 bool qjl_make_bf16_map(void* map, const void* ptr, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows);
 // FQJL keys with the first randomized Hadamard transform on tcgen05
 // (fqjl_tc.cu): bf16 keys, d in {128, 256}, m a multiple of 256, the default
-// order, no dither, not a paged append. When the projection is made, fqjl_tc_shape
+// order, not a paged append, and the D-FQJL dither only for d = 128. When the projection is made, fqjl_tc_shape
 // decides whether it gets S1 (fqjl_tc_matrix, uploaded to S1_bf16), and
 // fqjl_tc_prepare encodes S1's tensor map into s_map.
 bool fqjl_tc_shape(int d, int m, bool dg_outer);
 std::vector<uint16_t> fqjl_tc_matrix(int d, int m, const float* D_r, const int32_t* perm);
 void fqjl_tc_prepare(qjl_projection* P);
 bool fqjl_tc_supported(const qjl_projection* P, int dtype, int64_t n);
-qjl_status launch_fqjl_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld, uint32_t* bits,
-                          float* norms, cudaStream_t st);
+qjl_status launch_fqjl_tc(const qjl_projection* P, const void* keys, int64_t n, int64_t ld, uint64_t first_token,
+                          uint32_t* bits, float* norms, cudaStream_t st);
 qjl_status launch_fqjl_queries(const qjl_projection* P, const float* q, int64_t nq, int64_t ld,
                                float* out, cudaStream_t st);
 std::vector<float> fqjl_key_tables(int d, int m, const float* D_r, const int32_t* perm, const float* D_g);

@@ -51,9 +51,13 @@ def test_fqjl_kernels(cuda_ok):
     D0 = qjl.Projection(5, 128, 256, "dfqjl", dither_sigma_rel=0.0)
     names = _kernels(lambda: qjl.quantize_keys(D0, wl.normal((300, 128), 3, "cuda", torch.bfloat16)))
     assert sum("fqjl_tc_kernel" in n for n in names) == 1, names
-    # the dither, fp32 keys, other widths and the literal order keep the register Walsh-Hadamard kernel
     D = qjl.Projection(5, 128, 256, "dfqjl")
-    assert _has(_kernels(lambda: qjl.quantize_keys(D, wl.normal((300, 128), 3, "cuda", torch.bfloat16))),
+    names = _kernels(lambda: qjl.quantize_keys(D, wl.normal((300, 128), 3, "cuda", torch.bfloat16)))
+    assert sum("fqjl_tc_kernel" in n for n in names) == 1, names
+    # the dither at d = 256, fp32 keys, other widths and the literal order keep the register
+    # Walsh-Hadamard kernel
+    D2 = qjl.Projection(5, 256, 256, "dfqjl")
+    assert _has(_kernels(lambda: qjl.quantize_keys(D2, wl.normal((300, 256), 3, "cuda", torch.bfloat16))),
                 "fqjl_keys_kernel")
     assert _has(_kernels(lambda: qjl.quantize_keys(P, keys.float())), "fqjl_keys_kernel")
     E = qjl.Projection(4, 512, 1024, "pfqjl")
