@@ -12,9 +12,10 @@
 //   y = D_g H Pi H D_r x            (dg_outer, the literal order)
 // and the stored bit is [y + sqrt(d) sigma_rel ||x|| xi >= 0] (the positive
 // factor sqrt(d) between y and the normalised map does not move a sign).
-// The dither xi for coordinate e = b*d + i of token t comes four coordinates
-// to a Philox4x32-10 block at counter (e/4, t_lo, t_hi, 3): Box-Muller on
-// 23-bit draws, cos and sin outputs, from words (0,1) and (2,3).
+// The dither xi for coordinate e = b*d + i of token t comes eight coordinates
+// to a Philox4x32-10 block at counter (e/8, t_lo, t_hi, 3): word w gives
+// coordinates 8c + 2w and 8c + 2w + 1, the cos and sin outputs of Box-Muller
+// on its two 16-bit halves.
 //
 // Work split. A thread holds E = min(d, 128) elements of one key in registers
 // as E/2 packed pairs V[t] = (v_t, v_{t+E/2}), so most butterflies are sm_100
@@ -303,24 +304,28 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) fqjl_keys_kernel(const Keys
       if (MODE == MODE_D) {
         const float amp = a.amp_rel * norm;
         if (amp != 0.f) {
-          const uint32_t cb = (uint32_t)((b * d + s * E) >> 2);
+          const uint32_t cb = (uint32_t)((b * d + s * E) >> 3);
           const uint32_t tlo = (uint32_t)tok, thi = (uint32_t)(tok >> 32);
 #pragma unroll
-          for (int c = 0; c < E / 4; c += 4) {
+          for (int c = 0; c < E / 8; c += 4) {
             qjl::U32x4 w[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) w[j] = qjl::U32x4{cb + c + j, tlo, thi, qjl::kStreamDither};
             philox_x4(w, a.k0, a.k1);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              float xi[4];
-              box_muller23(w[j].x, w[j].y, amp, xi[0], xi[1]);
-              box_muller23(w[j].z, w[j].w, amp, xi[2], xi[3]);
+              const uint32_t x[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const int r = 4 * (c + j) + e;
-                if (r < E / 2) V[r].x += xi[e];
-                else V[r - E / 2].y += xi[e];
+                const float2 xi = box_muller16(x[e], amp);
+                const int r = 8 * (c + j) + 2 * e;
+                if (r < E / 2) {
+                  V[r].x += xi.x;
+                  V[r + 1].x += xi.y;
+                } else {
+                  V[r - E / 2].y += xi.x;
+                  V[r + 1 - E / 2].y += xi.y;
+                }
               }
             }
           }

@@ -133,26 +133,24 @@ __device__ __forceinline__ void sign_words128(const float2 (&V)[64], uint32_t (&
 
 // D-FQJL dither of coordinates e0 .. e0 + 127 of token tok, scaled by amp, added to V: the
 // register kernel's draw (fqjl_keys.cu). Coordinate e comes from the Philox4x32-10 block at
-// counter (e/4, tok_lo, tok_hi, dither stream): words (0, 1) give coordinates 4c, 4c + 1 and
-// words (2, 3) give 4c + 2, 4c + 3, by Box-Muller on 23-bit draws.
+// counter (e/8, tok_lo, tok_hi, dither stream): word w gives coordinates 8c + 2w and
+// 8c + 2w + 1, the pair V[4c + w], by Box-Muller on its two 16-bit halves.
 __device__ __forceinline__ void add_dither(float2 (&V)[64], uint32_t e0, uint64_t tok, float amp, uint32_t k0,
                                            uint32_t k1) {
-  const uint32_t cb = e0 >> 2, tlo = (uint32_t)tok, thi = (uint32_t)(tok >> 32);
+  const uint32_t cb = e0 >> 3, tlo = (uint32_t)tok, thi = (uint32_t)(tok >> 32);
 #pragma unroll
-  for (int c = 0; c < 32; c += 4) {
+  for (int c = 0; c < 16; c += 4) {
     qjl::U32x4 w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) w[j] = qjl::U32x4{cb + c + j, tlo, thi, qjl::kStreamDither};
     philox_x4(w, k0, k1);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      float xi[4];
-      box_muller23(w[j].x, w[j].y, amp, xi[0], xi[1]);
-      box_muller23(w[j].z, w[j].w, amp, xi[2], xi[3]);
-      V[2 * (c + j)].x += xi[0];
-      V[2 * (c + j)].y += xi[1];
-      V[2 * (c + j) + 1].x += xi[2];
-      V[2 * (c + j) + 1].y += xi[3];
+      const int q = 4 * (c + j);
+      add2(V[q], box_muller16(w[j].x, amp));
+      add2(V[q + 1], box_muller16(w[j].y, amp));
+      add2(V[q + 2], box_muller16(w[j].z, amp));
+      add2(V[q + 3], box_muller16(w[j].w, amp));
     }
   }
 }

@@ -81,13 +81,13 @@ __device__ __forceinline__ void sq_acc_bf16x2(uint32_t u, float& acc) {
 
 // ---- dither ------------------------------------------------------------------------------------
 
-// Box-Muller on 23-bit draws, scaled by amp: (amp r cos 2 pi v, amp r sin 2 pi v) with
-// u = ((xr >> 9) + 1/2) 2^-23 and v = (xa >> 9) 2^-23. Both draws are exact fp32 values:
-// u = (1 + k 2^-23) - (1 - 2^-24) is an exact subtraction. The angle is taken as 2 pi (1 + v),
-// which has the same sine and cosine.
-__device__ __forceinline__ void box_muller23(uint32_t xr, uint32_t xa, float amp, float& c, float& s) {
-  const float u = __uint_as_float((xr >> 9) | 0x3f800000u) - __uint_as_float(0x3f7fffffu);
-  const float f = __uint_as_float((xa >> 9) | 0x3f800000u);
+// Box-Muller on the two 16-bit halves of x, scaled by amp: (amp r cos 2 pi v, amp r sin 2 pi v)
+// with u = ((x & 0xFFFF) + 1/2) 2^-16 from the low half and v = (x >> 16) 2^-16 from the high
+// half. Both draws are exact fp32 values: u = (1 + k 2^-16) - (1 - 2^-17) is an exact
+// subtraction. The angle is taken as 2 pi (1 + v), which has the same sine and cosine.
+__device__ __forceinline__ float2 box_muller16(uint32_t x, float amp) {
+  const float u = __uint_as_float(((x & 0xFFFFu) << 7) | 0x3f800000u) - __uint_as_float(0x3f7fff80u);
+  const float f = __uint_as_float(((x >> 16) << 7) | 0x3f800000u);
   float l, rs, sn, cs;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(u));
   const float t = -1.38629436f * l;  // -2 ln u > 0
@@ -96,16 +96,26 @@ __device__ __forceinline__ void box_muller23(uint32_t xr, uint32_t xa, float amp
   const float th = 6.28318548f * f;
   asm("sin.approx.ftz.f32 %0, %1;" : "=f"(sn) : "f"(th));
   asm("cos.approx.ftz.f32 %0, %1;" : "=f"(cs) : "f"(th));
-  c = r * cs;
-  s = r * sn;
+  return make_float2(r * cs, r * sn);
 }
 
-// Philox4x32-10 on four counters at once, rounds interleaved for instruction-level parallelism.
-__device__ __forceinline__ void philox_x4(qjl::U32x4 (&c)[4], uint32_t k0, uint32_t k1) {
+// a <- a + b pairwise
+__device__ __forceinline__ void add2(float2& a, float2 b) {
+  asm("{\n\t.reg .b64 x, y;\n\t"
+      "mov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "add.rn.f32x2 x, x, y;\n\t"
+      "mov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a.x), "+f"(a.y)
+      : "f"(b.x), "f"(b.y));
+}
+
+// Philox4x32-10 on N counters at once, rounds interleaved for instruction-level parallelism.
+template <int N>
+__device__ __forceinline__ void philox_xn(qjl::U32x4 (&c)[N], uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < N; ++j) {
       uint32_t hA, lA, hB, lB;
       qjl::mul_hi_lo(0xD2511F53u, c[j].x, hA, lA);
       qjl::mul_hi_lo(0xCD9E8D57u, c[j].z, hB, lB);
@@ -115,5 +125,7 @@ __device__ __forceinline__ void philox_x4(qjl::U32x4 (&c)[4], uint32_t k0, uint3
     k1 += 0xBB67AE85u;
   }
 }
+
+__device__ __forceinline__ void philox_x4(qjl::U32x4 (&c)[4], uint32_t k0, uint32_t k1) { philox_xn<4>(c, k0, k1); }
 
 }  // namespace qjl_km

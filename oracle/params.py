@@ -97,23 +97,26 @@ def fisher_yates(seed, d, nblocks):
 def dither(seed, d, m, tokens):
     """D-FQJL dither xi[t][e] ~ N(0,1) for coordinate e = b*d + i of token t.
 
-    The pages ask for Gaussian dither and fix no generator for it. Here one
-    Philox block gives four coordinates. The block at counter
-    (e // 4, t_lo, t_hi, STREAM_DITHER) returns the words x0..x3. Box-Muller
-    (``philox.box_muller_pair23``) turns (x0, x1) into xi[4c], xi[4c+1] and
-    (x2, x3) into xi[4c+2], xi[4c+3].
+    The pages ask for Gaussian dither ("Key concepts": non-subtractive Gaussian
+    dithering) and fix no generator for it. Here one Philox block gives eight
+    coordinates. The block at counter (e // 8, t_lo, t_hi, STREAM_DITHER)
+    returns the words x0..x3, and word w gives coordinates 8c + 2w and
+    8c + 2w + 1 as the cos and sin outputs of Box-Muller on its two 16-bit
+    halves (``philox.box_muller_pair16``).
 
     ``tokens`` are absolute token indices (first_token + row), so an appended
     key gets the same dither whatever batch it was quantised in.
     """
     tokens = np.asarray(tokens, dtype=np.uint64).reshape(-1, 1)
-    c = np.arange(m // 4, dtype=np.uint64).reshape(1, -1)
+    c = np.arange(m // 8, dtype=np.uint64).reshape(1, -1)
     k0, k1 = ph.seed_key(seed)
-    x0, x1, x2, x3 = ph.philox4x32_10(c, tokens & np.uint64(ph.MASK32), tokens >> np.uint64(32),
-                                      ph.STREAM_DITHER, k0, k1)
-    a0, a1 = ph.box_muller_pair23(x0, x1)
-    b0, b1 = ph.box_muller_pair23(x2, x3)
-    xi = np.stack([a0, a1, b0, b1], axis=-1)      # [t][c][j], coordinate 4c + j
+    words = ph.philox4x32_10(c, tokens & np.uint64(ph.MASK32), tokens >> np.uint64(32),
+                             ph.STREAM_DITHER, k0, k1)
+    outs = []
+    for x in words:
+        a, b = ph.box_muller_pair16(x)
+        outs += [a, b]
+    xi = np.stack(outs, axis=-1)                  # [t][c][2w + j], coordinate 8c + 2w + j
     return xi.reshape(tokens.shape[0], m)  # fp64; the library evaluates the same formula in fp32
 
 

@@ -35,7 +35,7 @@ MASK32 = 0xFFFFFFFF
 STREAM_GAUSS = 0       # dense S entries, Gaussian diagonal D_g
 STREAM_RADEMACHER = 1  # Rademacher diagonal D_r
 STREAM_PERM = 2        # Fisher-Yates draws for the permutation Pi
-STREAM_DITHER = 3      # D-FQJL dither, one block per (token, 4 coordinates)
+STREAM_DITHER = 3      # D-FQJL dither, one block per (token, 8 coordinates)
 
 
 def _u32(x):
@@ -82,17 +82,18 @@ def box_muller(x0, x1):
     return np.sqrt(-2.0 * np.log(u0)) * np.cos(2.0 * np.pi * u1)
 
 
-def box_muller_pair23(xr, xa):
-    """Two independent standard normals from two words, on 23-bit draws (fp64).
+def box_muller_pair16(x):
+    """Two independent standard normals from the two 16-bit halves of a word (fp64).
 
-    The radius draw is u = ((xr >> 9) + 1/2) / 2^23, in (0, 1). The angle draw
-    is v = (xa >> 9) / 2^23, in [0, 1). The pair is sqrt(-2 ln u) times
-    (cos 2 pi v, sin 2 pi v). These are the two outputs of Box and Muller,
-    "A Note on the Generation of Random Normal Deviates" (1958), and they are
-    independent N(0, 1).
+    The radius draw is u = ((x & 0xFFFF) + 1/2) / 2^16, in (0, 1), from the low
+    half. The angle draw is v = (x >> 16) / 2^16, in [0, 1), from the high half.
+    The pair is sqrt(-2 ln u) times (cos 2 pi v, sin 2 pi v): the two outputs of
+    Box and Muller, "A Note on the Generation of Random Normal Deviates" (1958),
+    which are independent N(0, 1). The radius is at most sqrt(-2 ln 2^-17) = 4.85.
     """
-    u = (np.asarray(xr, dtype=np.uint64) >> np.uint64(9)).astype(np.float64) * 2.0 ** -23 + 2.0 ** -24
-    v = (np.asarray(xa, dtype=np.uint64) >> np.uint64(9)).astype(np.float64) * 2.0 ** -23
+    x = np.asarray(x, dtype=np.uint64)
+    u = (x & np.uint64(0xFFFF)).astype(np.float64) * 2.0 ** -16 + 2.0 ** -17
+    v = (x >> np.uint64(16)).astype(np.float64) * 2.0 ** -16
     r = np.sqrt(-2.0 * np.log(u))
     return r * np.cos(2.0 * np.pi * v), r * np.sin(2.0 * np.pi * v)
 

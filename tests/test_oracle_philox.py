@@ -138,11 +138,14 @@ def test_dither_depends_on_absolute_token():
 
 def test_dither_is_standard_normal_per_coordinate():
     xi = P.dither(21, 64, 128, np.arange(4000))
-    for j in range(4):     # each of the four coordinates one block yields
-        col = xi[:, j::4].ravel()
+    for j in range(8):     # each of the eight coordinates one block yields
+        col = xi[:, j::8].ravel()
         assert scipy.stats.kstest(col, "norm").pvalue > 1e-4
     # variance 1 to within the sampling error of 512000 draws
     assert abs(xi.var() - 1.0) < 0.01
+    # the fourth moment of N(0, 1) is 3 (the 4.85-sigma cut of the 16-bit radius draw removes
+    # a 1.3e-6 tail, far below the sampling error here)
+    assert abs((xi ** 4).mean() - 3.0) < 0.05
 
 
 def test_dither_pairs_are_independent_normals():
@@ -150,25 +153,44 @@ def test_dither_pairs_are_independent_normals():
     chi-square with 2 degrees of freedom, and any rotation of the pair is
     again standard normal. Pairs from different words of one block do not
     correlate."""
-    xi = P.dither(22, 32, 64, np.arange(5000)).reshape(-1, 4)
-    for a, b in ((0, 1), (2, 3)):
+    xi = P.dither(22, 32, 64, np.arange(5000)).reshape(-1, 8)
+    for a in range(0, 8, 2):
+        b = a + 1
         r2 = xi[:, a] ** 2 + xi[:, b] ** 2
         assert scipy.stats.kstest(r2, "chi2", args=(2,)).pvalue > 1e-4
         rot = (xi[:, a] + xi[:, b]) / math.sqrt(2.0)
         assert scipy.stats.kstest(rot, "norm").pvalue > 1e-4
     c = np.corrcoef(xi.T)
-    assert np.max(np.abs(c - np.eye(4))) < 0.02
+    assert np.max(np.abs(c - np.eye(8))) < 0.02
 
 
 def test_dither_prefix_and_block_structure():
-    """Coordinates come in fours from one block: the dither of the first m'
+    """Coordinates come in eights from one block: the dither of the first m'
     coordinates does not depend on m, and neither on d."""
     a = P.dither(23, 32, 64, [5, 6])
     b = P.dither(23, 64, 256, [5, 6])
     assert np.array_equal(a, b[:, :64])
     assert np.all(np.isfinite(b))
-    # the radius draw is never 0 or 1: |xi| is bounded by sqrt(-2 ln 2^-24)
-    assert np.max(np.abs(P.dither(24, 128, 1024, np.arange(500)))) < math.sqrt(2 * 24 * math.log(2)) + 1e-9
+    # the radius draw is never 0 or 1: |xi| is bounded by sqrt(-2 ln 2^-17)
+    assert np.max(np.abs(P.dither(24, 128, 1024, np.arange(500)))) < math.sqrt(2 * 17 * math.log(2)) + 1e-9
+
+
+def test_dither_word_brute_force():
+    """Coordinates 8c + 2w and 8c + 2w + 1 of a token, written out from the block's word w:
+    u from its low 16 bits, v from its high 16 bits, Box-Muller's cos and sin outputs."""
+    seed, t = 0x1234_5678_9ABC_DEF0, (1 << 32) + 77
+    xi = P.dither(seed, 32, 64, [t])[0]
+    k0, k1 = seed & 0xFFFFFFFF, seed >> 32
+    for c in range(8):
+        words = ph.philox4x32_10(np.uint64(c), np.uint64(t & 0xFFFFFFFF), np.uint64(t >> 32),
+                                 ph.STREAM_DITHER, np.uint64(k0), np.uint64(k1))
+        for w in range(4):
+            x = int(words[w])
+            u = ((x & 0xFFFF) + 0.5) / 65536.0
+            v = (x >> 16) / 65536.0
+            r = math.sqrt(-2.0 * math.log(u))
+            assert abs(xi[8 * c + 2 * w] - r * math.cos(2 * math.pi * v)) < 1e-12
+            assert abs(xi[8 * c + 2 * w + 1] - r * math.sin(2 * math.pi * v)) < 1e-12
 
 
 @pytest.mark.parametrize("ctr,key,want", [
