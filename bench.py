@@ -551,8 +551,11 @@ def build_workload(name, dev, qjl, wl, torch):
         ws = torch.empty((qjl.decode_workspace_bytes(G, 1, Nd, D),), dtype=torch.uint8, device=dev)
         smx = 1.0 / math.sqrt(D)
         stages = [
+            # the first Hadamard factor on tcgen05, the second and the dither on the lanes: reported
+            # against the FP32 lane ceiling with the second factor's fp32 operations only (the
+            # dither's Philox multiplies and Box-Muller are not fp32 adds or multiplies)
             Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), G * Nd,
-                  2 * D + m // 8 + 4, fqjl_flops_per_key(D, m), "fqjl_keys_kernel", "fqjl_keys.cu", "alu"),
+                  2 * D + m // 8 + 4, (m // D) * (D + D * int(math.log2(D))), "fqjl_tc_kernel", "fqjl_tc.cu", "alu"),
             Stage("quantize_values", lambda: qjl.quantize_values_2bit(vals, codes=codes, scale=sc, zero=zr), G * Nd,
                   2 * D + D // 4 + D // 8, 0, "values_2bit_kernel", "values.cu"),
             Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * m, bound="launch"),
