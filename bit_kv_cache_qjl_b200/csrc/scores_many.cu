@@ -184,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
   constexpr int KC = kc_words(W);         // sign words per A buffer
   constexpr int NCH = W / KC;             // A buffers per tile
   constexpr int NA = n_abuf(W);
+  constexpr int ND = 2;  // D buffers
   constexpr int JH = JP / (kEpiWarps / 4);  // queries per epilogue warp (even)
   static_assert(JH % 2 == 0, "query pairs");
   constexpr uint32_t TAB = (uint32_t)NCOL * 32 * W;
@@ -199,9 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
   uint64_t* empty = full + P.NS;
   uint64_t* afull = empty + P.NS;    // [NA]
   uint64_t* aempty = afull + NA;     // [NA]
-  uint64_t* dfull = aempty + NA;     // [2]
-  uint64_t* dempty = dfull + 2;      // [2]
-  uint64_t* tfull = dempty + 2;      // [2]
+  uint64_t* dfull = aempty + NA;     // [ND]
+  uint64_t* dempty = dfull + ND;     // [ND]
+  uint64_t* tfull = dempty + ND;     // [2]
   uint64_t* dbar = tfull + 2;        // [1]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(dbar + 1);
 
@@ -222,11 +223,11 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
       mbar_init(&afull[a], kExpWarps);
       mbar_init(&aempty[a], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < ND; ++b) {
       mbar_init(&dfull[b], 1);
       mbar_init(&dempty[b], kEpiWarps);
-      mbar_init(&tfull[b], 1);
     }
+    for (int b = 0; b < 2; ++b) mbar_init(&tfull[b], 1);
     mbar_init(dbar, 1);
     mbar_fence_init();
   }
@@ -294,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
         }
         if (!ok) break;
         qjl_tc::commit(&dfull[db]);
-        if (++db == 2) { db = 0; dpar ^= 1u; }
+        if (++db == ND) { db = 0; dpar ^= 1u; }
         if (++c == tpg) { c = 0; ++g; }
       }
       // every MMA issued has completed before TMEM is freed
@@ -372,6 +373,14 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
     int gi = 0, tb = 0, db = 0;
     uint32_t dpar = 0;
     bool dead = false;  // a timed-out wait: keep the builds' barriers, skip the work
+    // A tile's norms come from HBM, and the epilogue is the stage that releases the D buffers,
+    // so they are fetched one tile ahead: the load for tile it + 1 is issued while tile it's
+    // accumulator is awaited and stored.
+    auto norm_of = [&](int64_t gg, int64_t cc) {
+      const int64_t nn = cc * kTile + r;
+      return nn < N ? __ldg(P.norms + gg * N + nn) : 0.f;
+    };
+    float nrm_next = i0 < i1 ? norm_of(g, c) : 0.f;
     for (int64_t it = i0; it < i1; ++it) {
       if (g != cur_g) {
         cur_g = g;
@@ -380,8 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
       }
       const int64_t n0 = c * kTile;
       const int cnt = (int)(N - n0 < kTile ? N - n0 : kTile);
-      // the tile's norm is fetched before the wait for its accumulator
-      const float nrm = r < cnt ? __ldg(P.norms + g * N + n0 + r) : 0.f;
+      const float nrm = nrm_next;
+      if (it + 1 < i1) nrm_next = c + 1 == tpg ? norm_of(g + 1, 0) : norm_of(g, c + 1);
       if (!dead && !__all_sync(0xffffffffu, mbar_wait(&dfull[db], dpar))) { atomicOr(P.err, 16); dead = true; }
       if (!dead) {
         qjl_tc::fence_after();
@@ -415,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
           }
         }
       }
-      if (++db == 2) { db = 0; dpar ^= 1u; }
+      if (++db == ND) { db = 0; dpar ^= 1u; }
       // after the last tile of this group in the range, the MMAs that read its table are
       // complete: the buffer takes the table of the group ntab places further on
       const bool last = (c + 1 == tpg) || (it + 1 == i1);
