@@ -93,6 +93,15 @@ def test_dense_bf16_keys_fp32_matrix_simt(cuda_ok):
     # more blocks than one launch's table budget: several launches over block ranges
     ("pfqjl", 1024, 4096, 37, torch.bfloat16, 0),
     ("dfqjl", 128, 4096, 70, torch.float32, 11),
+    # the tcgen05 kernel (bf16, d in {128, 256}, m a multiple of 256): one key; the dither past
+    # 2^32 tokens; several 256-coordinate passes (the dither's coordinate offset per pass)
+    ("pfqjl", 256, 256, 1, torch.bfloat16, 0),
+    ("dfqjl", 128, 256, 129, torch.bfloat16, (1 << 32) + 7),
+    ("dfqjl", 128, 512, 300, torch.bfloat16, 5),
+    ("pfqjl", 128, 768, 200, torch.bfloat16, 0),
+    # every CTA of the persistent grid takes two tiles or more (ring and TMEM phases wrap)
+    ("dfqjl", 128, 256, 148 * 128 * 2 + 77, torch.bfloat16, 1),
+    ("pfqjl", 256, 256, 148 * 128 * 2 + 5, torch.bfloat16, 0),
 ])
 def test_fqjl(cuda_ok, kind, d, m, n, dtype, ft):
     P = Projection(4, d, m, kind)
