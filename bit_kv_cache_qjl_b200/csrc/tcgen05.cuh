@@ -95,7 +95,7 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uin
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
-// 2-D tiled TMA load (no multicast) of the box at (x, y), completion counted on `bar`.
+// 2-D tiled TMA load of the box at (x, y) into this CTA's shared memory, completion counted on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, uint64_t* bar, int x, int y) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
