@@ -91,7 +91,10 @@ typedef struct qjl_projection qjl_projection;
  * Generator: Philox4x32-10 (Salmon et al., SC'11) with key = seed and
  * counter = (index_lo, index_hi, block, stream). The streams are 0 Gaussian
  * (S, D_g), 1 Rademacher (D_r), 2 permutation (Fisher-Yates) and 3 dither.
- * Gaussians use Box-Muller in fp64 and are rounded to fp32.
+ * Gaussians use Box-Muller in fp64 and are rounded to fp32. The D-FQJL dither
+ * of coordinate e of token t takes the block at counter (e/8, t_lo, t_hi, 3):
+ * word w gives coordinates 8(e/8) + 2w and + 1 by Box-Muller on its two
+ * 16-bit halves.
  *   d     head dimension, 1..4096. FQJL: a power of two, 32..1024.
  *   m     sketch size, a multiple of 32, 32..16384. FQJL: a multiple of d.
  *   opt   NULL for the defaults.
@@ -130,7 +133,10 @@ qjl_status qjl_projection_export(const qjl_projection* proj, qjl_export_what wha
  *   bits        out [n][m/32] uint32, 16-byte aligned.
  *   norms       out [n] fp32: ||k||_2.
  * Dense with bf16 keys and bf16 S_eff runs the tcgen05/TMA kernel. Every
- * other dense case runs an fp32 SIMT kernel. FQJL runs the fast
+ * other dense case runs an fp32 SIMT kernel. FQJL with bf16 keys, d in
+ * {128, 256}, m a multiple of 256 and the default order (D-FQJL: d = 128)
+ * runs its first Hadamard factor as an exact +-1 contraction on tcgen05 and
+ * the rest on the FP32 lanes; every other FQJL case runs the register
  * Walsh-Hadamard kernel.
  */
 qjl_status qjl_quantize_keys(const qjl_projection* proj, const void* keys, qjl_dtype dtype,
