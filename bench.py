@@ -524,7 +524,7 @@ def build_workload(name, dev, qjl, wl, torch):
             # the first Hadamard factor runs as an exact +-1 contraction on tcgen05 (2 d m flops per
             # key), the second (D_g and d log2 d additions per block) on the FP32 lanes
             Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), n,
-                  2 * d + m // 8 + 4, 2 * d * m, "fqjl_tc_kernel", "fqjl_tc.cu", "tensor", launches=m // 256,
+                  2 * d + m // 8 + 4, 2 * d * m, "fqjl_tc_kernel", "fqjl_tc.cu", "tensor",
                   alu_ops_per_unit=(m // d) * (d + d * int(math.log2(d)))),
             Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), J, 4 * d + 4 * m, bound="launch"),
             Stage("scores", lambda: qjl.scores(P, bits[:ns].view(1, ns, m // 32), norms[:ns].view(1, ns),

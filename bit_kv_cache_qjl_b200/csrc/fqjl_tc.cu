@@ -31,7 +31,9 @@
 //              output half of d = 256).
 //   warps 10-11 ||x|| from the swizzled key slots (as in the dense sketch).
 // A pass covers 256 output coordinates (one block of d = 256 or two of
-// d = 128). The host runs m/256 passes; each reads the keys again.
+// d = 128). For m > 256 one launch runs m/256 groups of CTAs, one per pass,
+// that walk the same tiles in step: each key tile comes from HBM once and is
+// an L2 hit for the other passes.
 //
 // No output bit comes from a -0. D_g is applied as fma(g, u, +0), or for the
 // fused top butterfly as fma(g, a, fma(+-g', b, +0)), so an exact zero is
@@ -83,14 +85,15 @@ constexpr size_t kSmemLimit = 227 * 1024;
 struct FtcParams {
   int64_t n;
   int W;                 // sign words per key row
-  int pass;              // output coordinates 256 pass .. 256 pass + 255
+  int npass;             // m / 256: CTA c takes pass c % npass (coordinates 256 pass ..
+                         // 256 pass + 255) and every (gridDim / npass)-th tile from c / npass
   int ns;                // ring slots
   const float* D_g;      // [m], all blocks
   float sigma;           // D-FQJL dither sigma_rel (the dithered instantiation)
   uint32_t k0, k1;       // the seed as the Philox key
   uint64_t first_token;  // token index of row 0 (the dither's counter)
   uint32_t* bits;
-  float* norms;          // the first pass only, else nullptr
+  float* norms;          // written by the CTAs of pass 0
   int* err;
 };
 
@@ -190,12 +193,16 @@ __global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_const
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ntiles = (prm.n + BM - 1) / BM;
+  // the npass CTAs of a group walk the same tiles in step, so a key tile read from HBM by one
+  // of them is an L2 hit for the others
+  const int pass = (int)(blockIdx.x % (unsigned)prm.npass);
+  const int cta0 = (int)(blockIdx.x / (unsigned)prm.npass), ncta = (int)(gridDim.x / (unsigned)prm.npass);
 
   // D_g of this pass's coordinates. Row h scales the upper 128 by (+1, -1)[h]: the fused
   // top butterfly of d = 256 reads row h for output half h. d = 128 reads row 0 only.
   for (int i = threadIdx.x; i < 2 * kPass; i += blockDim.x) {
     const int h = i / kPass, c = i % kPass;
-    const float g = __ldg(prm.D_g + (size_t)kPass * prm.pass + c);
+    const float g = __ldg(prm.D_g + (size_t)kPass * pass + c);
     sG[i] = (h == 1 && c >= 128) ? -g : g;
   }
   if (threadIdx.x == 0) {
@@ -223,12 +230,12 @@ __global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_const
     if (warp == 0) {
       if (lane == 0) {
         mbar_expect_tx(sbar, (uint32_t)(KA * kPass * 128));
-        for (int a = 0; a < KA; ++a) qjl_tc::tma_load_2d(sS + (size_t)a * kPass * 128, &tmS, sbar, a * 64, kPass * prm.pass);
+        for (int a = 0; a < KA; ++a) qjl_tc::tma_load_2d(sS + (size_t)a * kPass * 128, &tmS, sbar, a * 64, kPass * pass);
         int64_t issued = 0;
         int s = 0;
         uint32_t ph = 0;
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        for (int64_t t = cta0; t < ntiles && ok; t += ncta) {
           for (int a = 0; a < KA; ++a, ++issued) {
             if (!mbar_wait(&empty[s], ph ^ 1u)) { flag_error(prm.err, 1); ok = false; break; }
             mbar_expect_tx(&full[s], kSlotBytes);
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_const
         uint32_t u = 0;
         int s = 0;
         uint32_t ph = 0;
-        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++u) {
+        for (int64_t t = cta0; t < ntiles && ok; t += ncta, ++u) {
           const int buf = (int)(u & 1u);
           if (!mbar_wait(&tempty[buf], ((u >> 1) & 1u) ^ 1u)) { flag_error(prm.err, 4); break; }
           qjl_tc::fence_after();
@@ -287,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_const
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      for (int64_t t = cta0; t < ntiles && ok; t += ncta) {
         float acc[2][4];
 #pragma unroll
         for (int j = 0; j < 2; ++j)
@@ -312,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_const
           if (lane == 0) mbar_arrive(&empty[s]);
           if (++s == NS) { s = 0; ph ^= 1u; }
         }
-        if (!ok || !prm.norms) continue;
+        if (!ok || pass != 0) continue;
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const int64_t row = t * BM + r0 + 64 * j;
@@ -330,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_const
     const uint32_t lane_base = tmem_base + ((uint32_t)(quarter * 32) << 16);
     const uint64_t pol = qjl_hint::evict_first();
     uint32_t u = 0;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++u) {
+    for (int64_t t = cta0; t < ntiles; t += ncta, ++u) {
       const int buf = (int)(u & 1u);
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (u >> 1) & 1u))) { flag_error(prm.err, 16); break; }
       qjl_tc::fence_after();
@@ -412,11 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1) fqjl_tc_kernel(const __grid_const
       }
       fwht128(V);
       if (DITHER && amp != 0.f)
-        add_dither(V, (uint32_t)(kPass * prm.pass + 128 * part), prm.first_token + (uint64_t)row, amp, prm.k0,
+        add_dither(V, (uint32_t)(kPass * pass + 128 * part), prm.first_token + (uint64_t)row, amp, prm.k0,
                    prm.k1);
       uint32_t w[4];
       sign_words128(V, w);
-      if (row < prm.n) qjl_hint::st_v4(prm.bits + row * (int64_t)prm.W + 8 * prm.pass + 4 * part, w[0], w[1], w[2], w[3], pol);
+      if (row < prm.n) qjl_hint::st_v4(prm.bits + row * (int64_t)prm.W + 8 * pass + 4 * part, w[0], w[1], w[2], w[3], pol);
     }
   }
   qjl_tc::fence_before();
@@ -501,17 +508,14 @@ qjl_status launch_fqjl_tc(const qjl_projection* P, const void* keys, int64_t n, 
       P->d == 256 ? fqjl_tc_kernel<256, false> : (dither ? fqjl_tc_kernel<128, true> : fqjl_tc_kernel<128, false>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return qjl_check_launch("fqjl_tc_kernel smem attribute");
+  // one launch: npass groups of CTAs, one per 256 coordinates, each walking all tiles
+  const int npass = P->m / kPass;
   const int64_t ntiles = (n + BM - 1) / BM;
-  const int grid = (int)std::min<int64_t>(ntiles, qjl_num_sms(P->device));
-  FtcParams prm{n, P->m / 32, 0, ns, P->D_g, P->dither_sigma, (uint32_t)P->seed, (uint32_t)(P->seed >> 32),
+  const int64_t per = std::min<int64_t>(ntiles, std::max(1, qjl_num_sms(P->device) / npass));
+  const int grid = (int)(per * npass);
+  FtcParams prm{n, P->m / 32, npass, ns, P->D_g, P->dither_sigma, (uint32_t)P->seed, (uint32_t)(P->seed >> 32),
                 first_token, bits, norms, err};
-  for (int pass = 0; pass < P->m / kPass; ++pass) {
-    prm.pass = pass;
-    prm.norms = pass == 0 ? norms : nullptr;
-    qjl_log_launch("fqjl_tc_kernel", grid, kThreads, smem, 1);
-    kern<<<grid, kThreads, smem, st>>>(tmK, tmS, prm);
-    const qjl_status s = qjl_check_launch("fqjl_tc_kernel");
-    if (s != QJL_OK) return s;
-  }
-  return QJL_OK;
+  qjl_log_launch("fqjl_tc_kernel", grid, kThreads, smem, 1);
+  kern<<<grid, kThreads, smem, st>>>(tmK, tmS, prm);
+  return qjl_check_launch("fqjl_tc_kernel");
 }

@@ -42,11 +42,12 @@ def test_fp32_keys_use_simt_kernel(cuda_ok):
 
 
 def test_fqjl_kernels(cuda_ok):
-    # bf16 keys with d in {128, 256} and m a multiple of 256: the tcgen05 kernel, one launch per 256 coordinates
+    # bf16 keys with d in {128, 256} and m a multiple of 256: the tcgen05 kernel, one launch for all
+    # 256-coordinate passes
     P = qjl.Projection(4, 256, 1024, "pfqjl")
     keys = wl.normal((512, 256), 1, "cuda", torch.bfloat16)
     names = _kernels(lambda: qjl.quantize_keys(P, keys))
-    assert sum("fqjl_tc_kernel" in n for n in names) == 4, names
+    assert sum("fqjl_tc_kernel" in n for n in names) == 1, names
     assert not _has(names, "fqjl_keys_kernel")
     D0 = qjl.Projection(5, 128, 256, "dfqjl", dither_sigma_rel=0.0)
     names = _kernels(lambda: qjl.quantize_keys(D0, wl.normal((300, 128), 3, "cuda", torch.bfloat16)))
