@@ -50,6 +50,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "cache_hint.cuh"
 #include "mbarrier.cuh"
@@ -406,22 +407,29 @@ __global__ void __launch_bounds__(kThreads, 1) scores_many_kernel(const __grid_c
           const int64_t n = n0 + r;
           float* out = P.scores + (g * J + hq * JH) * N + n;
           const float2* cst = s_cst + 64 * tb + hq * JH;
+          // ALL: every query of this warp's share exists, so the stores need no per-query branch
+          // (each guarded store of the other form is a branch around the store instruction)
+          auto write = [&](auto all_c) {
+            constexpr bool ALL = decltype(all_c)::value;
 #pragma unroll
-          for (int jj = 0; jj < JH; jj += 2) {
-            // sum b Q = 256 D_hi + D_lo, exact in int32 (|.| <= m * 32639 < 2^31); two queries at once
-            const float4 cc = *reinterpret_cast<const float4*>(cst + jj);  // (c1, c0) of queries jj, jj + 1
-            const float d0 = (float)((int)hi[jj] * 256 + (int)lo[jj]);
-            const float d1 = (float)((int)hi[jj + 1] * 256 + (int)lo[jj + 1]);
-            float e0, e1;
-            asm("{\n\t.reg .b64 a, b, c;\n\t"
-                "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
-                "fma.rn.f32x2 a, a, b, c;\n\tmov.b64 b, {%8, %8};\n\tmul.rn.f32x2 a, a, b;\n\t"
-                "mov.b64 {%0, %1}, a;\n\t}"
-                : "=f"(e0), "=f"(e1)
-                : "f"(cc.x), "f"(cc.z), "f"(d0), "f"(d1), "f"(cc.y), "f"(cc.w), "f"(nrm));
-            if (hq * JH + jj < J) qjl_hint::st_f32(out + (int64_t)jj * N, e0, pol);
-            if (hq * JH + jj + 1 < J) qjl_hint::st_f32(out + (int64_t)(jj + 1) * N, e1, pol);
-          }
+            for (int jj = 0; jj < JH; jj += 2) {
+              // sum b Q = 256 D_hi + D_lo, exact in int32 (|.| <= m * 32639 < 2^31); two queries at once
+              const float4 cc = *reinterpret_cast<const float4*>(cst + jj);  // (c1, c0) of queries jj, jj + 1
+              const float d0 = (float)((int)hi[jj] * 256 + (int)lo[jj]);
+              const float d1 = (float)((int)hi[jj + 1] * 256 + (int)lo[jj + 1]);
+              float e0, e1;
+              asm("{\n\t.reg .b64 a, b, c;\n\t"
+                  "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+                  "fma.rn.f32x2 a, a, b, c;\n\tmov.b64 b, {%8, %8};\n\tmul.rn.f32x2 a, a, b;\n\t"
+                  "mov.b64 {%0, %1}, a;\n\t}"
+                  : "=f"(e0), "=f"(e1)
+                  : "f"(cc.x), "f"(cc.z), "f"(d0), "f"(d1), "f"(cc.y), "f"(cc.w), "f"(nrm));
+              if (ALL || hq * JH + jj < J) qjl_hint::st_f32(out + (int64_t)jj * N, e0, pol);
+              if (ALL || hq * JH + jj + 1 < J) qjl_hint::st_f32(out + (int64_t)(jj + 1) * N, e1, pol);
+            }
+          };
+          if (hq * JH + JH <= J) write(std::true_type());
+          else write(std::false_type());
         }
       }
       if (++db == ND) { db = 0; dpar ^= 1u; }
