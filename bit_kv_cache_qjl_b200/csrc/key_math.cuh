@@ -82,21 +82,46 @@ __device__ __forceinline__ void sq_acc_bf16x2(uint32_t u, float& acc) {
 // ---- dither ------------------------------------------------------------------------------------
 
 // Box-Muller on the two 16-bit halves of x, scaled by amp: (amp r cos 2 pi v, amp r sin 2 pi v)
-// with u = ((x & 0xFFFF) + 1/2) 2^-16 from the low half and v = (x >> 16) 2^-16 from the high
-// half. Both draws are exact fp32 values: u = (1 + k 2^-16) - (1 - 2^-17) is an exact
-// subtraction. The angle is taken as 2 pi (1 + v), which has the same sine and cosine.
+// with r = sqrt(-2 ln u), u = ((x & 0xFFFF) + 1/2) 2^-16 from the low half and v = (x >> 16) 2^-16
+// from the high half. A byte permute puts a half under the exponent of 1.0, h = 1 + k 2^-23,
+// and one FMA rescales it exactly: u = 128 h - (128 - 2^-17) = (2k + 1) 2^-17 (the constant has
+// 24 significant bits, the product and the sum are exact), and the angle 256 pi (h - 1) =
+// 2 pi k 2^-16 carries one rounding of 256 pi and one of the product.
 __device__ __forceinline__ float2 box_muller16(uint32_t x, float amp) {
-  const float u = __uint_as_float(((x & 0xFFFFu) << 7) | 0x3f800000u) - __uint_as_float(0x3f7fff80u);
-  const float f = __uint_as_float(((x >> 16) << 7) | 0x3f800000u);
-  float l, rs, sn, cs;
+  const float hu = __uint_as_float(__byte_perm(x, 0x3f800000u, 0x7610));  // 1 + (x & 0xFFFF) 2^-23
+  const float hv = __uint_as_float(__byte_perm(x, 0x3f800000u, 0x7632));  // 1 + (x >> 16) 2^-23
+  const float u = fmaf(hu, 128.f, -127.99999237060546875f);
+  const float th = fmaf(hv, 804.247741699f, -804.247741699f);
+  float l, rt, sn, cs;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(u));
   const float t = -1.38629436f * l;  // -2 ln u > 0
-  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(rs) : "f"(t));
-  const float r = t * rs * amp;
-  const float th = 6.28318548f * f;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(rt) : "f"(t));
+  const float r = rt * amp;
   asm("sin.approx.ftz.f32 %0, %1;" : "=f"(sn) : "f"(th));
   asm("cos.approx.ftz.f32 %0, %1;" : "=f"(cs) : "f"(th));
   return make_float2(r * cs, r * sn);
+}
+
+// acc <- acc + dither: the Box-Muller pair of x (box_muller16) scaled by amp, with the radius
+// multiplying both outputs in one packed FMA
+__device__ __forceinline__ void add_box_muller16(float2& acc, uint32_t x, float amp) {
+  const float hu = __uint_as_float(__byte_perm(x, 0x3f800000u, 0x7610));
+  const float hv = __uint_as_float(__byte_perm(x, 0x3f800000u, 0x7632));
+  const float u = fmaf(hu, 128.f, -127.99999237060546875f);
+  const float th = fmaf(hv, 804.247741699f, -804.247741699f);
+  float l, rt, sn, cs;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(u));
+  const float t = -1.38629436f * l;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(rt) : "f"(t));
+  const float r = rt * amp;
+  asm("sin.approx.ftz.f32 %0, %1;" : "=f"(sn) : "f"(th));
+  asm("cos.approx.ftz.f32 %0, %1;" : "=f"(cs) : "f"(th));
+  asm("{\n\t.reg .b64 a, rr, cs;\n\t"
+      "mov.b64 a, {%0, %1};\n\tmov.b64 rr, {%2, %2};\n\tmov.b64 cs, {%3, %4};\n\t"
+      "fma.rn.f32x2 a, rr, cs, a;\n\t"
+      "mov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(acc.x), "+f"(acc.y)
+      : "f"(r), "f"(cs), "f"(sn));
 }
 
 // a <- a + b pairwise
@@ -123,6 +148,30 @@ __device__ __forceinline__ void philox_xn(qjl::U32x4 (&c)[N], uint32_t k0, uint3
     }
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
+  }
+}
+
+// The same on round keys given as a table: rk[2 r], rk[2 r + 1] = the key after r bumps. A
+// table in a kernel's parameters is read straight from the constant bank by the XORs.
+template <int N>
+__device__ __forceinline__ void philox_xn_rk(qjl::U32x4 (&c)[N], const uint32_t (&rk)[20]) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      uint32_t hA, lA, hB, lB;
+      qjl::mul_hi_lo(0xD2511F53u, c[j].x, hA, lA);
+      qjl::mul_hi_lo(0xCD9E8D57u, c[j].z, hB, lB);
+      c[j] = qjl::U32x4{hB ^ c[j].y ^ rk[2 * r], lB, hA ^ c[j].w ^ rk[2 * r + 1], lA};
+    }
+  }
+}
+
+// Philox round keys of the key (k0, k1) as the table philox_xn_rk reads.
+__host__ __device__ inline void philox_round_keys(uint32_t k0, uint32_t k1, uint32_t (&rk)[20]) {
+  for (int r = 0; r < 10; ++r) {
+    rk[2 * r] = k0 + (uint32_t)r * 0x9E3779B9u;
+    rk[2 * r + 1] = k1 + (uint32_t)r * 0xBB67AE85u;
   }
 }
 
