@@ -215,9 +215,13 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partial_kernel(
 
 // ---------------------------------------------------------------------------
 // Streaming fused decode for one query per group (the decode step proper).
-// Each CTA owns one split of one group. A producer lane moves 512-token
-// stages (bits, norms, codes, scales, zeros) into a shared-memory ring with
-// cp.async.bulk. Eight consumer warps take 64 tokens each per stage:
+// Each CTA owns one split of one group. A producer lane moves stages of 64
+// tokens per consumer warp (bits, norms, codes, scales, zeros) into a
+// shared-memory ring with cp.async.bulk. The consumer warps (12 at m = 256,
+// d <= 128, three per SM sub-partition, so that their latencies overlap;
+// 8 where 12 would spill, where two stages would not fit, and for the paged
+// cache, whose 256-token pages split 768-token stages into three copies per
+// array and measured slower) take 64 tokens each per stage:
 //   * estimates by the class-in-column s8 MMAs (one fragment per tile, two
 //     xor-shuffles merge the four weight classes; each lane ends with the
 //     logits of 2 tokens);
@@ -228,9 +232,12 @@ __global__ void __launch_bounds__(kWarps * 32) decode_partial_kernel(
 //     with no shift and no int-to-float conversion, and the 4^c is divided
 //     out once at the end.
 // The warps are merged in shared memory into one (max, sum, acc[d]) partial.
-constexpr int kDsConsumers = 8;
-constexpr int kDsThreads = (kDsConsumers + 1) * 32;
-constexpr int kDsStage = 512;
+template <int W, int CPL, bool PAGED>
+__host__ __device__ constexpr int ds_consumers() { return (W == 8 && CPL <= 4 && !PAGED) ? 12 : 8; }
+template <int W, int CPL, bool PAGED>
+__host__ __device__ constexpr int ds_threads() { return (ds_consumers<W, CPL, PAGED>() + 1) * 32; }
+template <int W, int CPL, bool PAGED>
+__host__ __device__ constexpr int ds_stage() { return ds_consumers<W, CPL, PAGED>() * 64; }
 
 __device__ __forceinline__ void mma_u8s8_acc(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                              uint32_t b0, uint32_t b1) {
@@ -291,14 +298,14 @@ struct DsLayout {
   uint32_t bits, norms, codes, scale, zero, bytes;
 };
 
-__host__ __device__ inline DsLayout ds_layout(int W, int d) {
+__host__ __device__ inline DsLayout ds_layout(int W, int d, int stage) {
   DsLayout L;
   L.bits = 0;
-  L.norms = L.bits + kDsStage * W * 4;
-  L.codes = L.norms + kDsStage * 4;
-  L.scale = L.codes + kDsStage * (d / 16) * 4;
-  L.zero = L.scale + kDsStage * (d / 32) * 2;
-  L.bytes = L.zero + kDsStage * (d / 32) * 2;
+  L.norms = L.bits + stage * W * 4;
+  L.codes = L.norms + stage * 4;
+  L.scale = L.codes + stage * (d / 16) * 4;
+  L.zero = L.scale + stage * (d / 32) * 2;
+  L.bytes = L.zero + stage * (d / 32) * 2;
   return L;
 }
 
@@ -342,13 +349,15 @@ __device__ __forceinline__ bool bulk_ok(const void* src, uint32_t bytes) {
 // segment, rounded up to 4 tokens (never past the page: pages hold a multiple
 // of 16 tokens, and segments start 16-token aligned).
 template <int W, int CPL, bool PAGED>
-__global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
+__global__ void __launch_bounds__(ds_threads<W, CPL, PAGED>(), 1) decode_stream_kernel(
     const uint32_t* __restrict__ bits, const float* __restrict__ norms, const uint32_t* __restrict__ codes,
     const uint16_t* __restrict__ scale, const uint16_t* __restrict__ zero, const float* __restrict__ sq, int64_t G,
     int64_t N, int NS, float est_scale, float logit_scale, float* __restrict__ ws, int* __restrict__ err,
     PagedRead pr) {
   using namespace qjl_sync;
   constexpr int d = 32 * CPL;
+  constexpr int kDsConsumers = ds_consumers<W, CPL, PAGED>();
+  constexpr int kDsStage = ds_stage<W, CPL, PAGED>();
   constexpr int CW = d / 16;  // code words per token
   constexpr int GW = d / 32;  // scale / zero halves per token
   constexpr int KT = 4;       // 16-token tiles per warp per stage
@@ -359,7 +368,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(
   uint2* Btab = reinterpret_cast<uint2*>(smem_raw + 3 * 64 * 4);
   float* s_red = reinterpret_cast<float*>(Btab + W * 32);                      // [kDsConsumers][d + 2]
   unsigned char* ring = reinterpret_cast<unsigned char*>(s_red + kDsConsumers * (d + 2));
-  const DsLayout L = ds_layout(W, d);
+  const DsLayout L = ds_layout(W, d, kDsStage);
   uint64_t* full = reinterpret_cast<uint64_t*>(ring + (size_t)NS * L.bytes);
   uint64_t* empty = full + NS;
 
@@ -719,8 +728,10 @@ qjl_status launch_stream(const qjl_projection* P, const uint32_t* bits, const fl
                          float softmax_scale, float* out, float* ws, cudaStream_t st,
                          const PagedRead& pr = PagedRead()) {
   constexpr int d = 32 * CPL;
-  const DsLayout L = ds_layout(W, d);
-  int NS = 4;  // one CTA per SM: about 168 KB in flight at d = 128, m = 256
+  constexpr int kDsConsumers = ds_consumers<W, CPL, PAGED>();
+  constexpr int kDsThreads = ds_threads<W, CPL, PAGED>();
+  const DsLayout L = ds_layout(W, d, ds_stage<W, CPL, PAGED>());
+  int NS = 4;  // one CTA per SM: three 768-token stages (194 KB) at d = 128, m = 256
   while (NS > 2 && 3 * 64 * 4 + (size_t)W * 32 * sizeof(uint2) + (size_t)kDsConsumers * (d + 2) * 4 +
                        (size_t)NS * L.bytes + (size_t)2 * NS * 8 > 220 * 1024)
     --NS;

@@ -202,7 +202,9 @@ def test_decode_paged_identity_table_equals_contiguous(cuda_ok):
     cache = qjl.PagedCache(T, table, seq, bits, norms, codes, sc, zr)
     got = qjl.decode_attention_paged(P, cache, sq, N, 0.1)
     torch.cuda.synchronize()
-    assert torch.equal(got, want.view(G, d))
+    # the contiguous kernel merges the partial sums of 12 consumer warps and the paged one of 8,
+    # so the two add in a different order: equal up to fp32 rounding
+    torch.testing.assert_close(got, want.view(G, d), rtol=1e-5, atol=2e-6)
 
 
 def test_bad_page_entries_are_skipped(cuda_ok):
