@@ -59,9 +59,14 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_hash(paths):
+    """sha256 prefix of a kernel's source file, or of several concatenated (the .cu and the headers
+    whose arithmetic it runs)."""
+    h = hashlib.sha256()
+    for path in ([paths] if isinstance(paths, str) else paths):
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel, workload, src):
@@ -69,7 +74,8 @@ def ncu_traffic(kernel, workload, src):
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    h = source_hash(os.path.join(ROOT, "bit_kv_cache_qjl_b200", "csrc", src))
+    srcs = [src] if isinstance(src, str) else list(src)
+    h = source_hash([os.path.join(ROOT, "bit_kv_cache_qjl_b200", "csrc", f) for f in srcs])
     for line in open(p):
         f = line.split()
         if len(f) >= 4 and not line.startswith("#") and f[0] == kernel and f[1] == workload and f[3] == h:
@@ -524,7 +530,7 @@ def build_workload(name, dev, qjl, wl, torch):
             # the first Hadamard factor runs as an exact +-1 contraction on tcgen05 (2 d m flops per
             # key), the second (D_g and d log2 d additions per block) on the FP32 lanes
             Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), n,
-                  2 * d + m // 8 + 4, 2 * d * m, "fqjl_tc_kernel", "fqjl_tc.cu", "tensor",
+                  2 * d + m // 8 + 4, 2 * d * m, "fqjl_tc_kernel", ("fqjl_tc.cu", "key_math.cuh"), "tensor",
                   alu_ops_per_unit=(m // d) * (d + d * int(math.log2(d)))),
             Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), J, 4 * d + 4 * m, bound="launch"),
             Stage("scores", lambda: qjl.scores(P, bits[:ns].view(1, ns, m // 32), norms[:ns].view(1, ns),
@@ -555,7 +561,7 @@ def build_workload(name, dev, qjl, wl, torch):
             # against the FP32 lane ceiling with the second factor's fp32 operations only (the
             # dither's Philox multiplies and Box-Muller are not fp32 adds or multiplies)
             Stage("quantize_keys", lambda: qjl.quantize_keys(P, keys, bits=bits, norms=norms), G * Nd,
-                  2 * D + m // 8 + 4, (m // D) * (D + D * int(math.log2(D))), "fqjl_tc_kernel", "fqjl_tc.cu", "alu"),
+                  2 * D + m // 8 + 4, (m // D) * (D + D * int(math.log2(D))), "fqjl_tc_kernel", ("fqjl_tc.cu", "key_math.cuh"), "alu"),
             Stage("quantize_values", lambda: qjl.quantize_values_2bit(vals, codes=codes, scale=sc, zero=zr), G * Nd,
                   2 * D + D // 4 + D // 8, 0, "values_2bit_kernel", "values.cu"),
             Stage("project_queries", lambda: qjl.project_queries(P, q, out=sq), G, 4 * D + 4 * m, bound="launch"),

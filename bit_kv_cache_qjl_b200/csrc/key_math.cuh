@@ -94,9 +94,9 @@ __device__ __forceinline__ float2 box_muller16(uint32_t x, float amp) {
   const float th = fmaf(hv, 804.247741699f, -804.247741699f);
   float l, rt, sn, cs;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(u));
-  const float t = -1.38629436f * l;  // -2 ln u > 0
-  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(rt) : "f"(t));
-  const float r = rt * amp;
+  // sqrt(-2 ln u) = sqrt(-log2 u) sqrt(2 ln 2); the negation can ride on the sqrt's operand
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(rt) : "f"(-l));
+  const float r = rt * (amp * 1.17741002f);
   asm("sin.approx.ftz.f32 %0, %1;" : "=f"(sn) : "f"(th));
   asm("cos.approx.ftz.f32 %0, %1;" : "=f"(cs) : "f"(th));
   return make_float2(r * cs, r * sn);
@@ -111,9 +111,8 @@ __device__ __forceinline__ void add_box_muller16(float2& acc, uint32_t x, float 
   const float th = fmaf(hv, 804.247741699f, -804.247741699f);
   float l, rt, sn, cs;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(u));
-  const float t = -1.38629436f * l;
-  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(rt) : "f"(t));
-  const float r = rt * amp;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(rt) : "f"(-l));
+  const float r = rt * (amp * 1.17741002f);
   asm("sin.approx.ftz.f32 %0, %1;" : "=f"(sn) : "f"(th));
   asm("cos.approx.ftz.f32 %0, %1;" : "=f"(cs) : "f"(th));
   asm("{\n\t.reg .b64 a, rr, cs;\n\t"
